@@ -1,0 +1,271 @@
+// CPU oracle for the FP8 blockwise linear layer -- TEST INFRASTRUCTURE ONLY.
+//
+// Only the tests, the smoke check and the bench's CPU-baseline leg may load
+// this library.  It shares no code, header, table or constant with the CUDA
+// path: every step is written out here from the pages' description, slowly
+// and plainly, so that a reader can check it against them by eye.
+//
+// Sources (web pages on the Puro-2B FP8 recipe):
+//   [EXPL]   "用 RTX 5090 花 $7000 训练 2B 大模型：Puro-2B 低成本预训练技术解析"
+//            (hankli.space), sections "Blackwell 的 FP8 Tensor Core" (the two
+//            FP8 formats), "核心挑战：Scale Factor 管理" (FP8Linear._quantize
+//            and forward) and "常见错误：直接转换而不加 Scale".
+//   [DIGEST] "Puro-2B: Poor Lab's Qwen2-1.5B Trained on RTX 5090 within $5090"
+//            (AI Papers Daily), sections "工作参考价值" bullet 2 and
+//            "方法关键点" bullet "FP8 blockwise 混合精度".
+//   [NEWS]   "小团队也能预训练！普罗2B：RTX5090训练成本不到5090美元" (66bd.net),
+//            paragraph on DeepSeek-V3-style fine-grained block quantisation.
+//
+// Readings where the pages leave a step open (each also listed in the design
+// notes): scale floor 1e-12 applied (R2); x/scale is a correctly rounded
+// fp32 division (R1); clamp to +-448 then round to nearest, ties to even
+// (R3, R4); the sign of zero is kept (R5); NaN/Inf inputs are outside the
+// contract (R6); every dimension is a multiple of 128 (R11); per-row scales
+// are stored block-major S[kb][row] and block scales row-major S[nb][kb]
+// (R12).
+//
+// Parity pins: every function here is pinned by tests/test_oracle_*.py
+// against the pages' constants, closed forms, invariants, torch's CPU
+// float8_e4m3fn cast (a library routine) and brute-force fp64 matmuls.
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+namespace {
+
+// ---------------------------------------------------------------- threading
+int oracle_threads() {
+  if (const char* e = std::getenv("ORACLE_THREADS")) {
+    int v = std::atoi(e);
+    if (v > 0) return v;
+  }
+  unsigned hc = std::thread::hardware_concurrency();
+  return hc ? static_cast<int>(hc) : 1;
+}
+
+// Runs fn(i) for i in [0, n) on a pool of std::threads (dynamic scheduling).
+template <class F>
+void parallel_for(int64_t n, F fn) {
+  int nt = static_cast<int>(std::min<int64_t>(oracle_threads(), std::max<int64_t>(n, 1)));
+  std::atomic<int64_t> next{0};
+  auto worker = [&]() {
+    for (int64_t i = next.fetch_add(1); i < n; i = next.fetch_add(1)) fn(i);
+  };
+  std::vector<std::thread> pool;
+  for (int t = 1; t < nt; ++t) pool.emplace_back(worker);
+  worker();
+  for (auto& th : pool) th.join();
+}
+
+// ---------------------------------------------------------------- bfloat16
+// bfloat16 is the upper half of an IEEE binary32, so widening is exact.
+float bf16_to_float(uint16_t b) {
+  uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+// ---------------------------------------------------------------- E4M3 codec
+// [EXPL] "Blackwell 的 FP8 Tensor Core": E4M3 (float8_e4m3fn) has 4 exponent
+// bits and 3 mantissa bits, and its largest value is 448.  With those widths
+// 448 = 1.75 * 2^8 forces exponent bias 7 and the "fn" encoding: the top
+// exponent field (15) still holds finite numbers and only mantissa 111 there
+// is NaN, so there is no infinity.  Byte layout: s eeee mmm.
+//   normal     (e = 1..15):  (-1)^s * 2^(e-7) * (1 + m/8)
+//   subnormal  (e = 0)    :  (-1)^s * 2^(-6) * (m/8)
+constexpr double kE4M3Max = 448.0;
+
+double e4m3_decode(uint8_t c) {
+  const int s = c >> 7, e = (c >> 3) & 0xF, m = c & 7;
+  if (e == 15 && m == 7) return std::nan("");
+  double mag = (e == 0) ? std::ldexp(m / 8.0, -6) : std::ldexp(1.0 + m / 8.0, e - 7);
+  return s ? -mag : mag;
+}
+
+// Round a non-negative double t to the nearest integer, ties to even.
+double round_half_even(double t) {
+  double f = std::floor(t);
+  double r = t - f;  // exact: t has at most 53 significant bits
+  if (r > 0.5) return f + 1.0;
+  if (r < 0.5) return f;
+  return (std::fmod(f, 2.0) == 0.0) ? f : f + 1.0;
+}
+
+// fp32 -> E4M3, round to nearest with ties to the even mantissa, sign kept
+// on zero results; magnitudes above 448 saturate to 448 (the quantiser clamps
+// before casting, so that branch only serves direct codec calls).
+uint8_t e4m3_encode(float v) {
+  const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+  const double a = std::fabs(static_cast<double>(v));  // exact
+  if (!(a <= kE4M3Max)) return sign | 0x7E;            // saturate (NaN is outside the contract)
+  // The representable magnitudes in [2^e, 2^(e+1)) are k * 2^(e-3), k = 8..15;
+  // below 2^-6 they are k * 2^-9, k = 0..7 (subnormals).
+  int e;
+  std::frexp(a, &e);  // a = f * 2^e, f in [0.5, 1)  =>  a in [2^(e-1), 2^e)
+  int exp2 = e - 1;   // a in [2^exp2, 2^(exp2+1)) for a > 0
+  if (a == 0.0 || exp2 < -6) {
+    // Subnormal grid, spacing 2^-9.  k = 8 lands on 2^-6, which is the first
+    // normal code 0x08, so the code is k itself in both cases.
+    double k = round_half_even(std::ldexp(a, 9));
+    return sign | static_cast<uint8_t>(k);
+  }
+  double k = round_half_even(std::ldexp(a, 3 - exp2));  // in [8, 16]
+  if (k == 16.0) {  // rounded up into the next binade
+    k = 8.0;
+    exp2 += 1;
+  }
+  int efield = exp2 + 7;
+  uint8_t code = static_cast<uint8_t>((efield << 3) | (static_cast<int>(k) - 8));
+  if (code > 0x7E) code = 0x7E;  // 480 and above would be NaN in the fn encoding
+  return sign | code;
+}
+
+// ---------------------------------------------------------------- one group
+// [EXPL] "核心挑战：Scale Factor 管理" (_quantize) and "常见错误：直接转换而不加
+// Scale": scale = amax / 448, floored at 1e-12; the value cast to E4M3 is
+// (x / scale) clamped to [-448, 448].  [DIGEST] "方法关键点": the amax is taken
+// over one block (1x128 for activations, 128x128 for weights), i.e. current
+// scaling of the block itself, with no history.
+constexpr float kScaleFloor = 1e-12f;  // fl32(1e-12) = 0x2B8CBCCC
+
+float group_scale(float amax) {
+  float s = amax / 448.0f;  // IEEE binary32 division, round to nearest even
+  return s < kScaleFloor ? kScaleFloor : s;
+}
+
+uint8_t quantize_value(float x, float s) {
+  float v = x / s;  // IEEE binary32 division
+  if (v > 448.0f) v = 448.0f;
+  if (v < -448.0f) v = -448.0f;
+  return e4m3_encode(v);
+}
+
+constexpr int64_t kBlock = 128;
+
+}  // namespace
+
+extern "C" {
+
+int orc_num_threads() { return oracle_threads(); }
+
+void orc_e4m3_encode(const float* v, int64_t n, uint8_t* out) {
+  const int64_t chunk = 1 << 20;
+  parallel_for((n + chunk - 1) / chunk, [&](int64_t c) {
+    int64_t lo = c * chunk, hi = std::min(n, lo + chunk);
+    for (int64_t i = lo; i < hi; ++i) out[i] = e4m3_encode(v[i]);
+  });
+}
+
+void orc_e4m3_decode(const uint8_t* c, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_decode(c[i]);
+}
+
+float orc_group_scale(float amax) { return group_scale(amax); }
+
+// Activations, 1x128 groups along the contiguous (feature) dimension.
+//   x [rows][cols] bf16  ->  q [rows][cols] E4M3,  s [cols/128][rows] fp32.
+void orc_quantize_act_rowwise(const uint16_t* x, int64_t rows, int64_t cols,
+                              uint8_t* q, float* s) {
+  const int64_t groups = cols / kBlock;
+  parallel_for(rows, [&](int64_t r) {
+    for (int64_t g = 0; g < groups; ++g) {
+      const uint16_t* xg = x + r * cols + g * kBlock;
+      float amax = 0.0f;
+      for (int64_t j = 0; j < kBlock; ++j) amax = std::max(amax, std::fabs(bf16_to_float(xg[j])));
+      const float sc = group_scale(amax);
+      s[g * rows + r] = sc;
+      for (int64_t j = 0; j < kBlock; ++j) q[r * cols + g * kBlock + j] = quantize_value(bf16_to_float(xg[j]), sc);
+    }
+  });
+}
+
+// Activations, 1x128 groups along the token (row) dimension, codes written
+// transposed so that tokens are contiguous:
+//   x [rows][cols] bf16  ->  qT [cols][rows] E4M3,  s [rows/128][cols] fp32.
+void orc_quantize_act_colwise_t(const uint16_t* x, int64_t rows, int64_t cols,
+                                uint8_t* qT, float* s) {
+  const int64_t groups = rows / kBlock;
+  parallel_for(cols, [&](int64_t c) {
+    for (int64_t g = 0; g < groups; ++g) {
+      float amax = 0.0f;
+      for (int64_t j = 0; j < kBlock; ++j)
+        amax = std::max(amax, std::fabs(bf16_to_float(x[(g * kBlock + j) * cols + c])));
+      const float sc = group_scale(amax);
+      s[g * cols + c] = sc;
+      for (int64_t j = 0; j < kBlock; ++j) {
+        const int64_t r = g * kBlock + j;
+        qT[c * rows + r] = quantize_value(bf16_to_float(x[r * cols + c]), sc);
+      }
+    }
+  });
+}
+
+// Weights, 128x128 blocks.  transposed = 0:  q [n][k], s [n/128][k/128];
+// transposed = 1:  q [k][n], s [k/128][n/128] (the same blocks, so the same
+// scales and codes, laid out as the operand of the data-gradient GEMM).
+void orc_quantize_weight(const uint16_t* w, int64_t n, int64_t k, int transposed,
+                         uint8_t* q, float* s) {
+  const int64_t nb = n / kBlock, kb = k / kBlock;
+  parallel_for(nb * kb, [&](int64_t blk) {
+    const int64_t bi = blk / kb, bj = blk % kb;
+    float amax = 0.0f;
+    for (int64_t i = 0; i < kBlock; ++i)
+      for (int64_t j = 0; j < kBlock; ++j)
+        amax = std::max(amax, std::fabs(bf16_to_float(w[(bi * kBlock + i) * k + bj * kBlock + j])));
+    const float sc = group_scale(amax);
+    if (transposed) s[bj * nb + bi] = sc; else s[bi * kb + bj] = sc;
+    for (int64_t i = 0; i < kBlock; ++i)
+      for (int64_t j = 0; j < kBlock; ++j) {
+        const int64_t r = bi * kBlock + i, c = bj * kBlock + j;
+        const uint8_t code = quantize_value(bf16_to_float(w[r * k + c]), sc);
+        if (transposed) q[c * n + r] = code; else q[r * k + c] = code;
+      }
+  });
+}
+
+// GEMM over dequantised operands, in fp64, not rounded:
+//   D[m][n] = sum_k (qa[m][k] * sa(m, k)) * (qb[n][k] * sb(n, k))
+// [EXPL] "核心挑战：Scale Factor 管理" (forward): the layer's result is
+// linear(x_fp8 * x_scale, w_fp8 * w_scale), i.e. the matmul of the
+// dequantised operands; [DIGEST] "方法关键点" puts the linear-layer GEMMs on
+// E4M3 with per-block scales.  Both operands are K-major (row-major [.][K]).
+//   sa(m, k) = sa[(k/128) * M + m]                           (per row, per K-block)
+//   layout 0/1 (forward, data gradient):  sb(n, k) = sb[(n/128) * (K/128) + k/128]
+//   layout 2   (weight gradient):         sb(n, k) = sb[(k/128) * N + n]
+// rows: indices of the output rows to compute (nullptr = all M rows);
+// d receives nrows x N values in that order.
+void orc_gemm(int layout, int64_t M, int64_t N, int64_t K,
+              const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb,
+              const int64_t* rows, int64_t nrows, double* d) {
+  const int64_t kblocks = K / kBlock;
+  if (!rows) nrows = M;
+  // Dequantised B, one row of K values per output column n.
+  std::vector<double> bdq(static_cast<size_t>(N) * K);
+  parallel_for(N, [&](int64_t n) {
+    for (int64_t k = 0; k < K; ++k) {
+      const double scale = (layout == 2) ? sb[(k / kBlock) * N + n]
+                                         : sb[(n / kBlock) * kblocks + k / kBlock];
+      bdq[n * K + k] = e4m3_decode(qb[n * K + k]) * scale;  // exact in fp64
+    }
+  });
+  parallel_for(nrows, [&](int64_t i) {
+    const int64_t m = rows ? rows[i] : i;
+    std::vector<double> adq(K);
+    for (int64_t k = 0; k < K; ++k) adq[k] = e4m3_decode(qa[m * K + k]) * sa[(k / kBlock) * M + m];
+    for (int64_t n = 0; n < N; ++n) {
+      const double* bn = &bdq[n * K];
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += adq[k] * bn[k];
+      d[i * N + n] = acc;
+    }
+  });
+}
+
+}  // extern "C"
