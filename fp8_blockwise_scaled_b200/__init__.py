@@ -1,0 +1,161 @@
+"""Python binding of libfp8blk: FP8 (E4M3) blockwise quantisation and GEMM on B200.
+
+Argument marshalling only.  Every step runs in the library's CUDA kernels;
+torch provides device memory and the current stream.  There is no CPU
+fallback: importing this package without the built library (and without
+nvcc to build it) raises, and every call on a non-CUDA tensor raises.
+
+The functions carry the C-ABI's names (include/fp8blk.h).  Output tensors
+may be passed in (they must be contiguous CUDA tensors of the right dtype
+and shape); missing ones are allocated with torch.empty.
+
+Layouts (row-major, dimensions multiples of 128):
+  fp8blk_quantize_act_1x128(x[R,C], mode)
+      ROWWISE   -> q_row[R,C] float8_e4m3fn, s_row[C/128,R] float32
+      COLWISE_T -> q_colT[C,R],              s_colT[R/128,C]
+      BOTH      -> all four
+  fp8blk_quantize_weight_128x128(w[N,K])   -> q[N,K],  s[N/128,K/128]
+  fp8blk_quantize_weight_128x128_t(w[N,K]) -> qT[K,N], sT[K/128,N/128]
+  fp8blk_gemm(layout, a[M,K], sa[K/128,M], b[N,K], sb) -> d[M,N] bfloat16
+      sb = [N/128,K/128] for FWD/DGRAD, [K/128,N] for WGRAD
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._lib import (BOTH, COLWISE_T, DGRAD, FWD, ROWWISE, WGRAD, Fp8BlkError, LIB_PATH, check,
+                   lib, status_string)
+
+__all__ = [
+    "fp8blk_quantize_act_1x128", "fp8blk_quantize_weight_128x128", "fp8blk_quantize_weight_128x128_t",
+    "fp8blk_gemm", "fp8blk_get_device_error", "fp8blk_version", "linear_forward", "linear_backward",
+    "ROWWISE", "COLWISE_T", "BOTH", "FWD", "DGRAD", "WGRAD", "Fp8BlkError", "LIB_PATH", "status_string",
+]
+
+E4M3 = torch.float8_e4m3fn
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream))
+
+
+def _need_cuda(*tensors):
+    for t in tensors:
+        if t is not None and not t.is_cuda:
+            raise ValueError("fp8blk runs on CUDA tensors only (no CPU fallback)")
+
+
+def _out(t, shape, dtype, device):
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"output must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+    return t
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _bf16_2d(x):
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("input must be a 2-D bfloat16 tensor with unit column stride")
+    return x
+
+
+def fp8blk_quantize_act_1x128(x, mode=ROWWISE, q_row=None, s_row=None, q_colT=None, s_colT=None,
+                              stream=None):
+    """Activation quantisation in 1x128 groups.  Returns (q_row, s_row, q_colT, s_colT); unused are None."""
+    x = _bf16_2d(x)
+    _need_cuda(x)
+    rows, cols = x.shape
+    dev = x.device
+    if mode & ROWWISE:
+        q_row = _out(q_row, (rows, cols), E4M3, dev)
+        s_row = _out(s_row, (cols // 128, rows), torch.float32, dev)
+    else:
+        q_row = s_row = None
+    if mode & COLWISE_T:
+        q_colT = _out(q_colT, (cols, rows), E4M3, dev)
+        s_colT = _out(s_colT, (rows // 128, cols), torch.float32, dev)
+    else:
+        q_colT = s_colT = None
+    check(lib.fp8blk_quantize_act_1x128(_ptr(x), rows, cols, x.stride(0), int(mode), _ptr(q_row), _ptr(s_row),
+                                        _ptr(q_colT), _ptr(s_colT), _stream_handle(stream)))
+    return q_row, s_row, q_colT, s_colT
+
+
+def fp8blk_quantize_weight_128x128(w, q=None, s=None, stream=None):
+    """Weight quantisation in 128x128 blocks.  Returns (q[N,K], s[N/128,K/128])."""
+    w = _bf16_2d(w)
+    _need_cuda(w)
+    n, k = w.shape
+    q = _out(q, (n, k), E4M3, w.device)
+    s = _out(s, (n // 128, k // 128), torch.float32, w.device)
+    check(lib.fp8blk_quantize_weight_128x128(_ptr(w), n, k, w.stride(0), _ptr(q), _ptr(s), _stream_handle(stream)))
+    return q, s
+
+
+def fp8blk_quantize_weight_128x128_t(w, qT=None, sT=None, stream=None):
+    """The same blocks written transposed.  Returns (qT[K,N], sT[K/128,N/128])."""
+    w = _bf16_2d(w)
+    _need_cuda(w)
+    n, k = w.shape
+    qT = _out(qT, (k, n), E4M3, w.device)
+    sT = _out(sT, (k // 128, n // 128), torch.float32, w.device)
+    check(lib.fp8blk_quantize_weight_128x128_t(_ptr(w), n, k, w.stride(0), _ptr(qT), _ptr(sT),
+                                               _stream_handle(stream)))
+    return qT, sT
+
+
+def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None):
+    """Blockwise-scaled E4M3 GEMM, D[M,N] = dequant(A) . dequant(B)^T in bf16."""
+    _need_cuda(a, sa, b, sb, d)
+    m, k = a.shape
+    n = b.shape[0]
+    if b.shape[1] != k:
+        raise ValueError("A and B disagree on K")
+    if a.dtype != E4M3 or b.dtype != E4M3:
+        raise ValueError("A and B must be float8_e4m3fn")
+    want_sb = (k // 128, n) if layout == WGRAD else (n // 128, k // 128)
+    if tuple(sa.shape) != (k // 128, m) or tuple(sb.shape) != want_sb:
+        raise ValueError(f"scale shapes {tuple(sa.shape)}, {tuple(sb.shape)} do not match layout {layout}")
+    if not (a.is_contiguous() and b.is_contiguous() and sa.is_contiguous() and sb.is_contiguous()):
+        raise ValueError("operands and scales must be contiguous")
+    if d is None:
+        d = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
+    elif d.dtype != torch.bfloat16 or d.dim() != 2 or d.stride(1) != 1 or tuple(d.shape) != (m, n):
+        raise ValueError("d must be a bfloat16 [M,N] tensor with unit column stride")
+    check(lib.fp8blk_gemm(int(layout), m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d), d.stride(0),
+                          _stream_handle(stream)))
+    return d
+
+
+def fp8blk_get_device_error(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error status code."""
+    return int(lib.fp8blk_get_device_error(_stream_handle(stream)))
+
+
+def fp8blk_version() -> int:
+    return int(lib.fp8blk_version())
+
+
+def linear_forward(x, w, stream=None):
+    """Y = X . W^T through the FP8 blockwise path: quantise X (1x128) and W (128x128), then GEMM."""
+    qx, sx, _, _ = fp8blk_quantize_act_1x128(x, ROWWISE, stream=stream)
+    qw, sw = fp8blk_quantize_weight_128x128(w, stream=stream)
+    return fp8blk_gemm(FWD, qx, sx, qw, sw, stream=stream)
+
+
+def linear_backward(x, w, dy, stream=None):
+    """(dX, dW) of Y = X . W^T: dX = dY . W (dgrad), dW = dY^T . X (wgrad), both FP8 blockwise."""
+    qdy, sdy, qdyT, sdyT = fp8blk_quantize_act_1x128(dy, BOTH, stream=stream)
+    qwT, swT = fp8blk_quantize_weight_128x128_t(w, stream=stream)
+    _, _, qxT, sxT = fp8blk_quantize_act_1x128(x, COLWISE_T, stream=stream)
+    dx = fp8blk_gemm(DGRAD, qdy, sdy, qwT, swT, stream=stream)
+    dw = fp8blk_gemm(WGRAD, qdyT, sdyT, qxT, sxT, stream=stream)
+    return dx, dw

@@ -1,0 +1,61 @@
+"""ctypes loader for libfp8blk.so: declares every C-ABI entry point of include/fp8blk.h."""
+from __future__ import annotations
+
+import ctypes
+import os
+import shutil
+
+from . import build as _build
+
+LIB_PATH = _build.LIB
+
+# fp8blk_act_mode / fp8blk_layout
+ROWWISE, COLWISE_T, BOTH = 1, 2, 3
+FWD, DGRAD, WGRAD = 0, 1, 2
+
+STATUS_NAMES = {
+    0: "FP8BLK_OK", 1: "FP8BLK_ERR_INVALID_ARG", 2: "FP8BLK_ERR_SHAPE", 3: "FP8BLK_ERR_ALIGN",
+    4: "FP8BLK_ERR_UNSUPPORTED_DEVICE", 5: "FP8BLK_ERR_LAUNCH", 6: "FP8BLK_ERR_TIMEOUT", 7: "FP8BLK_ERR_CUDA",
+}
+
+
+class Fp8BlkError(RuntimeError):
+    def __init__(self, status: int):
+        self.status = status
+        super().__init__(f"fp8blk call failed: {STATUS_NAMES.get(status, status)}")
+
+
+def _load() -> ctypes.CDLL:
+    if _build._stale():
+        if shutil.which(os.environ.get("NVCC", "nvcc")) is None:
+            raise RuntimeError(f"{LIB_PATH} is missing or out of date and nvcc is not available to build it; "
+                               "this package has no CPU fallback")
+        _build.build()
+    so = ctypes.CDLL(LIB_PATH)
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    sigs = {
+        "fp8blk_quantize_act_1x128": [P, I64, I64, I64, I, P, P, P, P, P],
+        "fp8blk_quantize_weight_128x128": [P, I64, I64, I64, P, P, P],
+        "fp8blk_quantize_weight_128x128_t": [P, I64, I64, I64, P, P, P],
+        "fp8blk_gemm": [I, I64, I64, I64, P, P, P, P, P, I64, P],
+        "fp8blk_get_device_error": [P],
+        "fp8blk_status_string": [I],
+        "fp8blk_version": [],
+    }
+    for name, args in sigs.items():
+        fn = getattr(so, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_char_p if name == "fp8blk_status_string" else ctypes.c_int
+    return so
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.fp8blk_status_string(int(status)).decode()
+
+
+def check(status: int) -> None:
+    if status != 0:
+        raise Fp8BlkError(status)

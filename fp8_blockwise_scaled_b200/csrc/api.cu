@@ -1,0 +1,195 @@
+// C-ABI entry points of libfp8blk (declared in include/fp8blk.h): argument
+// checks, device check, dispatch to the kernels on the caller's stream.
+#include <cstdlib>
+#include <cstring>
+
+#include "../../include/fp8blk.h"
+#include "device.cuh"
+#include "kernels.h"
+
+namespace fp8blk {
+// Bit 0 (kErrTimeoutBit): a bounded device-side wait expired.
+__device__ unsigned int g_error_word = 0;
+}
+
+namespace {
+
+// Device address of g_error_word on the current device (looked up once per device).
+unsigned int* error_word() {
+  static thread_local int dev_cached = -1;
+  static thread_local unsigned int* ptr = nullptr;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != dev_cached) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, fp8blk::g_error_word) != cudaSuccess) return nullptr;
+    ptr = static_cast<unsigned int*>(p);
+    dev_cached = dev;
+  }
+  return ptr;
+}
+
+using fp8blk::QuantArgs;
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool dim_ok(int64_t d) { return d > 0 && d % 128 == 0; }
+
+// The kernels use tcgen05 and TMA features of compute capability 10.0.
+fp8blk_status check_device() {
+  static thread_local int cached_dev = -1;
+  static thread_local fp8blk_status cached = FP8BLK_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FP8BLK_ERR_CUDA;
+  if (dev != cached_dev) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return FP8BLK_ERR_CUDA;
+    cached = (major == 10 && minor == 0) ? FP8BLK_OK : FP8BLK_ERR_UNSUPPORTED_DEVICE;
+    cached_dev = dev;
+  }
+  return cached;
+}
+
+uint64_t wait_timeout_ns() {
+  // Bound on every device-side wait; FP8BLK_WAIT_TIMEOUT_MS overrides the default of 4 s.
+  if (const char* e = std::getenv("FP8BLK_WAIT_TIMEOUT_MS")) {
+    long v = std::atol(e);
+    if (v > 0) return static_cast<uint64_t>(v) * 1000000ull;
+  }
+  return 4000000000ull;
+}
+
+fp8blk_status launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return FP8BLK_OK;
+  cudaGetLastError();  // clear a sticky launch error so that later calls are not blamed
+  return FP8BLK_ERR_LAUNCH;
+}
+
+fp8blk_status check_quant_common(const void* x, int64_t rows, int64_t cols, int64_t ld) {
+  if (!x) return FP8BLK_ERR_INVALID_ARG;
+  if (!dim_ok(rows) || !dim_ok(cols)) return FP8BLK_ERR_SHAPE;
+  if (ld < cols) return FP8BLK_ERR_INVALID_ARG;
+  if (!aligned16(x) || ld % 8 != 0) return FP8BLK_ERR_ALIGN;
+  return FP8BLK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8blk_status fp8blk_quantize_act_1x128(const void* x, int64_t rows, int64_t cols, int64_t ldx, int mode,
+                                        uint8_t* q_row, float* s_row, uint8_t* q_colT, float* s_colT,
+                                        void* stream) {
+  fp8blk_status st = check_quant_common(x, rows, cols, ldx);
+  if (st != FP8BLK_OK) return st;
+  if (mode != FP8BLK_ROWWISE && mode != FP8BLK_COLWISE_T && mode != FP8BLK_BOTH) return FP8BLK_ERR_INVALID_ARG;
+  int kmode = 0;
+  if (mode & FP8BLK_ROWWISE) {
+    if (!q_row || !s_row) return FP8BLK_ERR_INVALID_ARG;
+    if (!aligned16(q_row) || !aligned16(s_row)) return FP8BLK_ERR_ALIGN;
+    kmode |= fp8blk::Q_ROW;
+  }
+  if (mode & FP8BLK_COLWISE_T) {
+    if (!q_colT || !s_colT) return FP8BLK_ERR_INVALID_ARG;
+    if (!aligned16(q_colT) || !aligned16(s_colT)) return FP8BLK_ERR_ALIGN;
+    kmode |= fp8blk::Q_COLT;
+  }
+  if ((st = check_device()) != FP8BLK_OK) return st;
+  QuantArgs a{static_cast<const uint16_t*>(x), rows, cols, ldx, q_row, s_row, q_colT, s_colT, rows / 128,
+              cols / 128};
+  return launch_status(fp8blk::launch_quant(kmode, a, static_cast<cudaStream_t>(stream)));
+}
+
+static fp8blk_status quantize_weight(const void* w, int64_t n, int64_t k, int64_t ldw, uint8_t* q, float* s,
+                                     bool transposed, void* stream) {
+  fp8blk_status st = check_quant_common(w, n, k, ldw);
+  if (st != FP8BLK_OK) return st;
+  if (!q || !s) return FP8BLK_ERR_INVALID_ARG;
+  if (!aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u)) return FP8BLK_ERR_ALIGN;
+  if ((st = check_device()) != FP8BLK_OK) return st;
+  QuantArgs a{static_cast<const uint16_t*>(w), n, k, ldw, nullptr, nullptr, nullptr, nullptr, n / 128, k / 128};
+  int kmode;
+  if (transposed) {
+    a.q_t = q;
+    a.s_t = s;
+    kmode = fp8blk::Q_BLKT;
+  } else {
+    a.q_row = q;
+    a.s_row = s;
+    kmode = fp8blk::Q_BLK;
+  }
+  return launch_status(fp8blk::launch_quant(kmode, a, static_cast<cudaStream_t>(stream)));
+}
+
+fp8blk_status fp8blk_quantize_weight_128x128(const void* w, int64_t n, int64_t k, int64_t ldw, uint8_t* q,
+                                             float* s, void* stream) {
+  return quantize_weight(w, n, k, ldw, q, s, false, stream);
+}
+
+fp8blk_status fp8blk_quantize_weight_128x128_t(const void* w, int64_t n, int64_t k, int64_t ldw, uint8_t* qT,
+                                               float* sT, void* stream) {
+  return quantize_weight(w, n, k, ldw, qT, sT, true, stream);
+}
+
+fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uint8_t* a, const float* sa,
+                          const uint8_t* b, const float* sb, void* d, int64_t ldd, void* stream) {
+  if (layout != FP8BLK_FWD && layout != FP8BLK_DGRAD && layout != FP8BLK_WGRAD) return FP8BLK_ERR_INVALID_ARG;
+  if (!a || !sa || !b || !sb || !d) return FP8BLK_ERR_INVALID_ARG;
+  if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K)) return FP8BLK_ERR_SHAPE;
+  // One CTA row/column of tiles is addressed with 32-bit TMA coordinates.
+  if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return FP8BLK_ERR_SHAPE;
+  if (ldd < N) return FP8BLK_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(b) || !aligned16(d) || ldd % 8 != 0) return FP8BLK_ERR_ALIGN;
+  if (!aligned16(sa) || !aligned16(sb)) return FP8BLK_ERR_ALIGN;
+  fp8blk_status st = check_device();
+  if (st != FP8BLK_OK) return st;
+  fp8blk::GemmArgs g{};
+  g.layout = layout;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.a = a;
+  g.sa = sa;
+  g.b = b;
+  g.sb = sb;
+  g.d = static_cast<uint16_t*>(d);
+  g.ldd = ldd;
+  g.timeout_ns = wait_timeout_ns();
+  g.inject_stall = 0;
+  g.block_n = 0;
+  g.err = error_word();
+  if (!g.err) return FP8BLK_ERR_CUDA;
+  if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);
+  if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) g.inject_stall = std::atoi(e) != 0;
+  return launch_status(fp8blk::launch_gemm(g, static_cast<cudaStream_t>(stream)));
+}
+
+fp8blk_status fp8blk_get_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP8BLK_ERR_CUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, fp8blk::g_error_word, sizeof word) != cudaSuccess) return FP8BLK_ERR_CUDA;
+  if (word && cudaMemcpyToSymbol(fp8blk::g_error_word, &zero, sizeof zero) != cudaSuccess) return FP8BLK_ERR_CUDA;
+  return (word & fp8blk::kErrTimeoutBit) ? FP8BLK_ERR_TIMEOUT : FP8BLK_OK;
+}
+
+const char* fp8blk_status_string(fp8blk_status status) {
+  switch (status) {
+    case FP8BLK_OK: return "FP8BLK_OK";
+    case FP8BLK_ERR_INVALID_ARG: return "FP8BLK_ERR_INVALID_ARG";
+    case FP8BLK_ERR_SHAPE: return "FP8BLK_ERR_SHAPE";
+    case FP8BLK_ERR_ALIGN: return "FP8BLK_ERR_ALIGN";
+    case FP8BLK_ERR_UNSUPPORTED_DEVICE: return "FP8BLK_ERR_UNSUPPORTED_DEVICE";
+    case FP8BLK_ERR_LAUNCH: return "FP8BLK_ERR_LAUNCH";
+    case FP8BLK_ERR_TIMEOUT: return "FP8BLK_ERR_TIMEOUT";
+    case FP8BLK_ERR_CUDA: return "FP8BLK_ERR_CUDA";
+  }
+  return "FP8BLK_UNKNOWN_STATUS";
+}
+
+int fp8blk_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,410 @@
+// Blockwise-scaled E4M3 GEMM for sm_100a (tcgen05 + TMA + TMEM).
+//
+//   D[m][n] = bf16( sum_kb  sa(m,kb) * sb(n,kb) * P_kb[m][n] ),
+//   P_kb    = sum over the 128 k of K-block kb of a[m][k] * b[n][k]
+//
+// This is the matmul of the dequantised operands that the page "Puro-2B
+// 低成本预训练技术解析" (section "核心挑战：Scale Factor 管理", FP8Linear.forward)
+// defines, with the per-group / per-block scales of the Puro-2B digest
+// ("方法关键点", FP8 blockwise): the scales change every 128 values of K, so
+// the tensor cores produce one fp32 partial product per K-block and the
+// scales are applied to it before it joins the running sum.
+//
+// Design (one persistent CTA per SM, 320 threads, 128 x BN output tiles):
+//   warp 0      TMA producer: per K-block, a 128x128 A tile and a BNx128 B
+//               tile (E4M3, 128-byte swizzle) into a ring of shared-memory
+//               stages; completion counted in bytes on a "full" mbarrier.
+//   warp 1      TMEM owner and MMA issuer (one thread): 4 x tcgen05.mma
+//               kind::f8f6f4 (M=128, N=BN, K=32) per K-block into one of two
+//               TMEM accumulators (2 x BN fp32 columns), then tcgen05.commit
+//               to release the smem stage and to signal the accumulator.
+//   warps 2..9  promotion + epilogue: two warpgroups, each owning BN/2
+//               columns of the tile (a warp reads the 32 TMEM lanes given by
+//               its index mod 4); per K-block they read the partial product
+//               from TMEM and fold it into fp32 registers,
+//                   FWD/DGRAD: acc += P * (sa[m] * sb[n-block])
+//                   WGRAD    : acc += (P * sb[n]) * sa[m]
+//               then hand the TMEM buffer back; after the last K-block they
+//               round the tile to bf16 and store it.
+// The MMA of K-block kb+1 runs while the promotion of kb is in flight
+// (double-buffered TMEM), and TMA runs up to kStages K-blocks ahead.
+//
+// Every mbarrier wait is bounded (see mbar_wait_bounded): on a timeout the
+// CTA raises its abort flag, each role leaves its loop, the producer waits
+// for its TMA loads in flight, the issuer waits for its MMAs, and the TMEM
+// is freed before the CTA exits.  Decisions that a whole warp must take
+// together (tcgen05.ld is warp-collective) are made warp-uniform.
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "device.cuh"
+#include "kernels.h"
+
+namespace fp8blk {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 128;
+constexpr int kThreads = 320;
+constexpr int kEpiWarp0 = 2;
+constexpr int kEpiWarps = 8;
+
+template <int BN>
+struct Cfg {
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kABytes = BM * BK;
+  static constexpr int kBBytes = BN * BK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kHalf = BN / 2;  // columns per epilogue warpgroup
+};
+
+struct Ctrl {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t mma_done;
+  uint64_t never;         // completed by nothing: the stall test waits on it
+  uint32_t tmem_base;
+  int abort;
+  float sbuf[kEpiWarps][2][128];  // WGRAD: per-warp copy of this K-block's B scales for its columns
+};
+
+template <int BN>
+constexpr int smem_bytes() {
+  return 1024 + Cfg<BN>::kStages * Cfg<BN>::kStageBytes + static_cast<int>(sizeof(Ctrl));
+}
+
+struct GemmParams {
+  int64_t M, N, K;
+  const float* sa;
+  const float* sb;
+  uint16_t* d;
+  int64_t ldd;
+  uint64_t timeout_ns;
+  unsigned int* err;
+  int inject_stall;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// tcgen05.wait::ld, tied to the registers it makes valid so that the
+// compiler cannot read them before the wait.
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                 "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+}  // namespace
+
+template <int BN, bool kWgrad>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_blockwise_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                          const GemmParams p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + C::kStages * C::kStageBytes);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_mb = static_cast<int>(p.M / BM);
+  const int num_nb = static_cast<int>(p.N / BN);
+  const int kblocks = static_cast<int>(p.K / BK);
+  const int tiles = num_mb * num_nb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&ctrl->full[s], 1);
+      mbar_init(&ctrl->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctrl->tfull[b], 1);
+      mbar_init(&ctrl->tempty[b], kEpiWarps);
+    }
+    mbar_init(&ctrl->mma_done, 1);
+    mbar_init(&ctrl->never, 1);
+    ctrl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tm_a);
+    tma_prefetch_map(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctrl->tmem_base, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = ctrl->tmem_base;
+  volatile int* abort = &ctrl->abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+        const int mb = tile % num_mb, nb = tile / num_mb;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(&ctrl->empty[stage], phase ^ 1u, abort, p.timeout_ns, p.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa_tile = smem + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(&ctrl->full[stage], C::kStageBytes);
+          tma_load_2d(sa_tile, &tm_a, &ctrl->full[stage], kb * BK, mb * BM);
+          tma_load_2d(sa_tile + C::kABytes, &tm_b, &ctrl->full[stage], kb * BK, nb * BN);
+          ++issued;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      {
+        // Let the loads still in flight land before the CTA's smem goes away
+        // (on the normal path they have all been consumed: no wait).
+        const int64_t first = issued > C::kStages ? issued - C::kStages : 0;
+        for (int64_t j = first; j < issued; ++j)
+          mbar_wait_bounded(&ctrl->full[j % C::kStages], static_cast<uint32_t>((j / C::kStages) & 1), nullptr,
+                            p.timeout_ns, p.err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0, abuf = 0, aphase = 0;
+      bool ok = true;
+      if (p.inject_stall) ok = mbar_wait_bounded(&ctrl->never, 0, abort, p.timeout_ns, p.err);
+      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(&ctrl->full[stage], phase, abort, p.timeout_ns, p.err) ||
+              !mbar_wait_bounded(&ctrl->tempty[abuf], aphase ^ 1u, abort, p.timeout_ns, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_addr = smem_addr(smem + stage * C::kStageBytes);
+          const uint64_t adesc = smem_desc_kmajor_sw128(a_addr);
+          const uint64_t bdesc = smem_desc_kmajor_sw128(a_addr + C::kABytes);
+          const uint32_t d_tmem = tmem_base + abuf * BN;
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)  // 32 E4M3 values = 32 bytes = 2 x 16 B per step
+            umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+          umma_commit(&ctrl->empty[stage]);
+          umma_commit(&ctrl->tfull[abuf]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          abuf ^= 1u;
+          if (abuf == 0) aphase ^= 1u;
+        }
+      }
+      // Every MMA issued so far has finished once this arrives.
+      umma_commit(&ctrl->mma_done);
+      mbar_wait_bounded(&ctrl->mma_done, 0, nullptr, p.timeout_ns, p.err);
+    }
+  } else {
+    // ------------------------------------------------------------ promotion + epilogue
+    const int ew = warp - kEpiWarp0;  // 0..7
+    const int wg = ew >> 2;           // which half of the tile's columns
+    const int quarter = warp & 3;     // TMEM lanes this warp may read
+    const int row = quarter * 32 + lane;
+    const int col0 = wg * C::kHalf;
+    uint32_t abuf = 0, aphase = 0;
+    float acc[C::kHalf];
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+      const int mb = tile % num_mb, nb = tile / num_mb;
+      const int64_t m = static_cast<int64_t>(mb) * BM + row;
+      const int64_t ncol0 = static_cast<int64_t>(nb) * BN + col0;
+#pragma unroll
+      for (int j = 0; j < C::kHalf; ++j) acc[j] = 0.0f;
+
+      // Scales of the next K-block are fetched one step ahead.
+      float sa_next = __ldg(p.sa + m);
+      float sb_next = 0.0f;
+      float4 sbv_next = make_float4(0.f, 0.f, 0.f, 0.f);
+      if constexpr (kWgrad) {
+        if (lane < C::kHalf / 4) sbv_next = __ldg(reinterpret_cast<const float4*>(p.sb + ncol0) + lane);
+      } else {
+        sb_next = __ldg(p.sb + (ncol0 / 128) * kblocks);
+      }
+
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const float sa_cur = sa_next;
+        const float sb_cur = sb_next;
+        float* sbuf = ctrl->sbuf[ew][kb & 1];
+        if constexpr (kWgrad) {
+          if (lane < C::kHalf / 4) reinterpret_cast<float4*>(sbuf)[lane] = sbv_next;
+          __syncwarp();
+        }
+        if (kb + 1 < kblocks) {
+          sa_next = __ldg(p.sa + static_cast<int64_t>(kb + 1) * p.M + m);
+          if constexpr (kWgrad) {
+            if (lane < C::kHalf / 4)
+              sbv_next = __ldg(reinterpret_cast<const float4*>(p.sb + static_cast<int64_t>(kb + 1) * p.N + ncol0) + lane);
+          } else {
+            sb_next = __ldg(p.sb + (ncol0 / 128) * kblocks + kb + 1);
+          }
+        }
+        const bool got = mbar_wait_bounded(&ctrl->tfull[abuf], aphase, abort, p.timeout_ns, p.err);
+        if (!__all_sync(0xFFFFFFFFu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * BN + col0;
+        const float f = sa_cur * sb_cur;
+#pragma unroll
+        for (int c = 0; c < C::kHalf; c += 16) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(taddr + c, r);
+          tmem_wait_ld16(r);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if constexpr (kWgrad)
+              acc[c + j] = fmaf(__uint_as_float(r[j]) * sbuf[c + j], sa_cur, acc[c + j]);
+            else
+              acc[c + j] = fmaf(__uint_as_float(r[j]), f, acc[c + j]);
+          }
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->tempty[abuf]);
+        abuf ^= 1u;
+        if (abuf == 0) aphase ^= 1u;
+      }
+      if (!ok) break;
+      uint16_t* drow = p.d + m * p.ldd + ncol0;
+#pragma unroll
+      for (int j = 0; j < C::kHalf; j += 8) {
+        uint4 v;
+        v.x = pack_bf16x2(acc[j + 0], acc[j + 1]);
+        v.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
+        v.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
+        v.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
+        *reinterpret_cast<uint4*>(drow + j) = v;
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major [rows][cols] E4M3 matrix, box = box_rows x 128 bytes, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  auto encode = get_encode_fn();
+  if (!encode) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 1;
+  }
+  return sms;
+}
+
+template <int BN, bool kWgrad>
+cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
+  static bool attr_set = false;
+  constexpr int kSmem = smem_bytes<BN>();
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_blockwise_kernel<BN, kWgrad>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BN)) return cudaErrorInvalidValue;
+  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall};
+  const int64_t tiles = (g.M / BM) * (g.N / BN);
+  const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
+  gemm_blockwise_kernel<BN, kWgrad><<<grid, kThreads, kSmem, stream>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+// Wave efficiency of a tiling on this GPU: tiles / (ceil(tiles / SMs) * SMs).
+double wave_eff(int64_t tiles) {
+  const int64_t s = num_sms();
+  const int64_t waves = (tiles + s - 1) / s;
+  return static_cast<double>(tiles) / static_cast<double>(waves * s);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream) {
+  int bn = g.block_n;
+  if (bn == 0) {
+    bn = 128;
+    if (g.N % 256 == 0) {
+      const double e256 = wave_eff((g.M / BM) * (g.N / 256));
+      const double e128 = wave_eff((g.M / BM) * (g.N / 128));
+      bn = (e128 > e256 + 0.10) ? 128 : 256;
+    }
+  }
+  if (bn == 256 && g.N % 256 != 0) return cudaErrorInvalidValue;
+  const bool wgrad = g.layout == 2;
+  if (bn == 256) return wgrad ? launch_variant<256, true>(g, stream) : launch_variant<256, false>(g, stream);
+  if (bn == 128) return wgrad ? launch_variant<128, true>(g, stream) : launch_variant<128, false>(g, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fp8blk

@@ -1,0 +1,41 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fp8blk {
+
+// Which outputs a quantiser launch writes (may be OR-ed: ROW|COLT, BLK|BLKT).
+enum QuantMode : int { Q_ROW = 1, Q_COLT = 2, Q_BLK = 4, Q_BLKT = 8 };
+
+struct QuantArgs {
+  const uint16_t* x;  // [rows][ldx] bf16
+  int64_t rows, cols, ldx;
+  uint8_t* q_row;     // Q_ROW: [rows][cols];  Q_BLK: [rows][cols]
+  float* s_row;       // Q_ROW: [cols/128][rows];  Q_BLK: [rows/128][cols/128]
+  uint8_t* q_t;       // Q_COLT / Q_BLKT: [cols][rows]
+  float* s_t;         // Q_COLT: [rows/128][cols];  Q_BLKT: [cols/128][rows/128]
+  int64_t tiles_r, tiles_c;
+};
+
+cudaError_t launch_quant(int mode, const QuantArgs& a, cudaStream_t stream);
+
+struct GemmArgs {
+  int layout;                 // 0 FWD, 1 DGRAD, 2 WGRAD
+  int64_t M, N, K;
+  const uint8_t* a;           // [M][K]
+  const float* sa;            // [K/128][M]
+  const uint8_t* b;           // [N][K]
+  const float* sb;            // FWD/DGRAD [N/128][K/128];  WGRAD [K/128][N]
+  uint16_t* d;                // [M][ldd] bf16
+  int64_t ldd;
+  uint64_t timeout_ns;        // bound on every device-side wait
+  int inject_stall;           // test hook: the MMA issuer waits on a barrier nothing completes
+  int block_n;                // 0 = choose, else 128 or 256
+  unsigned int* err;          // device error word
+};
+
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream);
+
+}  // namespace fp8blk

@@ -1,0 +1,155 @@
+/*
+ * fp8blk -- FP8 (E4M3) blockwise-scaled quantisation and GEMM for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the Puro-2B FP8 recipe as described on these pages:
+ *   [EXPL]   "用 RTX 5090 花 $7000 训练 2B 大模型：Puro-2B 低成本预训练技术解析"
+ *            (hankli.space): section "Blackwell 的 FP8 Tensor Core" (E4M3 =
+ *            float8_e4m3fn, 4 exponent / 3 mantissa bits, max 448), section
+ *            "核心挑战：Scale Factor 管理" (scale = amax/448 floored at 1e-12,
+ *            codes = cast(clamp(x/scale, +-448)); the layer's output is the
+ *            matmul of the dequantised operands) and section "常见错误：直接转换
+ *            而不加 Scale" (the same scale rule without the floor).
+ *   [DIGEST] "Puro-2B: Poor Lab's Qwen2-1.5B Trained on RTX 5090 within $5090"
+ *            (AI Papers Daily): "工作参考价值" bullet 2 and "方法关键点" bullet
+ *            "FP8 blockwise 混合精度": activations in 1-D groups of 128,
+ *            weights in 128x128 blocks, linear-layer GEMMs in E4M3.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates, frees or keeps a pointer after the call returns.
+ *  - Matrices are row-major; "[R][C]" means C contiguous elements per row.
+ *    bf16 inputs are raw bfloat16 bit patterns (uint16).  E4M3 codes are
+ *    float8_e4m3fn bytes.  Scales are IEEE binary32.
+ *  - Every dimension must be a positive multiple of 128 (FP8BLK_ERR_SHAPE).
+ *    Pointers must be 16-byte aligned and leading dimensions must give
+ *    16-byte aligned rows (FP8BLK_ERR_ALIGN).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Work is enqueued asynchronously; argument errors are returned
+ *    before anything is enqueued; a launch failure returns FP8BLK_ERR_LAUNCH.
+ *  - Inputs must be finite; NaN or Inf in an input gives unspecified codes.
+ *  - The quantisers are exact: codes and scales equal, bit for bit,
+ *        s = max(fl32(amax / 448), fl32(1e-12))
+ *        q = E4M3_round_nearest_even(clamp(fl32(x / s), -448, 448))
+ *    with amax the largest |x| of the group and x / s a correctly rounded
+ *    binary32 division.  The sign of zero is kept (-0 -> 0x80).
+ *  - Device-side waits are bounded in time.  A wait that expires makes the
+ *    kernel stop early, leaving its outputs unspecified, and records
+ *    FP8BLK_ERR_TIMEOUT in a device error word read by
+ *    fp8blk_get_device_error().
+ */
+#ifndef FP8BLK_H
+#define FP8BLK_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FP8BLK_OK = 0,
+  FP8BLK_ERR_INVALID_ARG = 1,        /* NULL pointer where one is required, bad mode/layout, ld too small */
+  FP8BLK_ERR_SHAPE = 2,              /* a dimension <= 0 or not a multiple of 128 */
+  FP8BLK_ERR_ALIGN = 3,              /* a pointer or row stride not 16-byte aligned */
+  FP8BLK_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0 (B200, sm_100a) */
+  FP8BLK_ERR_LAUNCH = 5,             /* the CUDA launch (or a CUDA call it needs) failed */
+  FP8BLK_ERR_TIMEOUT = 6,            /* a bounded device-side wait expired (reported by fp8blk_get_device_error) */
+  FP8BLK_ERR_CUDA = 7                /* a CUDA runtime call outside a launch failed */
+} fp8blk_status;
+
+typedef enum {
+  FP8BLK_ROWWISE = 1,   /* 1x128 groups along the contiguous (feature) dimension */
+  FP8BLK_COLWISE_T = 2, /* 1x128 groups along rows (tokens); codes written transposed */
+  FP8BLK_BOTH = 3       /* both of the above from one read of the input */
+} fp8blk_act_mode;
+
+typedef enum {
+  FP8BLK_FWD = 0,   /* B scales per 128x128 block: sb[N/128][K/128] */
+  FP8BLK_DGRAD = 1, /* same operand format as FWD (B = transposed weight) */
+  FP8BLK_WGRAD = 2  /* B scales per row and K-block: sb[K/128][N] */
+} fp8blk_layout;
+
+/*
+ * Activation quantisation, 1x128 groups ([DIGEST] "激活 1D 128"; scale and
+ * cast rule from [EXPL] "核心挑战：Scale Factor 管理").
+ *
+ *   x      [rows][ldx] bf16, the first `cols` columns of each row are used.
+ *   mode   FP8BLK_ROWWISE, FP8BLK_COLWISE_T or FP8BLK_BOTH.
+ *   ROWWISE outputs (required for ROWWISE and BOTH, else ignored):
+ *     q_row  [rows][cols] E4M3 codes, group = 128 consecutive columns of a row
+ *     s_row  [cols/128][rows] fp32, s_row[g][r] = scale of row r, group g
+ *   COLWISE_T outputs (required for COLWISE_T and BOTH, else ignored):
+ *     q_colT [cols][rows] E4M3 codes = the codes of x^T, group = 128
+ *            consecutive rows (tokens) of one column
+ *     s_colT [rows/128][cols] fp32, s_colT[g][c] = scale of column c, group g
+ *   The forward and data-gradient GEMMs take (q_row, s_row) as operand A;
+ *   the weight-gradient GEMM takes (q_colT, s_colT) of the output gradient as
+ *   A and of the layer input as B.
+ */
+fp8blk_status fp8blk_quantize_act_1x128(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                                        int mode, uint8_t* q_row, float* s_row,
+                                        uint8_t* q_colT, float* s_colT, void* stream);
+
+/*
+ * Weight quantisation, 128x128 blocks ([DIGEST] "权重 2D 128x128").
+ *   w  [n][ldw] bf16 (first k columns used)  ->  q [n][k] E4M3,  s [n/128][k/128] fp32.
+ * The forward GEMM takes (q, s) as operand B.
+ */
+fp8blk_status fp8blk_quantize_weight_128x128(const void* w, int64_t n, int64_t k, int64_t ldw,
+                                             uint8_t* q, float* s, void* stream);
+
+/*
+ * The same 128x128 blocks (so the same scales and codes), written transposed:
+ *   w  [n][ldw] bf16  ->  qT [k][n] E4M3,  sT [k/128][n/128] fp32.
+ * qT[j][i] == q[i][j] and sT[b][a] == s[a][b] for the outputs of
+ * fp8blk_quantize_weight_128x128.  The data-gradient GEMM
+ * dX = dY . W takes (qT, sT) as operand B.
+ */
+fp8blk_status fp8blk_quantize_weight_128x128_t(const void* w, int64_t n, int64_t k, int64_t ldw,
+                                               uint8_t* qT, float* sT, void* stream);
+
+/*
+ * Blockwise-scaled FP8 GEMM with bf16 output ([EXPL] "核心挑战：Scale Factor
+ * 管理": the output is linear(x_fp8 * x_scale, w_fp8 * w_scale); [DIGEST]
+ * "方法关键点": the linear-layer GEMMs run in E4M3):
+ *
+ *   D[m][n] = bf16( sum over K-blocks kb of  sa(m,kb) * sb(n,kb) * P_kb[m][n] ),
+ *   P_kb[m][n] = sum_{k in kb} a[m][k] * b[n][k]   (fp32 accumulation on the tensor cores)
+ *
+ *   a   [M][K] E4M3 codes (K contiguous),  sa [K/128][M] fp32 (per row, per K-block)
+ *   b   [N][K] E4M3 codes (K contiguous)
+ *   sb  FWD / DGRAD: [N/128][K/128] fp32 (per 128x128 block)
+ *       WGRAD      : [K/128][N] fp32     (per row of b, per K-block)
+ *   d   [M][ldd] bf16 output, ldd >= N, ldd % 8 == 0.
+ *
+ * Operands per pass of a linear layer Y = X . W^T (X [T][in], W [out][in]):
+ *   FWD   : a = X rowwise,      b = W (128x128),           d = Y  [T][out]
+ *   DGRAD : a = dY rowwise,     b = W transposed (128x128), d = dX [T][in]
+ *   WGRAD : a = dY colwise_T,   b = X colwise_T,            d = dW [out][in]
+ * The result is accumulated in fp32 and rounded once to bf16; it is not
+ * bitwise reproducible against another summation order.
+ */
+fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K,
+                          const uint8_t* a, const float* sa, const uint8_t* b, const float* sb,
+                          void* d, int64_t ldd, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  Returns FP8BLK_OK, FP8BLK_ERR_TIMEOUT if a kernel's
+ * bounded wait expired since the last call, or FP8BLK_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+fp8blk_status fp8blk_get_device_error(void* stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* fp8blk_status_string(fp8blk_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int fp8blk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8BLK_H */

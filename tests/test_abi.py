@@ -1,0 +1,108 @@
+"""The C-ABI library: it loads, exports every symbol the header declares, and
+rejects bad arguments on the host before any device work (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp8_blockwise_scaled_b200 as fb
+from fp8_blockwise_scaled_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8blk.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8blk_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("fp8blk_quantize_act_1x128", "fp8blk_quantize_weight_128x128",
+                 "fp8blk_quantize_weight_128x128_t", "fp8blk_gemm", "fp8blk_get_device_error",
+                 "fp8blk_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    so = ctypes.CDLL(fb.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(so, n)]
+    assert not missing, f"declared but not exported: {missing}"
+
+
+def test_binding_covers_every_declared_symbol():
+    exported = set(dir(fb)) | {"fp8blk_status_string"}
+    for n in declared_functions():
+        assert n in exported or n == "fp8blk_status_string"
+
+
+def test_status_strings_and_version():
+    for code, name in _lib.STATUS_NAMES.items():
+        assert fb.status_string(code) == name
+    assert fb.status_string(99) == "FP8BLK_UNKNOWN_STATUS"
+    assert fb.fp8blk_version() == 10000
+
+
+P = ctypes.c_void_p
+ALIGNED = P(0x10000)      # never dereferenced: every case below fails validation first
+MISALIGNED = P(0x10008)
+NULL = P(0)
+S = NULL                  # stream
+
+
+@pytest.mark.parametrize("args,code", [
+    ((ALIGNED, 128, 100, 128, 1, ALIGNED, ALIGNED, NULL, NULL, S), 2),      # cols % 128
+    ((ALIGNED, 0, 128, 128, 1, ALIGNED, ALIGNED, NULL, NULL, S), 2),        # rows <= 0
+    ((NULL, 128, 128, 128, 1, ALIGNED, ALIGNED, NULL, NULL, S), 1),         # null input
+    ((ALIGNED, 128, 128, 64, 1, ALIGNED, ALIGNED, NULL, NULL, S), 1),       # ldx < cols
+    ((ALIGNED, 128, 128, 132, 1, ALIGNED, ALIGNED, NULL, NULL, S), 3),      # row stride not 16-B
+    ((MISALIGNED, 128, 128, 128, 1, ALIGNED, ALIGNED, NULL, NULL, S), 3),   # input pointer
+    ((ALIGNED, 128, 128, 128, 4, ALIGNED, ALIGNED, NULL, NULL, S), 1),      # bad mode
+    ((ALIGNED, 128, 128, 128, 1, NULL, ALIGNED, NULL, NULL, S), 1),         # missing q_row
+    ((ALIGNED, 128, 128, 128, 2, ALIGNED, ALIGNED, NULL, NULL, S), 1),      # missing q_colT
+    ((ALIGNED, 128, 128, 128, 3, ALIGNED, ALIGNED, MISALIGNED, ALIGNED, S), 3),
+])
+def test_quantize_act_argument_errors(args, code):
+    assert _lib.lib.fp8blk_quantize_act_1x128(*args) == code
+
+
+@pytest.mark.parametrize("fn", ["fp8blk_quantize_weight_128x128", "fp8blk_quantize_weight_128x128_t"])
+def test_quantize_weight_argument_errors(fn):
+    f = getattr(_lib.lib, fn)
+    assert f(ALIGNED, 128, 200, 256, ALIGNED, ALIGNED, S) == 2
+    assert f(NULL, 128, 128, 128, ALIGNED, ALIGNED, S) == 1
+    assert f(ALIGNED, 128, 128, 128, NULL, ALIGNED, S) == 1
+    assert f(ALIGNED, 128, 128, 128, MISALIGNED, ALIGNED, S) == 3
+
+
+@pytest.mark.parametrize("args,code", [
+    ((3, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 1),   # bad layout
+    ((0, 100, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 2),
+    ((0, 128, 128, 96, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 2),
+    ((0, 128, 128, 128, NULL, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 1),
+    ((2, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, NULL, ALIGNED, 128, S), 1),
+    ((0, 128, 256, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 1),   # ldd < N
+    ((0, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 132, S), 3),   # ldd % 8
+    ((0, 128, 128, 128, MISALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 3),
+    ((1, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, MISALIGNED, 128, S), 3),
+])
+def test_gemm_argument_errors(args, code):
+    assert _lib.lib.fp8blk_gemm(*args) == code
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(128, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fb.fp8blk_quantize_act_1x128(x)
+    with pytest.raises(ValueError):
+        fb.fp8blk_quantize_weight_128x128(x)
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-GPU host path")
+def test_valid_call_without_a_gpu_reports_a_cuda_error():
+    st = _lib.lib.fp8blk_quantize_act_1x128(ALIGNED, 128, 128, 128, 1, ALIGNED, ALIGNED, NULL, NULL, S)
+    assert st in (4, 7)
