@@ -37,6 +37,8 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <cstddef>
+
 #include "device.cuh"
 #include "kernels.h"
 
@@ -69,8 +71,9 @@ struct Ctrl {
   uint64_t never;         // completed by nothing: the stall test waits on it
   uint32_t tmem_base;
   int abort;
-  float sbuf[kEpiWarps][2][128];  // WGRAD: per-warp copy of this K-block's B scales for its columns
+  alignas(16) float sbuf[kEpiWarps][2][128];  // WGRAD: per-warp copy of this K-block's B scales (float4 access)
 };
+static_assert(offsetof(Ctrl, sbuf) % 16 == 0, "sbuf is written with 16-byte vector stores");
 
 template <int BN>
 constexpr int smem_bytes() {
