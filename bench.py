@@ -1,0 +1,489 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 blockwise linear-layer hot path on B200.
+
+One step = the four linear GEMMs of a Qwen2-1.5B-shaped decoder layer (QKV
+2048x1536, O 1536x1536, gate+up 17920x1536, down 1536x8960), each run
+forward, data-gradient and weight-gradient at 16384 tokens per GPU, with
+every quantisation the pass needs inside the step (28 kernels):
+
+    per linear layer (X [T,K], W [N,K], dY [T,N]):
+      quantize_act_1x128(X, BOTH)          row-wise for FWD, along tokens for WGRAD
+      quantize_weight_128x128(W)           FWD operand
+      quantize_weight_128x128_t(W)         DGRAD operand
+      gemm FWD    Y  = X . W^T
+      quantize_act_1x128(dY, BOTH)
+      gemm DGRAD  dX = dY . W
+      gemm WGRAD  dW = dY^T . X
+
+value = GEMM FLOPs of all ranks / device time of the step (quantisation included),
+in TFLOP/s.  With --gpus N > 1 every rank runs its own 16384-token batch
+(weak scaling) and the weight gradients are summed over ranks with NCCL
+all-reduce inside the step (the data-parallel exchange).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload layer|qkv_fwd|mlp_fwd|down_bwd] [--tokens T] [--sweep]
+
+`--impl reference` times the CPU oracle (the slow, plain implementation the
+parity tests check against) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "blockwise-FP8 GEMM TFLOP/s incl. quantize (fraction of dense FP8 peak); quant GB/s"
+SPEC_FP8_TFLOPS = 4500.0          # B200 dense FP8, NVIDIA's published figure
+FP8_PER_BF16 = 2.0                # nominal dense FP8 / BF16 tensor throughput ratio
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+WORKLOAD_DESC = {
+    "layer": "qwen2-1.5b-shaped decoder layer linears (qkv 2048x1536, o 1536x1536, gate_up 17920x1536, "
+             "down 1536x8960), fwd+dgrad+wgrad, all quantisation included",
+    "qkv_fwd": "qkv projection fwd, X[Tx1536] with 0.1% outlier channels x20, W[2048x1536]",
+    "mlp_fwd": "mlp fwd: gate_up X[Tx1536].W[17920x1536]^T then down X[Tx8960].W[1536x8960]^T",
+    "down_bwd": "mlp down backward: dgrad dX=dY.W, wgrad dW=dY^T.X, dY[Tx1536], X[Tx8960]",
+}
+
+
+def load_peaks() -> tuple[dict, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- workload programs
+def workload_tensors(name: str, tokens: int) -> list[dict]:
+    """[{name, X, W, dY, passes}] with bf16 host arrays; passes in {"fwd", "dgrad", "wgrad"}."""
+    if name == "layer":
+        L = workloads.layer(seed=4, tokens=tokens)
+        return [{"name": g, **L[g], "passes": ("fwd", "dgrad", "wgrad")} for g, _, _ in workloads.LAYER_GEMMS]
+    if name == "qkv_fwd":
+        d = workloads.qkv_fwd(seed=1, tokens=tokens)
+        return [{"name": "qkv", "X": d["X"], "W": d["W"], "dY": None, "passes": ("fwd",)}]
+    if name == "mlp_fwd":
+        d = workloads.mlp_fwd(seed=2, tokens=tokens)
+        return [{"name": "gate_up", "X": d["X_gate_up"], "W": d["W_gate_up"], "dY": None, "passes": ("fwd",)},
+                {"name": "down", "X": d["X_down"], "W": d["W_down"], "dY": None, "passes": ("fwd",)}]
+    if name == "down_bwd":
+        d = workloads.down_bwd(seed=3, tokens=tokens)
+        return [{"name": "down", "X": d["X"], "W": d["W"], "dY": d["dY"], "passes": ("dgrad", "wgrad")}]
+    raise ValueError(name)
+
+
+class Program:
+    """Device buffers and the ordered kernel launches of one step."""
+
+    def __init__(self, specs, device, world):
+        import torch
+        import fp8_blockwise_scaled_b200 as fb
+        self.fb, self.torch, self.world = fb, torch, world
+        self.ops = []          # (label, kind, units, fn); kind "quant" (units = bytes) or "gemm" (units = flops)
+        self.inputs = []       # (device tensor, host array) copied in by the end-to-end run
+        self.outputs = []      # device tensors read back by the end-to-end run
+        self.grads = []        # weight gradients all-reduced across ranks
+        self.gemm_flops = 0
+        E4 = torch.float8_e4m3fn
+        for sp in specs:
+            x = self._dev(sp["X"], device)
+            w = self._dev(sp["W"], device)
+            T, K = x.shape
+            N = w.shape[0]
+            passes = sp["passes"]
+            need_row_x = "fwd" in passes
+            need_colt_x = "wgrad" in passes
+            g = sp["name"]
+            f = lambda *s, dt=E4: torch.empty(s, dtype=dt, device=device)  # noqa: E731
+            qx = f(T, K) if need_row_x else None
+            sx = f(K // 128, T, dt=torch.float32) if need_row_x else None
+            qxT = f(K, T) if need_colt_x else None
+            sxT = f(T // 128, K, dt=torch.float32) if need_colt_x else None
+            mode = (fb.ROWWISE if need_row_x else 0) | (fb.COLWISE_T if need_colt_x else 0)
+            qbytes = T * K * (2 + (1 + 4 / 128) * (int(need_row_x) + int(need_colt_x)))
+            self._op(f"{g}.quant_x", "quant", qbytes,
+                     lambda x=x, m=mode, a=qx, b=sx, c=qxT, d=sxT: fb.fp8blk_quantize_act_1x128(x, m, a, b, c, d))
+            if "fwd" in passes:
+                qw, sw = f(N, K), f(N // 128, K // 128, dt=torch.float32)
+                self._op(f"{g}.quant_w", "quant", N * K * (3 + 4 / 16384),
+                         lambda w=w, q=qw, s=sw: fb.fp8blk_quantize_weight_128x128(w, q, s))
+            if "dgrad" in passes:
+                qwT, swT = f(K, N), f(K // 128, N // 128, dt=torch.float32)
+                self._op(f"{g}.quant_wt", "quant", N * K * (3 + 4 / 16384),
+                         lambda w=w, q=qwT, s=swT: fb.fp8blk_quantize_weight_128x128_t(w, q, s))
+            if "fwd" in passes:
+                y = torch.empty(T, N, dtype=torch.bfloat16, device=device)
+                self._op(f"{g}.gemm_fwd", "gemm", 2 * T * N * K,
+                         lambda a=qx, sa=sx, b=qw, sb=sw, d=y: fb.fp8blk_gemm(fb.FWD, a, sa, b, sb, d))
+                self.outputs.append(y)
+            if "dgrad" in passes or "wgrad" in passes:
+                dy = self._dev(sp["dY"], device)
+                need_row_d = "dgrad" in passes
+                need_colt_d = "wgrad" in passes
+                qd = f(T, N) if need_row_d else None
+                sd = f(N // 128, T, dt=torch.float32) if need_row_d else None
+                qdT = f(N, T) if need_colt_d else None
+                sdT = f(T // 128, N, dt=torch.float32) if need_colt_d else None
+                mode_d = (fb.ROWWISE if need_row_d else 0) | (fb.COLWISE_T if need_colt_d else 0)
+                self._op(f"{g}.quant_dy", "quant", T * N * (2 + (1 + 4 / 128) * (int(need_row_d) + int(need_colt_d))),
+                         lambda x=dy, m=mode_d, a=qd, b=sd, c=qdT, d=sdT:
+                         fb.fp8blk_quantize_act_1x128(x, m, a, b, c, d))
+                if need_row_d:
+                    dx = torch.empty(T, K, dtype=torch.bfloat16, device=device)
+                    self._op(f"{g}.gemm_dgrad", "gemm", 2 * T * N * K,
+                             lambda a=qd, sa=sd, b=qwT, sb=swT, d=dx: fb.fp8blk_gemm(fb.DGRAD, a, sa, b, sb, d))
+                    self.outputs.append(dx)
+                if need_colt_d:
+                    dw = torch.empty(N, K, dtype=torch.bfloat16, device=device)
+                    self._op(f"{g}.gemm_wgrad", "gemm", 2 * T * N * K,
+                             lambda a=qdT, sa=sdT, b=qxT, sb=sxT, d=dw: fb.fp8blk_gemm(fb.WGRAD, a, sa, b, sb, d))
+                    self.outputs.append(dw)
+                    self.grads.append(dw)
+        self.gemm_flops = sum(u for _, k, u, _ in self.ops if k == "gemm")
+        self.quant_bytes = sum(u for _, k, u, _ in self.ops if k == "quant")
+
+    def _dev(self, host, device):
+        t = self.torch.from_numpy(np.ascontiguousarray(host)).view(self.torch.bfloat16).to(device)
+        self.inputs.append((t, host))
+        return t
+
+    def _op(self, label, kind, units, fn):
+        self.ops.append((label, kind, units, fn))
+
+    def run(self, events=None):
+        """One step.  events: list of (start, end) CUDA event pairs, one per op, or None."""
+        for i, (_, _, _, fn) in enumerate(self.ops):
+            if events is not None:
+                events[i][0].record()
+            fn()
+            if events is not None:
+                events[i][1].record()
+        if self.world > 1:
+            import torch.distributed as dist
+            for g in self.grads:
+                dist.all_reduce(g)
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_gpu{gpu_index}.csv")
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 10:
+                    rows.append(parts)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        loaded = [r for r in rows if _num(r[4]) is not None and _num(r[4]) >= 50] or rows
+        sm = [_num(r[1]) for r in loaded if _num(r[1]) is not None]
+        reasons = sorted({names[i] for r in loaded for i in range(4) if r[6 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": _num(rows[0][2]) if rows else None,
+                "reasons": reasons, "samples": len(loaded),
+                "power_w_max": max((_num(r[3]) or 0.0) for r in loaded) if loaded else None}
+
+
+def _num(s):
+    try:
+        return float(s)
+    except (TypeError, ValueError):
+        return None
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def oracle_pass(specs, tokens: int, col_frac: float = 1.0) -> tuple[float, float, str]:
+    """Runs the oracle over the first `tokens` tokens (and a fraction of each weight's rows)
+    of every GEMM of the workload.  Returns (flops, seconds, description)."""
+    import oracle
+    flops = 0
+    t0 = time.perf_counter()
+    for sp in specs:
+        n_all = sp["W"].shape[0]
+        n = max(128, int(n_all * col_frac) // 128 * 128)
+        x = sp["X"][:tokens]
+        w = sp["W"][:n]
+        k = x.shape[1]
+        passes = sp["passes"]
+        if "fwd" in passes:
+            qx, sx = oracle.quantize_act_rowwise(x)
+            qw, sw = oracle.quantize_weight(w)
+            oracle.gemm(oracle.FWD, qx, sx, qw, sw)
+            flops += 2 * tokens * n * k
+        if "dgrad" in passes or "wgrad" in passes:
+            dy = np.ascontiguousarray(sp["dY"][:tokens, :n])
+            if "dgrad" in passes:
+                qd, sd = oracle.quantize_act_rowwise(dy)
+                qwt, swt = oracle.quantize_weight_t(w)
+                oracle.gemm(oracle.DGRAD, qd, sd, qwt, swt)
+                flops += 2 * tokens * n * k
+            if "wgrad" in passes:
+                qdt, sdt = oracle.quantize_act_colwise_t(dy)
+                qxt, sxt = oracle.quantize_act_colwise_t(x)
+                oracle.gemm(oracle.WGRAD, qdt, sdt, qxt, sxt)
+                flops += 2 * tokens * n * k
+    dt = time.perf_counter() - t0
+    desc = (f"first {tokens} tokens of every GEMM of the workload"
+            + (f", first {col_frac:.0%} of each weight's output rows" if col_frac < 1 else "")
+            + ", quantisation + fp64 GEMM, all passes")
+    return flops, dt, desc
+
+
+def cpu_baseline(specs) -> dict:
+    import oracle
+    flops, dt, desc = oracle_pass(specs, tokens=256)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": desc, "seconds": round(dt, 3)}
+
+
+# --------------------------------------------------------------------------- arms
+def run_reference(args, rank: int, world: int):
+    """The oracle, as it stands, on the host cores: each step a bounded sample of the workload."""
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    tokens = args.tokens or (16384 if args.workload == "layer" else 8192)
+    specs = workload_tensors(args.workload, 256)
+    budget = 150.0 / max(1, args.steps + args.warmup)       # seconds per step
+    _, t_full, _ = oracle_pass(specs, tokens=128)
+    frac = min(1.0, budget / t_full) if t_full > 0 else 1.0
+    for _ in range(max(0, args.warmup - 1)):
+        oracle_pass(specs, 128, frac)
+    times, flops, desc = [], 0, ""
+    for _ in range(args.steps):
+        flops, dt, desc = oracle_pass(specs, 128, frac)
+        times.append(dt)
+    total = sum(times)
+    value = flops * args.steps / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD_DESC[args.workload], "tokens": tokens,
+                                        "sample_tokens": 128},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    tokens = args.tokens or (16384 if args.workload == "layer" else 8192)
+    specs = workload_tensors(args.workload, tokens)
+    prog = Program(specs, dev, world)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        prog.run()
+    barrier()
+
+    nops = len(prog.ops)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nops)]
+          for _ in range(args.steps)]
+    st = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    time.sleep(0.3)
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()                          # L2 flush, outside the timed events
+        st[i][0].record(stream)
+        prog.run(ev[i])
+        st[i][1].record(stream)
+    barrier()
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in st]
+    total_ms = sum(step_ms)
+    per_op_ms = [[a.elapsed_time(b) for a, b in ev[i]] for i in range(args.steps)]
+    gemm_ms = sum(per_op_ms[i][j] for i in range(args.steps) for j in range(nops) if prog.ops[j][1] == "gemm")
+    quant_ms = sum(per_op_ms[i][j] for i in range(args.steps) for j in range(nops) if prog.ops[j][1] == "quant")
+    if world > 1:
+        t = torch.tensor([total_ms, gemm_ms, quant_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, gemm_ms, quant_ms = t.tolist()
+
+    # End to end through the public API: pinned host inputs in, outputs back, every step.
+    h_in = [(d, torch.from_numpy(np.ascontiguousarray(h)).view(torch.bfloat16).pin_memory()) for d, h in prog.inputs]
+    h_out = [(d, torch.empty(d.shape, dtype=d.dtype, pin_memory=True)) for d in prog.outputs]
+    h2d = sum(h.numel() * h.element_size() for _, h in h_in)
+    d2h = sum(h.numel() * h.element_size() for _, h in h_out)
+    e2e_steps = max(3, min(args.steps, 10))
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for d, h in h_in:
+            d.copy_(h, non_blocking=True)
+        prog.run()
+        for d, h in h_out:
+            h.copy_(d, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    err = prog.fb.fp8blk_get_device_error()
+
+    peaks, peak_src = load_peaks()
+    fp8_peak = peaks["bf16_tflops_sustained"] * FP8_PER_BF16
+    flops_all = prog.gemm_flops * world
+    value = flops_all * args.steps / (total_ms * 1e-3) / 1e12
+    gemm_tflops = prog.gemm_flops * args.steps / (gemm_ms * 1e-3) / 1e12
+    quant_gbs = prog.quant_bytes * args.steps / (quant_ms * 1e-3) / 1e9
+    per_op = {}
+    for j, (label, kind, units, _) in enumerate(prog.ops):
+        ms = statistics.median(per_op_ms[i][j] for i in range(args.steps))
+        rate = units / (ms * 1e-3) / (1e12 if kind == "gemm" else 1e9)
+        per_op[label] = {"us": round(ms * 1e3, 1), ("tflops" if kind == "gemm" else "gbs"): round(rate, 1)}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": WORKLOAD_DESC[args.workload], "tokens_per_gpu": tokens,
+                   "l2": "flushed between steps (256 MiB write outside the timed events)",
+                   "streams": 1, "seed": {"layer": 4, "qkv_fwd": 1, "mlp_fwd": 2, "down_bwd": 3}[args.workload],
+                   "parallelism": f"dp{world}" if world > 1 else "single-gpu"},
+        "frac_of_spec_fp8_peak": value / SPEC_FP8_TFLOPS,
+        "roofline": {"bound": "tensor", "kernel": "gemm_blockwise_kernel", "achieved": gemm_tflops,
+                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 sustained x {FP8_PER_BF16:g} (nominal fp8/bf16 ratio)",
+                     "frac_of_spec_fp8": gemm_tflops / SPEC_FP8_TFLOPS},
+        "quant": {"kernel": "quant_tile_kernel", "achieved_gbs": quant_gbs, "peak_gbs": peaks["hbm_gbs"],
+                  "frac": quant_gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm copy"},
+        "per_op_median": per_op,
+        "e2e": {"value": flops_all * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": nops * args.steps,
+        "clocks": clocks,
+        "device_error": prog.fb.status_string(err),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(workload_tensors(args.workload, 256) if tokens != 256 else specs)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0 if err == 0 else 1
+
+
+def run_sweep(args, local_rank: int):
+    """Token sweep: each linear layer fwd (quantise X, W + GEMM) at M in the sweep list."""
+    import torch
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    results = []
+    for m in workloads.TOKEN_SWEEP:
+        specs = [dict(s, passes=("fwd", "dgrad", "wgrad")) for s in workload_tensors("layer", m)]
+        prog = Program(specs, dev, 1)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            prog.run()
+        torch.cuda.synchronize()
+        n = max(5, min(args.steps, 20))
+        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in prog.ops] for _ in range(n)]
+        for i in range(n):
+            flush.zero_()
+            prog.run(ev[i])
+        torch.cuda.synchronize()
+        row = {"tokens": m}
+        for j, (label, kind, units, _) in enumerate(prog.ops):
+            if kind == "gemm":
+                ms = statistics.median(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(n))
+                row[label] = round(units / (ms * 1e-3) / 1e12, 1)
+        tot = sum(statistics.median(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(n))
+                  for j in range(len(prog.ops)))
+        row["layer_tflops_incl_quant"] = round(prog.gemm_flops / (tot * 1e-3) / 1e12, 1)
+        results.append(row)
+        del prog
+        torch.cuda.empty_cache()
+    print(json.dumps({"sweep": results, "unit": "TFLOP/s (median per-kernel events, L2 flushed)"}), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(WORKLOAD_DESC), default="layer")
+    ap.add_argument("--tokens", type=int, default=0, help="tokens per GPU (default 16384 for layer, else 8192)")
+    ap.add_argument("--sweep", action="store_true", help="token sweep of the layer GEMMs (one JSON line)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}; launch N>1 with torch.distributed.run")
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        if args.sweep:
+            return run_sweep(args, local_rank) if rank == 0 else 0
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -11,9 +11,13 @@
 // scales are applied to it before it joins the running sum.
 //
 // Design (one persistent CTA per SM, 320 threads, 128 x BN output tiles):
-//   warp 0      TMA producer: per K-block, a 128x128 A tile and a BNx128 B
-//               tile (E4M3, 128-byte swizzle) into a ring of shared-memory
-//               stages; completion counted in bytes on a "full" mbarrier.
+//   warp 0      producer.  Lane 0 issues, per K-block, TMA loads of a 128x128
+//               A tile and a BNx128 B tile (E4M3, 128-byte swizzle) into a
+//               ring of shared-memory stages ("full" mbarrier counts bytes).
+//               All 32 lanes stream the K-block's scales (sa for the tile's
+//               128 rows; sb for its columns or n-blocks) into a separate
+//               8-deep shared-memory ring with cp.async, completion tracked
+//               by an mbarrier, so no global load sits on the promotion path.
 //   warp 1      TMEM owner and MMA issuer (one thread): 4 x tcgen05.mma
 //               kind::f8f6f4 (M=128, N=BN, K=32) per K-block into one of two
 //               TMEM accumulators (2 x BN fp32 columns), then tcgen05.commit
@@ -21,11 +25,13 @@
 //   warps 2..9  promotion + epilogue: two warpgroups, each owning BN/2
 //               columns of the tile (a warp reads the 32 TMEM lanes given by
 //               its index mod 4); per K-block they read the partial product
-//               from TMEM and fold it into fp32 registers,
+//               from TMEM (16-column loads) and fold it into fp32
+//               registers with packed f32x2 FMAs,
 //                   FWD/DGRAD: acc += P * (sa[m] * sb[n-block])
 //                   WGRAD    : acc += (P * sb[n]) * sa[m]
-//               then hand the TMEM buffer back; after the last K-block they
-//               round the tile to bf16 and store it.
+//               then hand the TMEM buffer and the scale slot back; after the
+//               last K-block they round the tile to bf16 and store it with
+//               32-byte vector stores.
 // The MMA of K-block kb+1 runs while the promotion of kb is in flight
 // (double-buffered TMEM), and TMA runs up to kStages K-blocks ahead.
 //
@@ -51,6 +57,7 @@ constexpr int BK = 128;
 constexpr int kThreads = 320;
 constexpr int kEpiWarp0 = 2;
 constexpr int kEpiWarps = 8;
+constexpr int kSRing = 8;        // scale ring depth (K-blocks)
 
 template <int BN>
 struct Cfg {
@@ -62,18 +69,26 @@ struct Cfg {
   static constexpr int kHalf = BN / 2;  // columns per epilogue warpgroup
 };
 
+// One K-block's scales for one tile.
+struct ScaleSlot {
+  float sa[BM];       // sa[kb][m0 + r]
+  float sb[256];      // WGRAD: sb[kb][n0 + c];  FWD/DGRAD: sb[n-block][kb] in sb[0], sb[1]
+};
+
 struct Ctrl {
   uint64_t full[8];
   uint64_t empty[8];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t sfull[kSRing];
+  uint64_t sempty[kSRing];
   uint64_t mma_done;
   uint64_t never;         // completed by nothing: the stall test waits on it
   uint32_t tmem_base;
   int abort;
-  alignas(16) float sbuf[kEpiWarps][2][128];  // WGRAD: per-warp copy of this K-block's B scales (float4 access)
+  alignas(16) ScaleSlot slots[kSRing];
 };
-static_assert(offsetof(Ctrl, sbuf) % 16 == 0, "sbuf is written with 16-byte vector stores");
+static_assert(offsetof(Ctrl, slots) % 16 == 0, "scale slots are filled with 16-byte copies");
 
 template <int BN>
 constexpr int smem_bytes() {
@@ -96,6 +111,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(smem_dst)), "l"(gsrc) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gsrc) : "memory");
+}
+
+// The mbarrier receives one arrival from this thread once all its earlier cp.async copies have landed.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
 // tcgen05.wait::ld, tied to the registers it makes valid so that the
 // compiler cannot read them before the wait.
 __device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
@@ -114,6 +142,49 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
+}
+
+// acc(2) += p(2) * f   (packed, one instruction for two columns)
+__device__ __forceinline__ void ffma2_scalar(float& a0, float& a1, uint32_t p0, uint32_t p1, float f) {
+  asm("{\n\t.reg .b64 ra, rp, rf;\n\t"
+      "mov.b64 ra, {%0, %1};\n\t"
+      "mov.b64 rp, {%2, %3};\n\t"
+      "mov.b64 rf, {%4, %4};\n\t"
+      "fma.rn.f32x2 ra, rp, rf, ra;\n\t"
+      "mov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(p0), "r"(p1), "f"(f));
+}
+
+// acc(2) += (p(2) * sb(2)) * sa
+__device__ __forceinline__ void ffma2_cols(float& a0, float& a1, uint32_t p0, uint32_t p1, float2 sb, float sa) {
+  asm("{\n\t.reg .b64 ra, rp, rb, rs;\n\t"
+      "mov.b64 ra, {%0, %1};\n\t"
+      "mov.b64 rp, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rs, {%6, %6};\n\t"
+      "mul.rn.f32x2 rp, rp, rb;\n\t"
+      "fma.rn.f32x2 ra, rp, rs, ra;\n\t"
+      "mov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(p0), "r"(p1), "f"(sb.x), "f"(sb.y), "f"(sa));
+}
+
+template <bool kWgrad>
+__device__ __forceinline__ void promote16(float* acc, const uint32_t (&r)[16], float f, const float* sbc, float sa) {
+#pragma unroll
+  for (int j = 0; j < 16; j += 2) {
+    if constexpr (kWgrad)
+      ffma2_cols(acc[j], acc[j + 1], r[j], r[j + 1], *reinterpret_cast<const float2*>(sbc + j), sa);
+    else
+      ffma2_scalar(acc[j], acc[j + 1], r[j], r[j + 1], f);
+  }
+}
+
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&v)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]),
+               "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 
 }  // namespace
@@ -143,6 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctrl->tfull[b], 1);
       mbar_init(&ctrl->tempty[b], kEpiWarps);
     }
+    for (int s = 0; s < kSRing; ++s) {
+      mbar_init(&ctrl->sfull[s], 32);   // one cp.async arrival per producer lane
+      mbar_init(&ctrl->sempty[s], kEpiWarps);
+    }
     mbar_init(&ctrl->mma_done, 1);
     mbar_init(&ctrl->never, 1);
     ctrl->abort = 0;
@@ -163,38 +238,60 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = &ctrl->abort;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int64_t issued = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-        const int mb = tile % num_mb, nb = tile / num_mb;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded(&ctrl->empty[stage], phase ^ 1u, abort, p.timeout_ns, p.err)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sa_tile = smem + stage * C::kStageBytes;
-          mbar_arrive_expect_tx(&ctrl->full[stage], C::kStageBytes);
-          tma_load_2d(sa_tile, &tm_a, &ctrl->full[stage], kb * BK, mb * BM);
-          tma_load_2d(sa_tile + C::kABytes, &tm_b, &ctrl->full[stage], kb * BK, nb * BN);
-          ++issued;
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
+    // ------------------------------------------------------------ producer (whole warp)
+    int stage = 0, slot = 0;
+    uint32_t phase = 0, sphase = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+      const int mb = tile % num_mb, nb = tile / num_mb;
+      const int64_t m0 = static_cast<int64_t>(mb) * BM, n0 = static_cast<int64_t>(nb) * BN;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        // Scales of this K-block into the scale ring.
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&ctrl->sempty[slot], sphase ^ 1u, abort, p.timeout_ns, p.err))) {
+          ok = false;
+          break;
+        }
+        ScaleSlot& ss = ctrl->slots[slot];
+        cp_async_16(&ss.sa[lane * 4], p.sa + static_cast<int64_t>(kb) * p.M + m0 + lane * 4);
+        if constexpr (kWgrad) {
+          for (int c = lane * 4; c < BN; c += 128)
+            cp_async_16(&ss.sb[c], p.sb + static_cast<int64_t>(kb) * p.N + n0 + c);
+        } else {
+          if (lane < BN / 128) cp_async_4(&ss.sb[lane], p.sb + (n0 / 128 + lane) * kblocks + kb);
+        }
+        cp_async_arrive(&ctrl->sfull[slot]);
+        if (++slot == kSRing) {
+          slot = 0;
+          sphase ^= 1u;
+        }
+        // Operand tiles of this K-block into the stage ring.
+        if (lane == 0) {
+          ok = mbar_wait_bounded(&ctrl->empty[stage], phase ^ 1u, abort, p.timeout_ns, p.err);
+          if (ok) {
+            uint8_t* sa_tile = smem + stage * C::kStageBytes;
+            mbar_arrive_expect_tx(&ctrl->full[stage], C::kStageBytes);
+            tma_load_2d(sa_tile, &tm_a, &ctrl->full[stage], kb * BK, static_cast<int>(m0));
+            tma_load_2d(sa_tile + C::kABytes, &tm_b, &ctrl->full[stage], kb * BK, static_cast<int>(n0));
           }
         }
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) break;
+        ++issued;
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
-      {
-        // Let the loads still in flight land before the CTA's smem goes away
-        // (on the normal path they have all been consumed: no wait).
-        const int64_t first = issued > C::kStages ? issued - C::kStages : 0;
-        for (int64_t j = first; j < issued; ++j)
-          mbar_wait_bounded(&ctrl->full[j % C::kStages], static_cast<uint32_t>((j / C::kStages) & 1), nullptr,
-                            p.timeout_ns, p.err);
-      }
+    }
+    // Let the copies still in flight land before the CTA's smem goes away
+    // (on the normal path they have all been consumed: no wait).
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (lane == 0) {
+      const int64_t first = issued > C::kStages ? issued - C::kStages : 0;
+      for (int64_t j = first; j < issued; ++j)
+        mbar_wait_bounded(&ctrl->full[j % C::kStages], static_cast<uint32_t>((j / C::kStages) & 1), nullptr,
+                          p.timeout_ns, p.err);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -233,14 +330,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(&ctrl->mma_done);
       mbar_wait_bounded(&ctrl->mma_done, 0, nullptr, p.timeout_ns, p.err);
     }
-  } else {
+  } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ promotion + epilogue
     const int ew = warp - kEpiWarp0;  // 0..7
     const int wg = ew >> 2;           // which half of the tile's columns
     const int quarter = warp & 3;     // TMEM lanes this warp may read
     const int row = quarter * 32 + lane;
     const int col0 = wg * C::kHalf;
-    uint32_t abuf = 0, aphase = 0;
+    uint32_t abuf = 0, aphase = 0, sphase = 0;
+    int slot = 0;
     float acc[C::kHalf];
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
@@ -250,70 +348,47 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int j = 0; j < C::kHalf; ++j) acc[j] = 0.0f;
 
-      // Scales of the next K-block are fetched one step ahead.
-      float sa_next = __ldg(p.sa + m);
-      float sb_next = 0.0f;
-      float4 sbv_next = make_float4(0.f, 0.f, 0.f, 0.f);
-      if constexpr (kWgrad) {
-        if (lane < C::kHalf / 4) sbv_next = __ldg(reinterpret_cast<const float4*>(p.sb + ncol0) + lane);
-      } else {
-        sb_next = __ldg(p.sb + (ncol0 / 128) * kblocks);
-      }
-
       for (int kb = 0; kb < kblocks; ++kb) {
-        const float sa_cur = sa_next;
-        const float sb_cur = sb_next;
-        float* sbuf = ctrl->sbuf[ew][kb & 1];
-        if constexpr (kWgrad) {
-          if (lane < C::kHalf / 4) reinterpret_cast<float4*>(sbuf)[lane] = sbv_next;
-          __syncwarp();
-        }
-        if (kb + 1 < kblocks) {
-          sa_next = __ldg(p.sa + static_cast<int64_t>(kb + 1) * p.M + m);
-          if constexpr (kWgrad) {
-            if (lane < C::kHalf / 4)
-              sbv_next = __ldg(reinterpret_cast<const float4*>(p.sb + static_cast<int64_t>(kb + 1) * p.N + ncol0) + lane);
-          } else {
-            sb_next = __ldg(p.sb + (ncol0 / 128) * kblocks + kb + 1);
-          }
-        }
-        const bool got = mbar_wait_bounded(&ctrl->tfull[abuf], aphase, abort, p.timeout_ns, p.err);
+        const bool got = mbar_wait_bounded(&ctrl->sfull[slot], sphase, abort, p.timeout_ns, p.err) &&
+                         mbar_wait_bounded(&ctrl->tfull[abuf], aphase, abort, p.timeout_ns, p.err);
         if (!__all_sync(0xFFFFFFFFu, got)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
+        const ScaleSlot& ss = ctrl->slots[slot];
+        const float sa = ss.sa[row];
+        const float f = kWgrad ? 0.0f : sa * ss.sb[BN == 256 ? wg : 0];
+        const float* sbc = ss.sb + col0;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * BN + col0;
-        const float f = sa_cur * sb_cur;
 #pragma unroll
         for (int c = 0; c < C::kHalf; c += 16) {
           uint32_t r[16];
           tmem_ld_32x32b_x16(taddr + c, r);
           tmem_wait_ld16(r);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if constexpr (kWgrad)
-              acc[c + j] = fmaf(__uint_as_float(r[j]) * sbuf[c + j], sa_cur, acc[c + j]);
-            else
-              acc[c + j] = fmaf(__uint_as_float(r[j]), f, acc[c + j]);
-          }
+          promote16<kWgrad>(acc + c, r, f, sbc + c, sa);
         }
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ctrl->tempty[abuf]);
+        if (lane == 0) {
+          mbar_arrive(&ctrl->tempty[abuf]);
+          mbar_arrive(&ctrl->sempty[slot]);
+        }
         abuf ^= 1u;
         if (abuf == 0) aphase ^= 1u;
+        if (++slot == kSRing) {
+          slot = 0;
+          sphase ^= 1u;
+        }
       }
       if (!ok) break;
       uint16_t* drow = p.d + m * p.ldd + ncol0;
 #pragma unroll
-      for (int j = 0; j < C::kHalf; j += 8) {
-        uint4 v;
-        v.x = pack_bf16x2(acc[j + 0], acc[j + 1]);
-        v.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
-        v.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
-        v.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
-        *reinterpret_cast<uint4*>(drow + j) = v;
+      for (int j = 0; j < C::kHalf; j += 16) {
+        uint32_t v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = pack_bf16x2(acc[j + 2 * q], acc[j + 2 * q + 1]);
+        st_global_v8(drow + j, v);
       }
     }
   }

@@ -17,16 +17,23 @@
 // go through one shared-memory copy of the tile.  HBM bound: per element
 // 2 B read + 1 B code + 4/128 B scale per output layout.
 //
+// Exactness of the scale.  s = fl32(amax / 448) is computed as y = amax*2^-6
+// (exact) followed by a correctly rounded division by 7 with one FMA
+// correction step (Markstein's method for a known divisor): q0 = fl(y*c),
+// r = fma(-7, q0, y), s = fma(r, c, q0), c = fl(1/7).  amax is a bfloat16
+// magnitude, so the 2^15 possible inputs were checked exhaustively against
+// the correctly rounded quotient (tests/test_scale_division.py).
+//
 // Exactness of x / s.  A correctly rounded binary32 division per element
 // costs more issue slots than the HBM budget allows, so each value is
-// bracketed instead: with r = 1/s (correctly rounded), lo = x*fl(r(1-2^-20))
-// and hi = x*fl(r(1+2^-20)) satisfy |lo| <= |fl(x/s)| <= |hi| (the three
-// roundings move the product by at most 3*2^-24 relative, far inside the
-// 2^-20 margin).  Rounding to E4M3 is monotonic, so when lo and hi give the
-// same code that code is the one of fl(x/s); otherwise (about one value in
-// 2^16) the value is recomputed with the correctly rounded division.  The
-// saturating conversion equals clamp-then-round because every value above
-// 448 rounds or saturates to 448.
+// bracketed instead: with r ~ 1/s (hardware approximation, relative error
+// below 2^-22), lo = x*fl(r(1-2^-20)) and hi = x*fl(r(1+2^-20)) satisfy
+// |lo| <= |fl(x/s)| <= |hi| (all the roundings together move the product by
+// less than 2^-21 relative, inside the 2^-20 margin).  Rounding to E4M3 is
+// monotonic, so when lo and hi give the same code that code is the one of
+// fl(x/s); otherwise (about one value in 2^15) the value is recomputed with
+// the correctly rounded division.  The saturating conversion equals
+// clamp-then-round because every value above 448 rounds or saturates to 448.
 #include <cuda_fp8.h>
 
 #include "device.cuh"
@@ -38,20 +45,27 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kThreads = 256;
-constexpr int kXsStride = kTile + 8;     // bf16 elements per smem row (272 B, keeps 16-B alignment)
-constexpr int kCsStride = kTile + 16;    // code bytes per smem row (144 B)
-constexpr int kSmallBytes = 64 + 2 * kTile * 4 + kTile * 4;                   // warpmax, red, colamax
-constexpr int kSmemBytes = kSmallBytes + kTile * kXsStride * 2 + kTile * kCsStride;
+// Shared memory of the transposed paths (no padding needed: see the access patterns below).
+constexpr int kXsBytes = kTile * kTile * 2;       // bf16 tile, 256-byte rows
+constexpr int kCsBytes = kTile * kTile;           // transposed codes, 128-byte rows, 16-B chunks swizzled
+constexpr int kCpartBytes = 8 * 64 * 4;           // per-warp packed column maxima
+constexpr int kQsBytes = kTile * 16;              // per-column {s, r_lo, r_hi}
+constexpr int kSmallBytes = 64;                   // per-warp block maxima
+constexpr int kSmemBytes = kSmallBytes + kQsBytes + kCpartBytes + kXsBytes + kCsBytes;
 
 struct QScale {
   float s, rlo, rhi;
 };
 
 __device__ __forceinline__ QScale make_qscale(float amax) {
-  float s = __fdiv_rn(amax, 448.0f);
-  s = fmaxf(s, 1e-12f);
-  const float r = __frcp_rn(s);
-  return {s, r * (1.0f - 0x1p-20f), r * (1.0f + 0x1p-20f)};
+  const float c7 = 0x1.24924ap-3f;  // fl32(1/7)
+  const float y = amax * 0.015625f;
+  const float q0 = y * c7;
+  const float r = fmaf(-7.0f, q0, y);
+  const float s = fmaxf(fmaf(r, c7, q0), 1e-12f);
+  float rc;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(s));
+  return {s, rc * (1.0f - 0x1p-20f), rc * (1.0f + 0x1p-20f)};
 }
 
 // Two values -> two E4M3 codes, `a` in the low byte.
@@ -59,20 +73,41 @@ __device__ __forceinline__ uint32_t cvt2(float a, float b) {
   return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
 }
 
-__device__ __noinline__ uint2 quant8_slow(const float* x, float s) {
+// (a0, a1) * (b, b) with one packed multiply.
+__device__ __forceinline__ float2 mul2(float a0, float a1, float b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %4};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a0), "f"(a1), "f"(b));
+  return d;
+}
+
+__device__ __noinline__ uint2 quant8_slow(float x0, float x1, float x2, float x3, float x4, float x5, float x6,
+                                          float x7, float s) {
   uint2 out;
-  out.x = cvt2(__fdiv_rn(x[0], s), __fdiv_rn(x[1], s)) | (cvt2(__fdiv_rn(x[2], s), __fdiv_rn(x[3], s)) << 16);
-  out.y = cvt2(__fdiv_rn(x[4], s), __fdiv_rn(x[5], s)) | (cvt2(__fdiv_rn(x[6], s), __fdiv_rn(x[7], s)) << 16);
+  out.x = cvt2(__fdiv_rn(x0, s), __fdiv_rn(x1, s)) | (cvt2(__fdiv_rn(x2, s), __fdiv_rn(x3, s)) << 16);
+  out.y = cvt2(__fdiv_rn(x4, s), __fdiv_rn(x5, s)) | (cvt2(__fdiv_rn(x6, s), __fdiv_rn(x7, s)) << 16);
   return out;
 }
 
 // Eight values -> eight codes packed little-endian (x[0] in the lowest byte).
 __device__ __forceinline__ uint2 quant8(const float (&x)[8], const QScale& q) {
-  const uint32_t lo0 = cvt2(x[0] * q.rlo, x[1] * q.rlo) | (cvt2(x[2] * q.rlo, x[3] * q.rlo) << 16);
-  const uint32_t lo1 = cvt2(x[4] * q.rlo, x[5] * q.rlo) | (cvt2(x[6] * q.rlo, x[7] * q.rlo) << 16);
-  const uint32_t hi0 = cvt2(x[0] * q.rhi, x[1] * q.rhi) | (cvt2(x[2] * q.rhi, x[3] * q.rhi) << 16);
-  const uint32_t hi1 = cvt2(x[4] * q.rhi, x[5] * q.rhi) | (cvt2(x[6] * q.rhi, x[7] * q.rhi) << 16);
-  if (__builtin_expect(((lo0 ^ hi0) | (lo1 ^ hi1)) != 0, 0)) return quant8_slow(x, q.s);
+  uint32_t lo[4], hi[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 l = mul2(x[2 * j], x[2 * j + 1], q.rlo);
+    const float2 h = mul2(x[2 * j], x[2 * j + 1], q.rhi);
+    lo[j] = cvt2(l.x, l.y);
+    hi[j] = cvt2(h.x, h.y);
+  }
+  const uint32_t lo0 = lo[0] | (lo[1] << 16), lo1 = lo[2] | (lo[3] << 16);
+  const uint32_t hi0 = hi[0] | (hi[1] << 16), hi1 = hi[2] | (hi[3] << 16);
+  if (__builtin_expect(((lo0 ^ hi0) | (lo1 ^ hi1)) != 0, 0))
+    return quant8_slow(x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7], q.s);
   return make_uint2(lo0, lo1);
 }
 
@@ -83,13 +118,20 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
 }
 
+// |bf16| maxima on raw bits: clearing the sign keeps the order of finite magnitudes.
+constexpr uint32_t kAbs2 = 0x7FFF7FFFu;
+
 __device__ __forceinline__ float absmax8(const uint4& v) {
-  // |bf16| max on the raw bits: clearing the sign bits keeps the order of
-  // finite magnitudes, and the max is exact.
-  const uint32_t m = 0x7FFF7FFFu;
-  uint32_t a = __vmaxu2(__vmaxu2(v.x & m, v.y & m), __vmaxu2(v.z & m, v.w & m));
+  uint32_t a = __vmaxu2(__vmaxu2(v.x & kAbs2, v.y & kAbs2), __vmaxu2(v.z & kAbs2, v.w & kAbs2));
   a = max(a & 0xFFFFu, a >> 16);
   return __uint_as_float(a << 16);
+}
+
+__device__ __forceinline__ void load_tile(uint4 (&v)[8], const QuantArgs& a, int64_t tile, int rbase, int chunk) {
+  const int64_t tr = tile % a.tiles_r, tc = tile / a.tiles_r;
+  const uint16_t* base = a.x + (tr * kTile + rbase) * a.ldx + tc * kTile + chunk * 8;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = ld_nc_v4(base + 16 * i * a.ldx);
 }
 
 }  // namespace
@@ -104,41 +146,27 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
   constexpr bool kBlockScale = kBlk || kBlkT;
 
   extern __shared__ __align__(16) uint8_t smem[];
-  float* warpmax = reinterpret_cast<float*>(smem);                          // [8] (64 B reserved)
-  float* red = reinterpret_cast<float*>(smem + 64);                         // [2][128]
-  float* colamax = red + 2 * kTile;                                         // [128]
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + kSmallBytes);           // [128][136] bf16
-  uint8_t* cs = smem + kSmallBytes + kTile * kXsStride * 2;                 // [128][144] codes
+  float* warpmax = reinterpret_cast<float*>(smem);                                      // [8]
+  float4* qs = reinterpret_cast<float4*>(smem + kSmallBytes);                           // [128] column scales
+  uint32_t* cpart = reinterpret_cast<uint32_t*>(smem + kSmallBytes + kQsBytes);         // [8][64]
+  uint8_t* xs = smem + kSmallBytes + kQsBytes + kCpartBytes;                            // [128][256 B]
+  uint8_t* cs = xs + kXsBytes;                                                          // [128][128 B]
 
   const int t = threadIdx.x;
+  const int lane = t & 31, warp = t >> 5;
   const int chunk = t & 15;      // this thread's 16-byte column chunk of the tile
   const int rbase = t >> 4;      // rows rbase + 16 i, i = 0..7
   const int64_t tiles = a.tiles_r * a.tiles_c;
 
-  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+  uint4 v[8];
+  int64_t tile = blockIdx.x;
+  if (tile < tiles) load_tile(v, a, tile, rbase, chunk);
+
+  for (; tile < tiles; tile += gridDim.x) {
     const int64_t tr = tile % a.tiles_r, tc = tile / a.tiles_r;
     const int64_t row0 = tr * kTile, col0 = tc * kTile;
 
-    uint4 v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      v[i] = ld_nc_v4(a.x + (row0 + rbase + 16 * i) * a.ldx + col0 + chunk * 8);
-
-    if constexpr (kRow) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float amax = absmax8(v[i]);
-#pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-        const QScale q = make_qscale(amax);
-        float f[8];
-        unpack8(v[i], f);
-        const int64_t r = row0 + rbase + 16 * i;
-        *reinterpret_cast<uint2*>(a.q_row + r * a.cols + col0 + chunk * 8) = quant8(f, q);
-        if (chunk == 0) a.s_row[tc * a.rows + r] = q.s;
-      }
-    }
-
+    // ---------------------------------------------------------------- from registers
     QScale qblk{};
     if constexpr (kBlockScale) {
       float amax = 0.0f;
@@ -146,7 +174,7 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
       for (int i = 0; i < 8; ++i) amax = fmaxf(amax, absmax8(v[i]));
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-      if ((t & 31) == 0) warpmax[t >> 5] = amax;
+      if (lane == 0) warpmax[warp] = amax;
       __syncthreads();
       amax = warpmax[0];
 #pragma unroll
@@ -158,63 +186,107 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
       }
     }
 
-    if constexpr (kBlk) {
+    if constexpr (kRow || kBlk) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
+        QScale q;
+        if constexpr (kRow) {
+          float amax = absmax8(v[i]);
+#pragma unroll
+          for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+          q = make_qscale(amax);
+        } else {
+          q = qblk;
+        }
         float f[8];
         unpack8(v[i], f);
         const int64_t r = row0 + rbase + 16 * i;
-        *reinterpret_cast<uint2*>(a.q_row + r * a.cols + col0 + chunk * 8) = quant8(f, qblk);
+        *reinterpret_cast<uint2*>(a.q_row + r * a.cols + col0 + chunk * 8) = quant8(f, q);
+        if constexpr (kRow) {
+          if (chunk == 0) a.s_row[tc * a.rows + r] = q.s;
+        }
       }
     }
 
     if constexpr (kTileSmem) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        *reinterpret_cast<uint4*>(xs + (rbase + 16 * i) * kXsStride + chunk * 8) = v[i];
-      __syncthreads();
-
-      const int col = t & 127;
+      for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4*>(xs + (rbase + 16 * i) * 256 + chunk * 16) = v[i];
       if constexpr (kColT) {
-        const int half = t >> 7;
-        uint32_t m = 0;
-        for (int r = half * 64; r < half * 64 + 64; ++r) m = max(m, static_cast<uint32_t>(xs[r * kXsStride + col] & 0x7FFFu));
-        red[half * kTile + col] = __uint_as_float(m << 16);
-        __syncthreads();
-        if (t < kTile) {
-          const float am = fmaxf(red[t], red[kTile + t]);
-          colamax[t] = am;
-          a.s_t[tr * a.cols + col0 + t] = make_qscale(am).s;
+        // Column maxima of this thread's 8 rows, packed two columns per word,
+        // then across the two row sets of the warp.
+        uint32_t m[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          m[0] = __vmaxu2(m[0], v[i].x & kAbs2);
+          m[1] = __vmaxu2(m[1], v[i].y & kAbs2);
+          m[2] = __vmaxu2(m[2], v[i].z & kAbs2);
+          m[3] = __vmaxu2(m[3], v[i].w & kAbs2);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m[j] = __vmaxu2(m[j], __shfl_xor_sync(0xFFFFFFFFu, m[j], 16));
+        if (lane < 16) *reinterpret_cast<uint4*>(cpart + warp * 64 + chunk * 4) = make_uint4(m[0], m[1], m[2], m[3]);
+      }
+    }
+
+    // Registers are free: start loading the next tile while the shared-memory work runs.
+    if (tile + gridDim.x < tiles) load_tile(v, a, tile + gridDim.x, rbase, chunk);
+
+    if constexpr (kTileSmem) {
+      __syncthreads();
+      if constexpr (kColT) {
+        if (t < 64) {  // word t covers columns 2t and 2t+1
+          uint32_t mx = 0;
+#pragma unroll
+          for (int w = 0; w < 8; ++w) mx = __vmaxu2(mx, cpart[w * 64 + t]);
+          const QScale q0 = make_qscale(__uint_as_float(mx << 16));
+          const QScale q1 = make_qscale(__uint_as_float(mx & 0xFFFF0000u));
+          qs[2 * t] = make_float4(q0.s, q0.rlo, q0.rhi, 0.f);
+          qs[2 * t + 1] = make_float4(q1.s, q1.rlo, q1.rhi, 0.f);
+          *reinterpret_cast<float2*>(a.s_t + tr * a.cols + col0 + 2 * t) = make_float2(q0.s, q1.s);
         }
         __syncthreads();
       }
-
-      // Transposed codes: item = (column, 16-row chunk); write into the code tile.
+      // Transposed codes.  Item = (column pair cp, 16-row chunk rc); the 32 lanes
+      // of a warp read consecutive words of the same smem rows (conflict-free) and
+      // write 16-byte chunks whose position is XOR-swizzled by cp (conflict-free).
+      const uint32_t* xs32 = reinterpret_cast<const uint32_t*>(xs);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 2; ++j) {
         const int item = t + kThreads * j;
-        const int c = item & 127, rc = item >> 7;
-        QScale q;
-        if constexpr (kColT) q = make_qscale(colamax[c]); else q = qblk;
-        float f0[8], f1[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          f0[i] = __uint_as_float(static_cast<uint32_t>(xs[(rc * 16 + i) * kXsStride + c]) << 16);
-          f1[i] = __uint_as_float(static_cast<uint32_t>(xs[(rc * 16 + 8 + i) * kXsStride + c]) << 16);
+        const int cp = item & 63, rc = item >> 6;
+        QScale qa, qb;
+        if constexpr (kColT) {
+          const float4 fa = qs[2 * cp], fb = qs[2 * cp + 1];
+          qa = {fa.x, fa.y, fa.z};
+          qb = {fb.x, fb.y, fb.z};
+        } else {
+          qa = qb = qblk;
         }
-        const uint2 c0 = quant8(f0, q), c1 = quant8(f1, q);
-        *reinterpret_cast<uint4*>(cs + c * kCsStride + rc * 16) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+        float lo[16], hi[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t w = xs32[(rc * 16 + i) * 64 + cp];
+          lo[i] = bf16lo(w);
+          hi[i] = bf16hi(w);
+        }
+        const uint2 a0 = quant8(*reinterpret_cast<const float(*)[8]>(lo), qa);
+        const uint2 a1 = quant8(*reinterpret_cast<const float(*)[8]>(lo + 8), qa);
+        const uint2 b0 = quant8(*reinterpret_cast<const float(*)[8]>(hi), qb);
+        const uint2 b1 = quant8(*reinterpret_cast<const float(*)[8]>(hi + 8), qb);
+        const int phys = (rc ^ (cp & 7)) * 16;
+        *reinterpret_cast<uint4*>(cs + (2 * cp) * 128 + phys) = make_uint4(a0.x, a0.y, a1.x, a1.y);
+        *reinterpret_cast<uint4*>(cs + (2 * cp + 1) * 128 + phys) = make_uint4(b0.x, b0.y, b1.x, b1.y);
       }
       __syncthreads();
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int k = t + kThreads * j;
         const int c = k >> 3, part = k & 7;
-        const uint4 codes = *reinterpret_cast<const uint4*>(cs + c * kCsStride + part * 16);
+        const uint4 codes = *reinterpret_cast<const uint4*>(cs + c * 128 + ((part ^ ((c >> 1) & 7)) * 16));
         *reinterpret_cast<uint4*>(a.q_t + (col0 + c) * a.rows + row0 + part * 16) = codes;
       }
     }
-    if constexpr (kTileSmem || kBlockScale) __syncthreads();  // smem reused by the next tile
+    if constexpr (kTileSmem || kBlockScale) __syncthreads();  // shared memory is reused by the next tile
   }
 }
 

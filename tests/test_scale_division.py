@@ -1,0 +1,67 @@
+"""The quantisers' scale rule, proven exhaustively on the CPU with exact arithmetic.
+
+The kernels compute s = max(fl32(amax / 448), fl32(1e-12)) without a full
+IEEE division: with y = amax * 2^-6 (exact) and c = fl32(1/7),
+    q0 = fl32(y * c);   r = fma(-7, q0, y);   s = fma(r, c, q0)
+(the FMA correction step for division by a constant that Markstein
+introduced; Brisebarre, Muller and Raina, "Accelerating correctly rounded
+floating-point division when the divisor is known in advance", IEEE Trans.
+Computers 2004, analyse when it is correctly rounded).  amax is a bfloat16
+magnitude, so there are only 2^15 inputs; this test runs every one through
+an exact model of binary32 round-to-nearest-even and fused multiply-add and
+checks the result against the correctly rounded quotient.
+"""
+from fractions import Fraction
+
+import numpy as np
+
+
+def rn32(v: Fraction) -> Fraction:
+    """Round a rational to the nearest binary32 value, ties to even (no overflow in this test)."""
+    if v == 0:
+        return Fraction(0)
+    sign = -1 if v < 0 else 1
+    a = abs(v)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    # a in [2^e, 2^(e+1)); binary32 keeps 24 significant bits, subnormals below 2^-126
+    q = max(e, -126) - 23
+    m = a / Fraction(2) ** q
+    fl = m.numerator // m.denominator
+    rem = m - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return sign * fl * Fraction(2) ** q
+
+
+def bf16_value(bits: int) -> Fraction:
+    f = np.array([bits << 16], np.uint32).view(np.float32)[0]
+    return Fraction(float(f))
+
+
+C7 = rn32(Fraction(1, 7))
+FLOOR = Fraction(float(np.float32(1e-12)))
+
+
+def fast_scale(amax: Fraction) -> Fraction:
+    y = amax / 64                              # exact for every normal bf16 amax; subnormal y is exact too
+    q0 = rn32(y * C7)
+    r = rn32(y - 7 * q0)                       # fma(-7, q0, y): exact product, one rounding
+    s = rn32(r * C7 + q0)                      # fma(r, c, q0)
+    return max(s, FLOOR)
+
+
+def test_c7_is_the_rounded_reciprocal():
+    assert C7 == Fraction(float(np.float32(1.0) / np.float32(7.0)))
+    assert float(C7).hex() == "0x1.24924a0000000p-3"
+
+
+def test_scale_formula_is_correctly_rounded_for_every_bf16_amax():
+    bad = []
+    for bits in range(0, 0x7F80):                # every finite non-negative bfloat16
+        amax = bf16_value(bits)
+        want = max(rn32(amax / 448), FLOOR)
+        if fast_scale(amax) != want:
+            bad.append(bits)
+    assert not bad, f"{len(bad)} mismatches, first {[hex(b) for b in bad[:5]]}"

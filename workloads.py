@@ -9,8 +9,10 @@ heads of dim 128, MLP width 8960) and rounds them to bfloat16.
 Every tensor is returned as a numpy ``uint16`` array holding bfloat16 bit
 patterns, row-major.  ``bf16_to_f32`` widens them back for inspection.
 
-Recipes (all draws use ``numpy.random.default_rng(seed)`` in float32 and
-round to bfloat16 with round-to-nearest-even):
+Recipes (all draws start from ``numpy.random.default_rng(seed)``; each tensor's
+normal draws come in float32 from independent child streams, one per block of
+1024 rows, so the values do not depend on the thread count; values are
+rounded to bfloat16 with round-to-nearest-even):
 
 * tiny         X[256x256] ~ N(0,1), W[256x256] ~ N(0,0.02)               seed 0
 * qkv_fwd      X[Mx1536] ~ N(0,1) with ceil(0.001*1536)=2 outlier channels
@@ -28,8 +30,13 @@ round to bfloat16 with round-to-nearest-even):
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
+
+_CHUNK_ROWS = 1024          # rows per independently seeded chunk (fixed: values do not depend on threads)
+_THREADS = max(1, min(16, os.cpu_count() or 1))
 
 HIDDEN = 1536
 QKV_OUT = 2048          # 12 query heads + 2 key + 2 value heads, head_dim 128
@@ -45,11 +52,28 @@ LAYER_GEMMS = (
 )
 
 
+def _map_rows(fn, *arrays):
+    """Apply fn(*row_chunks) to fixed row chunks of 2-D arrays, in a thread pool."""
+    rows = arrays[0].shape[0]
+    spans = [(i, min(rows, i + _CHUNK_ROWS)) for i in range(0, rows, _CHUNK_ROWS)]
+    with ThreadPoolExecutor(_THREADS) as ex:
+        list(ex.map(lambda sp: fn(*(a[sp[0]:sp[1]] for a in arrays)), spans))
+
+
 def f32_to_bf16(a: np.ndarray) -> np.ndarray:
     """Round float32 values to bfloat16 (nearest, ties to even); finite input only."""
-    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
-    rounded = u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
-    return (rounded >> np.uint32(16)).astype(np.uint16)
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    out = np.empty(a.shape, np.uint16)
+
+    def conv(src, dst):
+        u = src.view(np.uint32)
+        dst[...] = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
+
+    if a.ndim == 2 and a.shape[0] > _CHUNK_ROWS:
+        _map_rows(conv, a, out)
+    else:
+        conv(a, out)
+    return out
 
 
 def bf16_to_f32(b: np.ndarray) -> np.ndarray:
@@ -58,9 +82,20 @@ def bf16_to_f32(b: np.ndarray) -> np.ndarray:
 
 
 def _normal(rng: np.random.Generator, shape, std: float) -> np.ndarray:
-    x = rng.standard_normal(shape, dtype=np.float32)
-    if std != 1.0:
-        x *= np.float32(std)
+    """N(0, std^2) float32 [rows, cols]; each 1024-row chunk from its own child stream of rng."""
+    rows, cols = shape
+    x = np.empty((rows, cols), np.float32)
+    starts = list(range(0, rows, _CHUNK_ROWS))
+    seeds = np.random.SeedSequence(int(rng.integers(2**63))).spawn(len(starts))
+
+    def fill(i):
+        chunk = x[starts[i]:starts[i] + _CHUNK_ROWS]
+        np.random.default_rng(seeds[i]).standard_normal(chunk.shape, dtype=np.float32, out=chunk)
+        if std != 1.0:
+            chunk *= np.float32(std)
+
+    with ThreadPoolExecutor(_THREADS) as ex:
+        list(ex.map(fill, range(len(starts))))
     return x
 
 
