@@ -163,7 +163,9 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   g.block_n = 0;
   g.err = error_word();
   if (!g.err) return FP8BLK_ERR_CUDA;
+  g.tmem_db = -1;
   if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);
+  if (const char* e = std::getenv("FP8BLK_GEMM_TMEM_DB")) g.tmem_db = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) g.inject_stall = std::atoi(e) != 0;
   return launch_status(fp8blk::launch_gemm(g, static_cast<cudaStream_t>(stream)));
 }

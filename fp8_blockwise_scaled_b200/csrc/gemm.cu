@@ -10,7 +10,7 @@
 // the tensor cores produce one fp32 partial product per K-block and the
 // scales are applied to it before it joins the running sum.
 //
-// Design (one persistent CTA per SM, 320 threads, 128 x BN output tiles):
+// Design (one persistent CTA per SM, 384 threads, 128 x BN output tiles):
 //   warp 0      producer.  Lane 0 issues, per K-block, TMA loads of a 128x128
 //               A tile and a BNx128 B tile (E4M3, 128-byte swizzle) into a
 //               ring of shared-memory stages ("full" mbarrier counts bytes).
@@ -22,10 +22,12 @@
 //               kind::f8f6f4 (M=128, N=BN, K=32) per K-block into one of two
 //               TMEM accumulators (2 x BN fp32 columns), then tcgen05.commit
 //               to release the smem stage and to signal the accumulator.
-//   warps 2..9  promotion + epilogue: two warpgroups, each owning BN/2
+//   warps 2,3   idle: with warps 0 and 1 they form warpgroup 0, which hands
+//               most of its registers to the promotion warpgroups (setmaxnreg).
+//   warps 4..11 promotion + epilogue: two warpgroups, each owning BN/2
 //               columns of the tile (a warp reads the 32 TMEM lanes given by
 //               its index mod 4); per K-block they read the partial product
-//               from TMEM (16-column loads) and fold it into fp32
+//               from TMEM (double-buffered 16-column loads) and fold it into fp32
 //               registers with packed f32x2 FMAs,
 //                   FWD/DGRAD: acc += P * (sa[m] * sb[n-block])
 //                   WGRAD    : acc += (P * sb[n]) * sa[m]
@@ -54,10 +56,21 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 128;
-constexpr int kThreads = 320;
-constexpr int kEpiWarp0 = 2;
 constexpr int kEpiWarps = 8;
 constexpr int kSRing = 8;        // scale ring depth (K-blocks)
+// Two thread layouts.  Plain: 320 threads (producer, MMA issuer, 8 promotion
+// warps), 168 registers each.  Split: 384 threads; warpgroup 0 (producer, MMA
+// issuer, two idle warps) hands registers to the two promotion warpgroups
+// with setmaxnreg, which pays for double-buffered TMEM reads.  The launch
+// allocates 168 per thread (ptxas pins it when setmaxnreg is used).
+constexpr int kLowRegs = 56;
+constexpr int kHighRegs = 224;
+static_assert(128 * kLowRegs + 256 * kHighRegs == 384 * 168, "register split must match the launch allocation");
+template <bool kSplit>
+struct Layout {
+  static constexpr int kThreads = kSplit ? 384 : 320;
+  static constexpr int kEpiWarp0 = kSplit ? 4 : 2;
+};
 
 template <int BN>
 struct Cfg {
@@ -189,11 +202,13 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&v)[8]) {
 
 }  // namespace
 
-template <int BN, bool kWgrad>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, bool kWgrad, bool kSplit>
+__global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     gemm_blockwise_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const GemmParams p) {
   using C = Cfg<BN>;
+  constexpr int kEpiWarp0 = Layout<kSplit>::kEpiWarp0;
+  constexpr bool kTmemDB = kSplit;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + C::kStages * C::kStageBytes);
@@ -237,6 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = ctrl->tmem_base;
   volatile int* abort = &ctrl->abort;
 
+  if (warp < kEpiWarp0) {
+  if constexpr (kSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
   if (warp == 0) {
     // ------------------------------------------------------------ producer (whole warp)
     int stage = 0, slot = 0;
@@ -330,7 +347,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(&ctrl->mma_done);
       mbar_wait_bounded(&ctrl->mma_done, 0, nullptr, p.timeout_ns, p.err);
     }
-  } else if (warp >= kEpiWarp0) {
+  }
+  } else {
+    if constexpr (kSplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
     // ------------------------------------------------------------ promotion + epilogue
     const int ew = warp - kEpiWarp0;  // 0..7
     const int wg = ew >> 2;           // which half of the tile's columns
@@ -361,12 +380,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float f = kWgrad ? 0.0f : sa * ss.sb[BN == 256 ? wg : 0];
         const float* sbc = ss.sb + col0;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * BN + col0;
+        if constexpr (kTmemDB) {
+          // Two 16-column buffers: the load of the next chunk overlaps the FMAs of this one.
+          uint32_t ra[16], rb[16];
+          tmem_ld_32x32b_x16(taddr, ra);
+          tmem_wait_ld16(ra);
 #pragma unroll
-        for (int c = 0; c < C::kHalf; c += 16) {
-          uint32_t r[16];
-          tmem_ld_32x32b_x16(taddr + c, r);
-          tmem_wait_ld16(r);
-          promote16<kWgrad>(acc + c, r, f, sbc + c, sa);
+          for (int c = 0; c < C::kHalf; c += 32) {
+            tmem_ld_32x32b_x16(taddr + c + 16, rb);
+            promote16<kWgrad>(acc + c, ra, f, sbc + c, sa);
+            tmem_wait_ld16(rb);
+            if (c + 32 < C::kHalf) tmem_ld_32x32b_x16(taddr + c + 32, ra);
+            promote16<kWgrad>(acc + c + 16, rb, f, sbc + c + 16, sa);
+            if (c + 32 < C::kHalf) tmem_wait_ld16(ra);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < C::kHalf; c += 16) {
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(taddr + c, r);
+            tmem_wait_ld16(r);
+            promote16<kWgrad>(acc + c, r, f, sbc + c, sa);
+          }
         }
         tc_fence_before_sync();
         __syncwarp();
@@ -440,12 +475,12 @@ int num_sms() {
   return sms;
 }
 
-template <int BN, bool kWgrad>
+template <int BN, bool kWgrad, bool kSplit>
 cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   static bool attr_set = false;
   constexpr int kSmem = smem_bytes<BN>();
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_blockwise_kernel<BN, kWgrad>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_blockwise_kernel<BN, kWgrad, kSplit>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -455,7 +490,7 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall};
   const int64_t tiles = (g.M / BM) * (g.N / BN);
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-  gemm_blockwise_kernel<BN, kWgrad><<<grid, kThreads, kSmem, stream>>>(ta, tb, p);
+  gemm_blockwise_kernel<BN, kWgrad, kSplit><<<grid, Layout<kSplit>::kThreads, kSmem, stream>>>(ta, tb, p);
   return cudaGetLastError();
 }
 
@@ -480,8 +515,18 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   }
   if (bn == 256 && g.N % 256 != 0) return cudaErrorInvalidValue;
   const bool wgrad = g.layout == 2;
-  if (bn == 256) return wgrad ? launch_variant<256, true>(g, stream) : launch_variant<256, false>(g, stream);
-  if (bn == 128) return wgrad ? launch_variant<128, true>(g, stream) : launch_variant<128, false>(g, stream);
+  // The register split with double-buffered TMEM reads pays off where the
+  // promotion does more work per column (WGRAD); measured on B200, the plain
+  // layout is faster for the forward/data-gradient promotion.
+  const bool db = g.tmem_db < 0 ? wgrad : g.tmem_db != 0;
+  if (bn == 256) {
+    if (wgrad) return db ? launch_variant<256, true, true>(g, stream) : launch_variant<256, true, false>(g, stream);
+    return db ? launch_variant<256, false, true>(g, stream) : launch_variant<256, false, false>(g, stream);
+  }
+  if (bn == 128) {
+    if (wgrad) return db ? launch_variant<128, true, true>(g, stream) : launch_variant<128, true, false>(g, stream);
+    return db ? launch_variant<128, false, true>(g, stream) : launch_variant<128, false, false>(g, stream);
+  }
   return cudaErrorInvalidValue;
 }
 

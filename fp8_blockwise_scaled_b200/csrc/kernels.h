@@ -33,6 +33,7 @@ struct GemmArgs {
   uint64_t timeout_ns;        // bound on every device-side wait
   int inject_stall;           // test hook: the MMA issuer waits on a barrier nothing completes
   int block_n;                // 0 = choose, else 128 or 256
+  int tmem_db;                // -1 = choose, 0/1 = single/double-buffered TMEM reads
   unsigned int* err;          // device error word
 };
 

@@ -68,47 +68,32 @@ __device__ __forceinline__ QScale make_qscale(float amax) {
   return {s, rc * (1.0f - 0x1p-20f), rc * (1.0f + 0x1p-20f)};
 }
 
-// Two values -> two E4M3 codes, `a` in the low byte.
-__device__ __forceinline__ uint32_t cvt2(float a, float b) {
-  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
-}
-
-// (a0, a1) * (b, b) with one packed multiply.
-__device__ __forceinline__ float2 mul2(float a0, float a1, float b) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %4};\n\t"
-      "mul.rn.f32x2 rd, ra, rb;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a0), "f"(a1), "f"(b));
-  return d;
-}
-
-__device__ __noinline__ uint2 quant8_slow(float x0, float x1, float x2, float x3, float x4, float x5, float x6,
-                                          float x7, float s) {
-  uint2 out;
-  out.x = cvt2(__fdiv_rn(x0, s), __fdiv_rn(x1, s)) | (cvt2(__fdiv_rn(x2, s), __fdiv_rn(x3, s)) << 16);
-  out.y = cvt2(__fdiv_rn(x4, s), __fdiv_rn(x5, s)) | (cvt2(__fdiv_rn(x6, s), __fdiv_rn(x7, s)) << 16);
-  return out;
+// Four values -> four E4M3 codes packed little-endian (x0 in the lowest byte):
+// two paired conversions (the second source goes to the low byte) and one move.
+__device__ __forceinline__ uint32_t cvt4(float x0, float x1, float x2, float x3) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 l, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h, %4, %3;\n\t"
+      "mov.b32 %0, {l, h};\n\t}"
+      : "=r"(r)
+      : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
+  return r;
 }
 
 // Eight values -> eight codes packed little-endian (x[0] in the lowest byte).
 __device__ __forceinline__ uint2 quant8(const float (&x)[8], const QScale& q) {
-  uint32_t lo[4], hi[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float2 l = mul2(x[2 * j], x[2 * j + 1], q.rlo);
-    const float2 h = mul2(x[2 * j], x[2 * j + 1], q.rhi);
-    lo[j] = cvt2(l.x, l.y);
-    hi[j] = cvt2(h.x, h.y);
+  const float lo = q.rlo, hi = q.rhi;
+  uint32_t l0 = cvt4(x[0] * lo, x[1] * lo, x[2] * lo, x[3] * lo);
+  uint32_t l1 = cvt4(x[4] * lo, x[5] * lo, x[6] * lo, x[7] * lo);
+  const uint32_t h0 = cvt4(x[0] * hi, x[1] * hi, x[2] * hi, x[3] * hi);
+  const uint32_t h1 = cvt4(x[4] * hi, x[5] * hi, x[6] * hi, x[7] * hi);
+  if (__builtin_expect(((l0 ^ h0) | (l1 ^ h1)) != 0, 0)) {
+    // The bracket straddles a rounding boundary: use the correctly rounded quotient.
+    l0 = cvt4(__fdiv_rn(x[0], q.s), __fdiv_rn(x[1], q.s), __fdiv_rn(x[2], q.s), __fdiv_rn(x[3], q.s));
+    l1 = cvt4(__fdiv_rn(x[4], q.s), __fdiv_rn(x[5], q.s), __fdiv_rn(x[6], q.s), __fdiv_rn(x[7], q.s));
   }
-  const uint32_t lo0 = lo[0] | (lo[1] << 16), lo1 = lo[2] | (lo[3] << 16);
-  const uint32_t hi0 = hi[0] | (hi[1] << 16), hi1 = hi[2] | (hi[3] << 16);
-  if (__builtin_expect(((lo0 ^ hi0) | (lo1 ^ hi1)) != 0, 0))
-    return quant8_slow(x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7], q.s);
-  return make_uint2(lo0, lo1);
+  return make_uint2(l0, l1);
 }
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
@@ -125,13 +110,6 @@ __device__ __forceinline__ float absmax8(const uint4& v) {
   uint32_t a = __vmaxu2(__vmaxu2(v.x & kAbs2, v.y & kAbs2), __vmaxu2(v.z & kAbs2, v.w & kAbs2));
   a = max(a & 0xFFFFu, a >> 16);
   return __uint_as_float(a << 16);
-}
-
-__device__ __forceinline__ void load_tile(uint4 (&v)[8], const QuantArgs& a, int64_t tile, int rbase, int chunk) {
-  const int64_t tr = tile % a.tiles_r, tc = tile / a.tiles_r;
-  const uint16_t* base = a.x + (tr * kTile + rbase) * a.ldx + tc * kTile + chunk * 8;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = ld_nc_v4(base + 16 * i * a.ldx);
 }
 
 }  // namespace
@@ -157,14 +135,20 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
   const int chunk = t & 15;      // this thread's 16-byte column chunk of the tile
   const int rbase = t >> 4;      // rows rbase + 16 i, i = 0..7
   const int64_t tiles = a.tiles_r * a.tiles_c;
+  const uint32_t ldx = static_cast<uint32_t>(a.ldx);
+  const uint32_t cols = static_cast<uint32_t>(a.cols);
+  const uint32_t rows = static_cast<uint32_t>(a.rows);
 
-  uint4 v[8];
-  int64_t tile = blockIdx.x;
-  if (tile < tiles) load_tile(v, a, tile, rbase, chunk);
-
-  for (; tile < tiles; tile += gridDim.x) {
+  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
     const int64_t tr = tile % a.tiles_r, tc = tile / a.tiles_r;
     const int64_t row0 = tr * kTile, col0 = tc * kTile;
+
+    uint4 v[8];
+    {
+      const uint16_t* src = a.x + row0 * a.ldx + col0 + rbase * ldx + chunk * 8;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = ld_nc_v4(src + 16u * i * ldx);
+    }
 
     // ---------------------------------------------------------------- from registers
     QScale qblk{};
@@ -186,12 +170,17 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
       }
     }
 
-    if constexpr (kRow || kBlk) {
+    // Row groups (or the whole block) in place: chunk i of this thread is rows
+    // rbase + 16 i, columns chunk*8 .. +7 of the tile.
+    auto quant_in_place = [&](auto chunk_of) {
+      uint8_t* qdst = a.q_row + row0 * a.cols + col0 + rbase * cols + chunk * 8;
+      [[maybe_unused]] float* sdst = kRow ? a.s_row + tc * a.rows + row0 + rbase : nullptr;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
+        const uint4 vi = chunk_of(i);
         QScale q;
         if constexpr (kRow) {
-          float amax = absmax8(v[i]);
+          float amax = absmax8(vi);
 #pragma unroll
           for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
           q = make_qscale(amax);
@@ -199,14 +188,14 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
           q = qblk;
         }
         float f[8];
-        unpack8(v[i], f);
-        const int64_t r = row0 + rbase + 16 * i;
-        *reinterpret_cast<uint2*>(a.q_row + r * a.cols + col0 + chunk * 8) = quant8(f, q);
+        unpack8(vi, f);
+        *reinterpret_cast<uint2*>(qdst + 16u * i * cols) = quant8(f, q);
         if constexpr (kRow) {
-          if (chunk == 0) a.s_row[tc * a.rows + r] = q.s;
+          if (chunk == 0) sdst[16 * i] = q.s;
         }
       }
-    }
+    };
+    if constexpr ((kRow || kBlk) && !kTileSmem) quant_in_place([&](int i) { return v[i]; });
 
     if constexpr (kTileSmem) {
 #pragma unroll
@@ -226,23 +215,20 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
         for (int j = 0; j < 4; ++j) m[j] = __vmaxu2(m[j], __shfl_xor_sync(0xFFFFFFFFu, m[j], 16));
         if (lane < 16) *reinterpret_cast<uint4*>(cpart + warp * 64 + chunk * 4) = make_uint4(m[0], m[1], m[2], m[3]);
       }
-    }
-
-    // Registers are free: start loading the next tile while the shared-memory work runs.
-    if (tile + gridDim.x < tiles) load_tile(v, a, tile + gridDim.x, rbase, chunk);
-
-    if constexpr (kTileSmem) {
       __syncthreads();
+      // With the tile in shared memory the in-place codes are made from there,
+      // so the input registers are free for the transposed pass.
+      if constexpr (kRow || kBlk)
+        quant_in_place([&](int i) { return *reinterpret_cast<const uint4*>(xs + (rbase + 16 * i) * 256 + chunk * 16); });
       if constexpr (kColT) {
-        if (t < 64) {  // word t covers columns 2t and 2t+1
+        if (t < kTile) {  // one column per thread
           uint32_t mx = 0;
 #pragma unroll
-          for (int w = 0; w < 8; ++w) mx = __vmaxu2(mx, cpart[w * 64 + t]);
-          const QScale q0 = make_qscale(__uint_as_float(mx << 16));
-          const QScale q1 = make_qscale(__uint_as_float(mx & 0xFFFF0000u));
-          qs[2 * t] = make_float4(q0.s, q0.rlo, q0.rhi, 0.f);
-          qs[2 * t + 1] = make_float4(q1.s, q1.rlo, q1.rhi, 0.f);
-          *reinterpret_cast<float2*>(a.s_t + tr * a.cols + col0 + 2 * t) = make_float2(q0.s, q1.s);
+          for (int w = 0; w < 8; ++w) mx = __vmaxu2(mx, cpart[w * 64 + (t >> 1)]);
+          const float am = __uint_as_float((t & 1) ? (mx & 0xFFFF0000u) : (mx << 16));
+          const QScale q = make_qscale(am);
+          qs[t] = make_float4(q.s, q.rlo, q.rhi, 0.f);
+          a.s_t[tr * a.cols + col0 + t] = q.s;
         }
         __syncthreads();
       }
@@ -278,12 +264,13 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
         *reinterpret_cast<uint4*>(cs + (2 * cp + 1) * 128 + phys) = make_uint4(b0.x, b0.y, b1.x, b1.y);
       }
       __syncthreads();
+      uint8_t* tdst = a.q_t + col0 * a.rows + row0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int k = t + kThreads * j;
         const int c = k >> 3, part = k & 7;
         const uint4 codes = *reinterpret_cast<const uint4*>(cs + c * 128 + ((part ^ ((c >> 1) & 7)) * 16));
-        *reinterpret_cast<uint4*>(a.q_t + (col0 + c) * a.rows + row0 + part * 16) = codes;
+        *reinterpret_cast<uint4*>(tdst + c * rows + part * 16) = codes;
       }
     }
     if constexpr (kTileSmem || kBlockScale) __syncthreads();  // shared memory is reused by the next tile
