@@ -24,16 +24,17 @@
 // magnitude, so the 2^15 possible inputs were checked exhaustively against
 // the correctly rounded quotient (tests/test_scale_division.py).
 //
-// Exactness of x / s.  A correctly rounded binary32 division per element
-// costs more issue slots than the HBM budget allows, so each value is
-// bracketed instead: with r ~ 1/s (hardware approximation, relative error
-// below 2^-22), lo = x*fl(r(1-2^-20)) and hi = x*fl(r(1+2^-20)) satisfy
-// |lo| <= |fl(x/s)| <= |hi| (all the roundings together move the product by
-// less than 2^-21 relative, inside the 2^-20 margin).  Rounding to E4M3 is
-// monotonic, so when lo and hi give the same code that code is the one of
-// fl(x/s); otherwise (about one value in 2^15) the value is recomputed with
-// the correctly rounded division.  The saturating conversion equals
-// clamp-then-round because every value above 448 rounds or saturates to 448.
+// Exactness of x / s.  Each quotient is computed exactly with Markstein's
+// FMA correction (P. Markstein, "Computation of elementary functions on the
+// IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with
+// r = RN(1/s) (the correctly rounded reciprocal, once per group) and
+// q = RN(x*r), which is within one ulp of x/s, the residual x - q*s is exact
+// in one FMA and RN(q + (x - q*s)*r) is the correctly rounded quotient.  The
+// kernel evaluates the negated form w = -RN(x/s) with packed f32x2
+// instructions and flips the sign bits of the codes afterwards, which also
+// gives -0 -> 0x80 and +0 -> 0x00.  No branch, no data-dependent cost.  The
+// saturating conversion equals clamp-then-round because every value above
+// 448 rounds or saturates to 448.
 #include <cuda_fp8.h>
 
 #include "device.cuh"
@@ -49,12 +50,13 @@ constexpr int kThreads = 256;
 constexpr int kXsBytes = kTile * kTile * 2;       // bf16 tile, 256-byte rows
 constexpr int kCsBytes = kTile * kTile;           // transposed codes, 128-byte rows, 16-B chunks swizzled
 constexpr int kCpartBytes = 8 * 64 * 4;           // per-warp packed column maxima
-constexpr int kQsBytes = kTile * 16;              // per-column {s, r_lo, r_hi}
+constexpr int kQsBytes = kTile * 8;               // per-column {s, -1/s}
 constexpr int kSmallBytes = 64;                   // per-warp block maxima
 constexpr int kSmemBytes = kSmallBytes + kQsBytes + kCpartBytes + kXsBytes + kCsBytes;
 
 struct QScale {
-  float s, rlo, rhi;
+  float s;    // the group's scale
+  float nr;   // -RN(1/s)
 };
 
 __device__ __forceinline__ QScale make_qscale(float amax) {
@@ -63,9 +65,7 @@ __device__ __forceinline__ QScale make_qscale(float amax) {
   const float q0 = y * c7;
   const float r = fmaf(-7.0f, q0, y);
   const float s = fmaxf(fmaf(r, c7, q0), 1e-12f);
-  float rc;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(s));
-  return {s, rc * (1.0f - 0x1p-20f), rc * (1.0f + 0x1p-20f)};
+  return {s, -__frcp_rn(s)};
 }
 
 // Four values -> four E4M3 codes packed little-endian (x0 in the lowest byte):
@@ -81,19 +81,27 @@ __device__ __forceinline__ uint32_t cvt4(float x0, float x1, float x2, float x3)
   return r;
 }
 
+// (w0, w1) = -RN((x0, x1) / s) with nr = -RN(1/s): qn = x*nr, e = qn*s + x
+// (exact), w = e*nr + qn.
+__device__ __forceinline__ void neg_quotient2(float& w0, float& w1, float x0, float x1, float s, float nr) {
+  asm("{\n\t.reg .b64 x, qn, e, ss, rr, w;\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 ss, {%4, %4};\n\t"
+      "mov.b64 rr, {%5, %5};\n\t"
+      "mul.rn.f32x2 qn, x, rr;\n\t"
+      "fma.rn.f32x2 e, qn, ss, x;\n\t"
+      "fma.rn.f32x2 w, e, rr, qn;\n\t"
+      "mov.b64 {%0, %1}, w;\n\t}"
+      : "=f"(w0), "=f"(w1)
+      : "f"(x0), "f"(x1), "f"(s), "f"(nr));
+}
+
 // Eight values -> eight codes packed little-endian (x[0] in the lowest byte).
 __device__ __forceinline__ uint2 quant8(const float (&x)[8], const QScale& q) {
-  const float lo = q.rlo, hi = q.rhi;
-  uint32_t l0 = cvt4(x[0] * lo, x[1] * lo, x[2] * lo, x[3] * lo);
-  uint32_t l1 = cvt4(x[4] * lo, x[5] * lo, x[6] * lo, x[7] * lo);
-  const uint32_t h0 = cvt4(x[0] * hi, x[1] * hi, x[2] * hi, x[3] * hi);
-  const uint32_t h1 = cvt4(x[4] * hi, x[5] * hi, x[6] * hi, x[7] * hi);
-  if (__builtin_expect(((l0 ^ h0) | (l1 ^ h1)) != 0, 0)) {
-    // The bracket straddles a rounding boundary: use the correctly rounded quotient.
-    l0 = cvt4(__fdiv_rn(x[0], q.s), __fdiv_rn(x[1], q.s), __fdiv_rn(x[2], q.s), __fdiv_rn(x[3], q.s));
-    l1 = cvt4(__fdiv_rn(x[4], q.s), __fdiv_rn(x[5], q.s), __fdiv_rn(x[6], q.s), __fdiv_rn(x[7], q.s));
-  }
-  return make_uint2(l0, l1);
+  float w[8];
+#pragma unroll
+  for (int j = 0; j < 8; j += 2) neg_quotient2(w[j], w[j + 1], x[j], x[j + 1], q.s, q.nr);
+  return make_uint2(cvt4(w[0], w[1], w[2], w[3]) ^ 0x80808080u, cvt4(w[4], w[5], w[6], w[7]) ^ 0x80808080u);
 }
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
@@ -125,7 +133,7 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
 
   extern __shared__ __align__(16) uint8_t smem[];
   float* warpmax = reinterpret_cast<float*>(smem);                                      // [8]
-  float4* qs = reinterpret_cast<float4*>(smem + kSmallBytes);                           // [128] column scales
+  float2* qs = reinterpret_cast<float2*>(smem + kSmallBytes);                           // [128] column scales
   uint32_t* cpart = reinterpret_cast<uint32_t*>(smem + kSmallBytes + kQsBytes);         // [8][64]
   uint8_t* xs = smem + kSmallBytes + kQsBytes + kCpartBytes;                            // [128][256 B]
   uint8_t* cs = xs + kXsBytes;                                                          // [128][128 B]
@@ -175,18 +183,20 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
     auto quant_in_place = [&](auto chunk_of) {
       uint8_t* qdst = a.q_row + row0 * a.cols + col0 + rbase * cols + chunk * 8;
       [[maybe_unused]] float* sdst = kRow ? a.s_row + tc * a.rows + row0 + rbase : nullptr;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint4 vi = chunk_of(i);
-        QScale q;
+      auto scale_of = [&](const uint4& vi) {
         if constexpr (kRow) {
           float amax = absmax8(vi);
 #pragma unroll
           for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-          q = make_qscale(amax);
+          return make_qscale(amax);
         } else {
-          q = qblk;
+          return qblk;
         }
+      };
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 vi = chunk_of(i);
+        const QScale q = scale_of(vi);
         float f[8];
         unpack8(vi, f);
         *reinterpret_cast<uint2*>(qdst + 16u * i * cols) = quant8(f, q);
@@ -195,7 +205,9 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
         }
       }
     };
-    if constexpr ((kRow || kBlk) && !kTileSmem) quant_in_place([&](int i) { return v[i]; });
+    if constexpr ((kRow || kBlk) && !kTileSmem) {
+      quant_in_place([&](int i) { return v[i]; });
+    }
 
     if constexpr (kTileSmem) {
 #pragma unroll
@@ -218,8 +230,10 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
       __syncthreads();
       // With the tile in shared memory the in-place codes are made from there,
       // so the input registers are free for the transposed pass.
-      if constexpr (kRow || kBlk)
-        quant_in_place([&](int i) { return *reinterpret_cast<const uint4*>(xs + (rbase + 16 * i) * 256 + chunk * 16); });
+      if constexpr (kRow || kBlk) {
+        auto from_smem = [&](int i) { return *reinterpret_cast<const uint4*>(xs + (rbase + 16 * i) * 256 + chunk * 16); };
+        quant_in_place(from_smem);
+      }
       if constexpr (kColT) {
         if (t < kTile) {  // one column per thread
           uint32_t mx = 0;
@@ -227,7 +241,7 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
           for (int w = 0; w < 8; ++w) mx = __vmaxu2(mx, cpart[w * 64 + (t >> 1)]);
           const float am = __uint_as_float((t & 1) ? (mx & 0xFFFF0000u) : (mx << 16));
           const QScale q = make_qscale(am);
-          qs[t] = make_float4(q.s, q.rlo, q.rhi, 0.f);
+          qs[t] = make_float2(q.s, q.nr);
           a.s_t[tr * a.cols + col0 + t] = q.s;
         }
         __syncthreads();
@@ -236,18 +250,19 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
       // of a warp read consecutive words of the same smem rows (conflict-free) and
       // write 16-byte chunks whose position is XOR-swizzled by cp (conflict-free).
       const uint32_t* xs32 = reinterpret_cast<const uint32_t*>(xs);
+      auto col_scale = [&](int c) {
+        if constexpr (kColT) {
+          const float2 fq = qs[c];
+          return QScale{fq.x, fq.y};
+        } else {
+          return qblk;
+        }
+      };
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int item = t + kThreads * j;
         const int cp = item & 63, rc = item >> 6;
-        QScale qa, qb;
-        if constexpr (kColT) {
-          const float4 fa = qs[2 * cp], fb = qs[2 * cp + 1];
-          qa = {fa.x, fa.y, fa.z};
-          qb = {fb.x, fb.y, fb.z};
-        } else {
-          qa = qb = qblk;
-        }
+        const QScale qa = col_scale(2 * cp), qb = col_scale(2 * cp + 1);
         float lo[16], hi[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {

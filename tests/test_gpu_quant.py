@@ -88,10 +88,10 @@ def test_special_blocks():
     _check_weight(x, "special")
 
 
-def test_rounding_ties_take_the_exact_path():
+def test_rounding_ties():
     # Groups with amax 448 (scale exactly 1) whose other values sit exactly on
-    # E4M3 rounding ties, so the reciprocal bracket cannot decide and the
-    # correctly rounded division has to.
+    # E4M3 rounding ties: the quotient must be exact for round-to-nearest-even
+    # to pick the even neighbour.
     ties = np.array([17.0, 19.0, 2.0**-10, 3 * 2.0**-10, 432.0, 424.0, 9.25, 0.0087890625], np.float32)
     rng = np.random.default_rng(8)
     x = rng.choice(np.concatenate([ties, -ties]), size=(256, 256)).astype(np.float32)
@@ -116,3 +116,21 @@ def test_full_mlp_fwd():
 
 def test_full_down_bwd_grad():
     _check_act(workloads.down_bwd(seed=3)["dY"], fb.BOTH, "dY 8192x1536")
+
+
+def test_adversarial_quotients():
+    # Every group's amax is 448*2^k (scale exactly 2^k: many quotients sit exactly on
+    # E4M3 rounding ties) or 1.0 (scale 1/448 rounded: many near-ties); the other values
+    # are random bf16 bit patterns below the amax, bf16 subnormals included.
+    rng = np.random.default_rng(99)
+    rows, cols = 512, 1024
+    amax_choices = np.array([0x43E0, 0x3FE0, 0x47E0, 0x3BE0, 0x3F80], np.uint16)
+    x = np.empty((rows, cols), np.uint16)
+    for r in range(rows):
+        for g in range(cols // 128):
+            a = int(rng.choice(amax_choices))
+            vals = rng.integers(0, a + 1, size=128).astype(np.uint16) | (rng.integers(0, 2, size=128) << 15).astype(np.uint16)
+            vals[rng.integers(0, 128)] = a
+            x[r, g * 128:(g + 1) * 128] = vals
+    _check_act(x, fb.BOTH, "adversarial act")
+    _check_weight(x, "adversarial weight")
