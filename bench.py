@@ -172,9 +172,8 @@ class Program:
             if events is not None:
                 events[i][1].record()
         if self.world > 1:
-            import torch.distributed as dist
-            for g in self.grads:
-                dist.all_reduce(g)
+            from fp8_blockwise_scaled_b200.dp import allreduce_weight_grads
+            allreduce_weight_grads(self.grads)
 
 
 # --------------------------------------------------------------------------- clocks

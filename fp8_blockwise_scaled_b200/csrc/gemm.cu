@@ -78,7 +78,10 @@ struct Cfg {
   static constexpr int kABytes = BM * BK;
   static constexpr int kBBytes = BN * BK;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kTmemCols = 2 * BN;
+  // TMEM accumulators: 2 x 256 columns for BN=256; 4 x 128 for BN=128, so
+  // that the MMA can run three K-blocks ahead of the promotion.
+  static constexpr int kAccBufs = (BN == 256) ? 2 : 4;
+  static constexpr int kTmemCols = kAccBufs * BN;
   static constexpr int kHalf = BN / 2;  // columns per epilogue warpgroup
 };
 
@@ -91,8 +94,8 @@ struct ScaleSlot {
 struct Ctrl {
   uint64_t full[8];
   uint64_t empty[8];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t tfull[4];
+  uint64_t tempty[4];
   uint64_t sfull[kSRing];
   uint64_t sempty[kSRing];
   uint64_t mma_done;
@@ -157,40 +160,52 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
-// acc(2) += p(2) * f   (packed, one instruction for two columns)
-__device__ __forceinline__ void ffma2_scalar(float& a0, float& a1, uint32_t p0, uint32_t p1, float f) {
-  asm("{\n\t.reg .b64 ra, rp, rf;\n\t"
-      "mov.b64 ra, {%0, %1};\n\t"
-      "mov.b64 rp, {%2, %3};\n\t"
-      "mov.b64 rf, {%4, %4};\n\t"
-      "fma.rn.f32x2 ra, rp, rf, ra;\n\t"
-      "mov.b64 {%0, %1}, ra;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "r"(p0), "r"(p1), "f"(f));
+__device__ __forceinline__ void tmem_ld_32x32b_x64(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
 }
 
-// acc(2) += (p(2) * sb(2)) * sa
-__device__ __forceinline__ void ffma2_cols(float& a0, float& a1, uint32_t p0, uint32_t p1, float2 sb, float sa) {
-  asm("{\n\t.reg .b64 ra, rp, rb, rs;\n\t"
-      "mov.b64 ra, {%0, %1};\n\t"
-      "mov.b64 rp, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %5};\n\t"
-      "mov.b64 rs, {%6, %6};\n\t"
-      "mul.rn.f32x2 rp, rp, rb;\n\t"
-      "fma.rn.f32x2 ra, rp, rs, ra;\n\t"
-      "mov.b64 {%0, %1}, ra;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "r"(p0), "r"(p1), "f"(sb.x), "f"(sb.y), "f"(sa));
+// tcgen05.wait::ld tied to all 64 registers of a 64-column load.
+__device__ __forceinline__ void tmem_wait_ld64(uint32_t (&r)[64]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                 "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]),
+                 "+r"(r[32]), "+r"(r[33]), "+r"(r[34]), "+r"(r[35]), "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]),
+                 "+r"(r[40]), "+r"(r[41]), "+r"(r[42]), "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]),
+                 "+r"(r[48]), "+r"(r[49]), "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]),
+                 "+r"(r[56]), "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]), "+r"(r[63])
+               :
+               : "memory");
 }
 
+// Promotion of 16 columns of one row with packed f32x2 FMAs:
+//   FWD/DGRAD: acc += P * f           (f = sa[m] * sb[n-block])
+//   WGRAD    : acc += (P * sb[n]) * sa[m]
 template <bool kWgrad>
-__device__ __forceinline__ void promote16(float* acc, const uint32_t (&r)[16], float f, const float* sbc, float sa) {
+__device__ __forceinline__ void promote16(float2* acc, const uint32_t (&r)[16], float f, const float* sbc, float sa) {
+  const float2 f2 = make_float2(f, f), sa2 = make_float2(sa, sa);
 #pragma unroll
-  for (int j = 0; j < 16; j += 2) {
+  for (int j = 0; j < 8; ++j) {
+    const float2 pj = make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
     if constexpr (kWgrad)
-      ffma2_cols(acc[j], acc[j + 1], r[j], r[j + 1], *reinterpret_cast<const float2*>(sbc + j), sa);
+      acc[j] = __ffma2_rn(__fmul2_rn(pj, *reinterpret_cast<const float2*>(sbc + 2 * j)), sa2, acc[j]);
     else
-      ffma2_scalar(acc[j], acc[j + 1], r[j], r[j + 1], f);
+      acc[j] = __ffma2_rn(pj, f2, acc[j]);
   }
 }
 
@@ -209,6 +224,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
   using C = Cfg<BN>;
   constexpr int kEpiWarp0 = Layout<kSplit>::kEpiWarp0;
   constexpr bool kTmemDB = kSplit;
+  constexpr bool kWide = kSplit;  // the split layout has the registers for 64-column TMEM reads
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + C::kStages * C::kStageBytes);
@@ -225,7 +241,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
       mbar_init(&ctrl->full[s], 1);
       mbar_init(&ctrl->empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&ctrl->tfull[b], 1);
       mbar_init(&ctrl->tempty[b], kEpiWarps);
     }
@@ -339,8 +355,10 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
             stage = 0;
             phase ^= 1u;
           }
-          abuf ^= 1u;
-          if (abuf == 0) aphase ^= 1u;
+          if (++abuf == C::kAccBufs) {
+            abuf = 0;
+            aphase ^= 1u;
+          }
         }
       }
       // Every MMA issued so far has finished once this arrives.
@@ -358,14 +376,14 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     const int col0 = wg * C::kHalf;
     uint32_t abuf = 0, aphase = 0, sphase = 0;
     int slot = 0;
-    float acc[C::kHalf];
+    float2 acc[C::kHalf / 2];
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
       const int mb = tile % num_mb, nb = tile / num_mb;
       const int64_t m = static_cast<int64_t>(mb) * BM + row;
       const int64_t ncol0 = static_cast<int64_t>(nb) * BN + col0;
 #pragma unroll
-      for (int j = 0; j < C::kHalf; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < C::kHalf / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
 
       for (int kb = 0; kb < kblocks; ++kb) {
         const bool got = mbar_wait_bounded(&ctrl->sfull[slot], sphase, abort, p.timeout_ns, p.err) &&
@@ -380,7 +398,34 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
         const float f = kWgrad ? 0.0f : sa * ss.sb[BN == 256 ? wg : 0];
         const float* sbc = ss.sb + col0;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * BN + col0;
-        if constexpr (kTmemDB) {
+        if constexpr (C::kHalf == 64) {
+          // 64 columns per thread: all four loads in flight, one wait.
+          uint32_t r0[16], r1[16], r2[16], r3[16];
+          tmem_ld_32x32b_x16(taddr, r0);
+          tmem_ld_32x32b_x16(taddr + 16, r1);
+          tmem_ld_32x32b_x16(taddr + 32, r2);
+          tmem_ld_32x32b_x16(taddr + 48, r3);
+          tmem_wait_ld16(r0);
+          tmem_wait_ld16(r1);
+          tmem_wait_ld16(r2);
+          tmem_wait_ld16(r3);
+          promote16<kWgrad>(acc, r0, f, sbc, sa);
+          promote16<kWgrad>(acc + 8, r1, f, sbc + 16, sa);
+          promote16<kWgrad>(acc + 16, r2, f, sbc + 32, sa);
+          promote16<kWgrad>(acc + 24, r3, f, sbc + 48, sa);
+        } else if constexpr (kTmemDB && kWide) {
+          // 64-column loads: two TMEM round trips per K-block for 128 columns.
+#pragma unroll
+          for (int c = 0; c < C::kHalf; c += 64) {
+            uint32_t r[64];
+            tmem_ld_32x32b_x64(taddr + c, r);
+            tmem_wait_ld64(r);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              promote16<kWgrad>(acc + c / 2 + 8 * q, *reinterpret_cast<const uint32_t(*)[16]>(r + 16 * q), f,
+                                sbc + c + 16 * q, sa);
+          }
+        } else if constexpr (kTmemDB) {
           // Two 16-column buffers: the load of the next chunk overlaps the FMAs of this one.
           uint32_t ra[16], rb[16];
           tmem_ld_32x32b_x16(taddr, ra);
@@ -388,10 +433,10 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < C::kHalf; c += 32) {
             tmem_ld_32x32b_x16(taddr + c + 16, rb);
-            promote16<kWgrad>(acc + c, ra, f, sbc + c, sa);
+            promote16<kWgrad>(acc + c / 2, ra, f, sbc + c, sa);
             tmem_wait_ld16(rb);
             if (c + 32 < C::kHalf) tmem_ld_32x32b_x16(taddr + c + 32, ra);
-            promote16<kWgrad>(acc + c + 16, rb, f, sbc + c + 16, sa);
+            promote16<kWgrad>(acc + c / 2 + 8, rb, f, sbc + c + 16, sa);
             if (c + 32 < C::kHalf) tmem_wait_ld16(ra);
           }
         } else {
@@ -400,7 +445,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
             uint32_t r[16];
             tmem_ld_32x32b_x16(taddr + c, r);
             tmem_wait_ld16(r);
-            promote16<kWgrad>(acc + c, r, f, sbc + c, sa);
+            promote16<kWgrad>(acc + c / 2, r, f, sbc + c, sa);
           }
         }
         tc_fence_before_sync();
@@ -409,8 +454,10 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
           mbar_arrive(&ctrl->tempty[abuf]);
           mbar_arrive(&ctrl->sempty[slot]);
         }
-        abuf ^= 1u;
-        if (abuf == 0) aphase ^= 1u;
+        if (++abuf == C::kAccBufs) {
+          abuf = 0;
+          aphase ^= 1u;
+        }
         if (++slot == kSRing) {
           slot = 0;
           sphase ^= 1u;
@@ -422,7 +469,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
       for (int j = 0; j < C::kHalf; j += 16) {
         uint32_t v[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = pack_bf16x2(acc[j + 2 * q], acc[j + 2 * q + 1]);
+        for (int q = 0; q < 8; ++q) v[q] = pack_bf16x2(acc[j / 2 + q].x, acc[j / 2 + q].y);
         st_global_v8(drow + j, v);
       }
     }

@@ -82,18 +82,14 @@ __device__ __forceinline__ uint32_t cvt4(float x0, float x1, float x2, float x3)
 }
 
 // (w0, w1) = -RN((x0, x1) / s) with nr = -RN(1/s): qn = x*nr, e = qn*s + x
-// (exact), w = e*nr + qn.
+// (exact), w = e*nr + qn, in packed f32x2 arithmetic.
 __device__ __forceinline__ void neg_quotient2(float& w0, float& w1, float x0, float x1, float s, float nr) {
-  asm("{\n\t.reg .b64 x, qn, e, ss, rr, w;\n\t"
-      "mov.b64 x, {%2, %3};\n\t"
-      "mov.b64 ss, {%4, %4};\n\t"
-      "mov.b64 rr, {%5, %5};\n\t"
-      "mul.rn.f32x2 qn, x, rr;\n\t"
-      "fma.rn.f32x2 e, qn, ss, x;\n\t"
-      "fma.rn.f32x2 w, e, rr, qn;\n\t"
-      "mov.b64 {%0, %1}, w;\n\t}"
-      : "=f"(w0), "=f"(w1)
-      : "f"(x0), "f"(x1), "f"(s), "f"(nr));
+  const float2 x = make_float2(x0, x1), s2 = make_float2(s, s), nr2 = make_float2(nr, nr);
+  const float2 qn = __fmul2_rn(x, nr2);
+  const float2 e = __ffma2_rn(qn, s2, x);
+  const float2 w = __ffma2_rn(e, nr2, qn);
+  w0 = w.x;
+  w1 = w.y;
 }
 
 // Eight values -> eight codes packed little-endian (x[0] in the lowest byte).

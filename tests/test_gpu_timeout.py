@@ -1,0 +1,54 @@
+"""Failure detection on the GPU without a fault: the GEMM's bounded waits.
+
+A test hook makes the MMA issuer wait on a barrier that nothing completes.
+With a 200 ms bound every role of the kernel must give up, drain its own
+copies, free its tensor memory and return; the host then reads
+FP8BLK_ERR_TIMEOUT from the device error word, and the context must still
+run a normal GEMM correctly."""
+import numpy as np
+import pytest
+import torch
+
+import fp8_blockwise_scaled_b200 as fb
+import oracle
+import workloads
+from tests.gpu_helpers import assert_gemm_close, require_cuda
+
+pytestmark = pytest.mark.gpu
+
+TIMEOUT_STATUS = 6
+
+
+def _operands(layout):
+    rng = np.random.default_rng(11)
+    if layout == fb.WGRAD:
+        dy = workloads.grad_output(rng, 512, 256)
+        x = workloads.swiglu_like(rng, 512, 256)
+        qa, sa = oracle.quantize_act_colwise_t(dy)
+        qb, sb = oracle.quantize_act_colwise_t(x)
+    else:
+        x = workloads.activation(rng, 512, 512)
+        w = workloads.weight(rng, 256, 512)
+        qa, sa = oracle.quantize_act_rowwise(x)
+        qb, sb = oracle.quantize_weight(w)
+    return qa, sa, qb, sb
+
+
+@pytest.mark.parametrize("layout", [0, 2])   # both thread layouts of the GEMM kernel
+def test_stalled_gemm_reports_timeout_and_recovers(layout, monkeypatch):
+    require_cuda()
+    qa, sa, qb, sb = _operands(layout)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
+    A, B = dev(qa).view(torch.float8_e4m3fn), dev(qb).view(torch.float8_e4m3fn)
+    SA, SB = dev(sa), dev(sb)
+    assert fb.fp8blk_get_device_error() == 0
+    monkeypatch.setenv("FP8BLK_TEST_INJECT_STALL", "1")
+    monkeypatch.setenv("FP8BLK_WAIT_TIMEOUT_MS", "200")
+    fb.fp8blk_gemm(layout, A, SA, B, SB)
+    assert fb.fp8blk_get_device_error() == TIMEOUT_STATUS
+    assert fb.fp8blk_get_device_error() == 0            # the word was cleared
+    monkeypatch.delenv("FP8BLK_TEST_INJECT_STALL")
+    d = fb.fp8blk_gemm(layout, A, SA, B, SB)
+    assert fb.fp8blk_get_device_error() == 0
+    ref = oracle.gemm(layout, qa, sa, qb, sb)
+    assert_gemm_close(d.float().cpu().numpy(), ref, "after timeout")
