@@ -164,6 +164,10 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   g.err = error_word();
   if (!g.err) return FP8BLK_ERR_CUDA;
   g.tmem_db = -1;
+  g.pair = 0;   // pair tiles measured slower (cross-SM hand-offs per K-block); opt in with FP8BLK_GEMM_PAIR=1
+  g.group_m = 0;
+  if (const char* e = std::getenv("FP8BLK_GEMM_PAIR")) g.pair = std::atoi(e);
+  if (const char* e = std::getenv("FP8BLK_GEMM_GROUP_M")) g.group_m = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_TMEM_DB")) g.tmem_db = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) g.inject_stall = std::atoi(e) != 0;

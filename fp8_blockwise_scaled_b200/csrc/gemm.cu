@@ -120,6 +120,7 @@ struct GemmParams {
   uint64_t timeout_ns;
   unsigned int* err;
   int inject_stall;
+  int group_m;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -217,6 +218,18 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&v)[8]) {
 
 }  // namespace
 
+// Tile order: groups of `group_m` M-blocks, N-blocks inside a group, M-blocks
+// fastest inside that.  The CTAs running at the same time then share each A tile
+// among ~#SMs/group_m CTAs and each B tile among group_m CTAs, instead of all
+// M-blocks asking for the same B tile at once.
+__device__ __forceinline__ void tile_coords(int tile, int num_mb, int num_nb, int group_m, int& mb, int& nb) {
+  const int per_group = group_m * num_nb;
+  const int g = tile / per_group, r = tile - g * per_group;
+  const int gm = min(group_m, num_mb - g * group_m);   // the last group may be short
+  mb = g * group_m + r % gm;
+  nb = r / gm;
+}
+
 template <int BN, bool kWgrad, bool kSplit>
 __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     gemm_blockwise_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -277,7 +290,8 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     int64_t issued = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-      const int mb = tile % num_mb, nb = tile / num_mb;
+      int mb, nb;
+      tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
       const int64_t m0 = static_cast<int64_t>(mb) * BM, n0 = static_cast<int64_t>(nb) * BN;
       for (int kb = 0; kb < kblocks; ++kb) {
         // Scales of this K-block into the scale ring.
@@ -379,7 +393,8 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     float2 acc[C::kHalf / 2];
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-      const int mb = tile % num_mb, nb = tile / num_mb;
+      int mb, nb;
+      tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
       const int64_t m = static_cast<int64_t>(mb) * BM + row;
       const int64_t ncol0 = static_cast<int64_t>(nb) * BN + col0;
 #pragma unroll
@@ -484,6 +499,275 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Pair-tile variant: a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256).  Each CTA keeps the same roles as above
+// and owns 128 rows of the tile in its own TMEM; it TMA-loads its own 128 A
+// rows and its half of the tile's 256 B rows, so a K-block moves 32 KB into
+// each SM instead of 48 KB (operand traffic was the limit of the 128 x 256
+// tile).  The loads complete on the leader's "full" barrier; the leader alone
+// issues the MMAs and commits them to the stage and accumulator barriers of
+// both CTAs; both CTAs' promotion warps hand each accumulator buffer back to
+// the leader.  Scale rings stay local.  A timeout raises the abort flag of
+// both CTAs; the TMEM is freed after a cluster barrier, once every MMA of the
+// pair has completed.
+namespace {
+constexpr int kPairStages = 6;
+constexpr int kPairHalfBytes = 128 * BK;              // own A rows, or own half of B
+constexpr int kPairStageBytes = 2 * kPairHalfBytes;
+constexpr int kPairBN = 256;
+constexpr int pair_smem_bytes() { return 1024 + kPairStages * kPairStageBytes + static_cast<int>(sizeof(Ctrl)); }
+static_assert(kPairStages <= 8, "Ctrl holds 8 stage barriers");
+}  // namespace
+
+template <bool kWgrad, bool kSplit>
+__global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                     const GemmParams p) {
+  constexpr int BN = kPairBN;
+  constexpr int kHalf = BN / 2;
+  constexpr int kEpiWarp0 = Layout<kSplit>::kEpiWarp0;
+  constexpr int kAccBufs = 2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + kPairStages * kPairStageBytes);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int num_mp = static_cast<int>(p.M / (2 * BM));
+  const int num_nb = static_cast<int>(p.N / BN);
+  const int kblocks = static_cast<int>(p.K / BK);
+  const int tiles = num_mp * num_nb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&ctrl->full[s], 1);     // the leader's arrive + the bytes of both CTAs
+      mbar_init(&ctrl->empty[s], 1);    // the leader's MMA commit
+    }
+    for (int b = 0; b < kAccBufs; ++b) {
+      mbar_init(&ctrl->tfull[b], 1);
+      mbar_init(&ctrl->tempty[b], 2 * kEpiWarps);   // promotion warps of both CTAs
+    }
+    for (int s = 0; s < kSRing; ++s) {
+      mbar_init(&ctrl->sfull[s], 32);
+      mbar_init(&ctrl->sempty[s], kEpiWarps);
+    }
+    mbar_init(&ctrl->mma_done, 1);
+    mbar_init(&ctrl->never, 1);
+    ctrl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tm_a);
+    tma_prefetch_map(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&ctrl->tmem_base, kAccBufs * BN);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
+  tc_fence_after_sync();
+  const uint32_t tmem_base = ctrl->tmem_base;
+  volatile int* abort = &ctrl->abort;
+  const uint32_t peer_abort = mapa_shared(smem_addr(&ctrl->abort), rank ^ 1u);
+
+  if (warp < kEpiWarp0) {
+  if constexpr (kSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (whole warp)
+    int stage = 0, slot = 0;
+    uint32_t phase = 0, sphase = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    for (int tile = pair; ok && tile < tiles; tile += npairs) {
+      const int mp = tile % num_mp, nb = tile / num_mp;
+      const int64_t m0 = static_cast<int64_t>(mp) * 2 * BM + rank * BM, n0 = static_cast<int64_t>(nb) * BN;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded_pair(&ctrl->sempty[slot], sphase ^ 1u, abort, peer_abort,
+                                                            p.timeout_ns, p.err, false))) {
+          ok = false;
+          break;
+        }
+        ScaleSlot& ss = ctrl->slots[slot];
+        cp_async_16(&ss.sa[lane * 4], p.sa + static_cast<int64_t>(kb) * p.M + m0 + lane * 4);
+        if constexpr (kWgrad) {
+          for (int c = lane * 4; c < BN; c += 128)
+            cp_async_16(&ss.sb[c], p.sb + static_cast<int64_t>(kb) * p.N + n0 + c);
+        } else {
+          if (lane < BN / 128) cp_async_4(&ss.sb[lane], p.sb + (n0 / 128 + lane) * kblocks + kb);
+        }
+        cp_async_arrive(&ctrl->sfull[slot]);
+        if (++slot == kSRing) {
+          slot = 0;
+          sphase ^= 1u;
+        }
+        if (lane == 0) {
+          ok = mbar_wait_bounded_pair(&ctrl->empty[stage], phase ^ 1u, abort, peer_abort, p.timeout_ns, p.err, true);
+          if (ok) {
+            uint8_t* st = smem + stage * kPairStageBytes;
+            const uint32_t full_leader = mapa_shared(smem_addr(&ctrl->full[stage]), 0);
+            if (leader) mbar_arrive_expect_tx(&ctrl->full[stage], 2 * kPairStageBytes);
+            tma_load_2d_pair(st, &tm_a, full_leader, kb * BK, static_cast<int>(m0));
+            tma_load_2d_pair(st + kPairHalfBytes, &tm_b, full_leader, kb * BK, static_cast<int>(n0 + rank * BM));
+          }
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) break;
+        ++issued;
+        if (++stage == kPairStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (leader && lane == 0) {
+      // The leader's full barriers count the bytes of both CTAs: once the last
+      // stages it armed are complete, no load of the pair is in flight.
+      const int64_t first = issued > kPairStages ? issued - kPairStages : 0;
+      for (int64_t j = first; j < issued; ++j)
+        mbar_wait_bounded(&ctrl->full[j % kPairStages], static_cast<uint32_t>((j / kPairStages) & 1), nullptr,
+                          p.timeout_ns, p.err);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader CTA only)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(2 * BM, BN);
+      int stage = 0;
+      uint32_t phase = 0, abuf = 0, aphase = 0;
+      bool ok = true;
+      if (p.inject_stall)
+        ok = mbar_wait_bounded_pair(&ctrl->never, 0, abort, peer_abort, p.timeout_ns, p.err, false);
+      for (int tile = pair; ok && tile < tiles; tile += npairs) {
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded_pair(&ctrl->full[stage], phase, abort, peer_abort, p.timeout_ns, p.err, true) ||
+              !mbar_wait_bounded_pair(&ctrl->tempty[abuf], aphase ^ 1u, abort, peer_abort, p.timeout_ns, p.err,
+                                      true)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_addr = smem_addr(smem + stage * kPairStageBytes);
+          const uint64_t adesc = smem_desc_kmajor_sw128(a_addr);
+          const uint64_t bdesc = smem_desc_kmajor_sw128(a_addr + kPairHalfBytes);
+          const uint32_t d_tmem = tmem_base + abuf * BN;
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)
+            umma_e4m3_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+          umma_commit_pair(&ctrl->empty[stage], 0x3);
+          umma_commit_pair(&ctrl->tfull[abuf], 0x3);
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          if (++abuf == kAccBufs) {
+            abuf = 0;
+            aphase ^= 1u;
+          }
+        }
+      }
+      umma_commit_pair(&ctrl->mma_done, 0x1);
+      mbar_wait_bounded(&ctrl->mma_done, 0, nullptr, p.timeout_ns, p.err);
+    }
+  }
+  } else {
+    if constexpr (kSplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
+    // ------------------------------------------------------------ promotion + epilogue
+    const int ew = warp - kEpiWarp0;  // 0..7
+    const int wg = ew >> 2;           // which half of the tile's columns
+    const int quarter = warp & 3;     // TMEM lanes this warp may read
+    const int row = quarter * 32 + lane;
+    const int col0 = wg * kHalf;
+    uint32_t abuf = 0, aphase = 0, sphase = 0;
+    int slot = 0;
+    float2 acc[kHalf / 2];
+    bool ok = true;
+    for (int tile = pair; ok && tile < tiles; tile += npairs) {
+      const int mp = tile % num_mp, nb = tile / num_mp;
+      const int64_t m = static_cast<int64_t>(mp) * 2 * BM + rank * BM + row;
+      const int64_t ncol0 = static_cast<int64_t>(nb) * BN + col0;
+#pragma unroll
+      for (int j = 0; j < kHalf / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
+
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const bool got =
+            mbar_wait_bounded_pair(&ctrl->sfull[slot], sphase, abort, peer_abort, p.timeout_ns, p.err, false) &&
+            mbar_wait_bounded_pair(&ctrl->tfull[abuf], aphase, abort, peer_abort, p.timeout_ns, p.err, true);
+        if (!__all_sync(0xFFFFFFFFu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const ScaleSlot& ss = ctrl->slots[slot];
+        const float sa = ss.sa[row];
+        const float f = kWgrad ? 0.0f : sa * ss.sb[wg];
+        const float* sbc = ss.sb + col0;
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * BN + col0;
+        if constexpr (kSplit) {
+#pragma unroll
+          for (int c = 0; c < kHalf; c += 64) {
+            uint32_t r[64];
+            tmem_ld_32x32b_x64(taddr + c, r);
+            tmem_wait_ld64(r);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              promote16<kWgrad>(acc + c / 2 + 8 * q, *reinterpret_cast<const uint32_t(*)[16]>(r + 16 * q), f,
+                                sbc + c + 16 * q, sa);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kHalf; c += 16) {
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(taddr + c, r);
+            tmem_wait_ld16(r);
+            promote16<kWgrad>(acc + c / 2, r, f, sbc + c, sa);
+          }
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader)
+            mbar_arrive(&ctrl->tempty[abuf]);
+          else
+            mbar_arrive_remote(mapa_shared(smem_addr(&ctrl->tempty[abuf]), 0));
+          mbar_arrive(&ctrl->sempty[slot]);
+        }
+        if (++abuf == kAccBufs) {
+          abuf = 0;
+          aphase ^= 1u;
+        }
+        if (++slot == kSRing) {
+          slot = 0;
+          sphase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      uint16_t* drow = p.d + m * p.ldd + ncol0;
+#pragma unroll
+      for (int j = 0; j < kHalf; j += 16) {
+        uint32_t v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = pack_bf16x2(acc[j / 2 + q].x, acc[j / 2 + q].y);
+        st_global_v8(drow + j, v);
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync();  // every MMA of the pair is done and no signal is left in flight
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc_pair(tmem_base, kAccBufs * BN);
+  }
+}
+
 namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -534,10 +818,46 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   }
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BN)) return cudaErrorInvalidValue;
-  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall};
+  const int num_mb = static_cast<int>(g.M / BM);
+  int group_m = g.group_m > 0 ? g.group_m : 8;
+  if (group_m > num_mb) group_m = num_mb;
+  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, group_m};
   const int64_t tiles = (g.M / BM) * (g.N / BN);
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
   gemm_blockwise_kernel<BN, kWgrad, kSplit><<<grid, Layout<kSplit>::kThreads, kSmem, stream>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+template <bool kWgrad, bool kSplit>
+cudaError_t launch_pair(const GemmArgs& g, cudaStream_t stream) {
+  static bool attr_set = false;
+  constexpr int kSmem = pair_smem_bytes();
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<kWgrad, kSplit>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BM)) return cudaErrorInvalidValue;
+  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, 0};
+  const int64_t tiles = (g.M / (2 * BM)) * (g.N / kPairBN);
+  const int64_t max_pairs = num_sms() / 2;
+  const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(Layout<kSplit>::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kWgrad, kSplit>, ta, tb, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -551,6 +871,13 @@ double wave_eff(int64_t tiles) {
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream) {
+  const bool wgrad = g.layout == 2;
+  // Pair tiles (256 x 256 over two SMs) whenever the shape allows them.
+  if (g.pair > 0 && g.block_n == 0 && g.M % 256 == 0 && g.N % 256 == 0) {
+    const bool split = g.tmem_db < 0 ? wgrad : g.tmem_db != 0;
+    if (wgrad) return split ? launch_pair<true, true>(g, stream) : launch_pair<true, false>(g, stream);
+    return split ? launch_pair<false, true>(g, stream) : launch_pair<false, false>(g, stream);
+  }
   int bn = g.block_n;
   if (bn == 0) {
     bn = 128;
@@ -561,7 +888,6 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream) {
     }
   }
   if (bn == 256 && g.N % 256 != 0) return cudaErrorInvalidValue;
-  const bool wgrad = g.layout == 2;
   // The register split with double-buffered TMEM reads pays off where the
   // promotion does more work per column (WGRAD); measured on B200, the plain
   // layout is faster for the forward/data-gradient promotion.
