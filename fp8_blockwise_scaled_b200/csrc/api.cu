@@ -69,6 +69,16 @@ fp8blk_status launch_status(cudaError_t e) {
   return FP8BLK_ERR_LAUNCH;
 }
 
+// Bounded device waits of a quantiser launch (and the stall test hook).
+fp8blk_status set_quant_waits(QuantArgs& a) {
+  a.timeout_ns = wait_timeout_ns();
+  a.err = error_word();
+  if (!a.err) return FP8BLK_ERR_CUDA;
+  a.inject_stall = 0;
+  if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) a.inject_stall = std::atoi(e) != 0;
+  return FP8BLK_OK;
+}
+
 fp8blk_status check_quant_common(const void* x, int64_t rows, int64_t cols, int64_t ld) {
   if (!x) return FP8BLK_ERR_INVALID_ARG;
   if (!dim_ok(rows) || !dim_ok(cols)) return FP8BLK_ERR_SHAPE;
@@ -101,6 +111,7 @@ fp8blk_status fp8blk_quantize_act_1x128(const void* x, int64_t rows, int64_t col
   if ((st = check_device()) != FP8BLK_OK) return st;
   QuantArgs a{static_cast<const uint16_t*>(x), rows, cols, ldx, q_row, s_row, q_colT, s_colT, rows / 128,
               cols / 128};
+  if ((st = set_quant_waits(a)) != FP8BLK_OK) return st;
   return launch_status(fp8blk::launch_quant(kmode, a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -112,6 +123,7 @@ static fp8blk_status quantize_weight(const void* w, int64_t n, int64_t k, int64_
   if (!aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u)) return FP8BLK_ERR_ALIGN;
   if ((st = check_device()) != FP8BLK_OK) return st;
   QuantArgs a{static_cast<const uint16_t*>(w), n, k, ldw, nullptr, nullptr, nullptr, nullptr, n / 128, k / 128};
+  if ((st = set_quant_waits(a)) != FP8BLK_OK) return st;
   int kmode;
   if (transposed) {
     a.q_t = q;

@@ -768,9 +768,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
   }
 }
 
-namespace {
-
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     void* ptr = nullptr;
@@ -782,9 +780,11 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
+namespace {
+
 // 2-D map over a row-major [rows][cols] E4M3 matrix, box = box_rows x 128 bytes, 128-byte swizzle.
 bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
-  auto encode = get_encode_fn();
+  auto encode = tensor_map_encoder();
   if (!encode) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
@@ -872,7 +872,7 @@ double wave_eff(int64_t tiles) {
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   const bool wgrad = g.layout == 2;
-  // Pair tiles (256 x 256 over two SMs) whenever the shape allows them.
+  // Pair tiles (256 x 256 over two SMs) only on request, when the shape allows them.
   if (g.pair > 0 && g.block_n == 0 && g.M % 256 == 0 && g.N % 256 == 0) {
     const bool split = g.tmem_db < 0 ? wgrad : g.tmem_db != 0;
     if (wgrad) return split ? launch_pair<true, true>(g, stream) : launch_pair<true, false>(g, stream);

@@ -1,6 +1,7 @@
 // Internal launch interface between the C-ABI layer (api.cu) and the kernels.
 #pragma once
 
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -17,6 +18,9 @@ struct QuantArgs {
   uint8_t* q_t;       // Q_COLT / Q_BLKT: [cols][rows]
   float* s_t;         // Q_COLT: [rows/128][cols];  Q_BLKT: [cols/128][rows/128]
   int64_t tiles_r, tiles_c;
+  uint64_t timeout_ns;   // bound on every device-side wait
+  int inject_stall;      // test hook: the consumers wait on a barrier nothing completes
+  unsigned int* err;     // device error word
 };
 
 cudaError_t launch_quant(int mode, const QuantArgs& a, cudaStream_t stream);
@@ -40,5 +44,8 @@ struct GemmArgs {
 };
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream);
+
+// The driver's cuTensorMapEncodeTiled (looked up once), or null if unavailable.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 }  // namespace fp8blk

@@ -7,15 +7,19 @@
 // with amax over a 1x128 group (activations) or a 128x128 block (weights).
 //
 // One kernel, templated on which outputs it writes, walks the input in
-// 128x128 tiles (one tile per CTA iteration, 256 threads):
+// 128x128 tiles:
 //   Q_ROW   1x128 groups along each row, codes in place      (activations, FWD/DGRAD A)
 //   Q_COLT  1x128 groups along each column, codes transposed  (activations, WGRAD A and B)
 //   Q_BLK   one 128x128 block, codes in place                 (weights, FWD B)
 //   Q_BLKT  one 128x128 block, codes transposed               (weights, DGRAD B)
-// Every input byte is read from HBM once, with 16-byte coalesced loads; the
-// row and block paths quantise straight from registers, the transposed paths
-// go through one shared-memory copy of the tile.  HBM bound: per element
-// 2 B read + 1 B code + 4/128 B scale per output layout.
+// Persistent CTAs, two per SM: one producer warp streams the CTA's tiles from
+// HBM into a ring of shared-memory stages with TMA; eight consumer warps each
+// load an 8x8 sub-block per thread from the stage (and hand the stage back at
+// once), reduce the row, column or block maxima with shuffles and one small
+// shared-memory exchange, and write both the in-place codes (8-byte stores,
+// whole 128-byte row segments per half-warp) and the transposed codes (through
+// a swizzled 16 KB code tile, 16-byte stores) from registers.  HBM bound: per
+// element 2 B read + 1 B code + 4/128 B scale per output layout.
 //
 // Exactness of the scale.  s = fl32(amax / 448) is computed as y = amax*2^-6
 // (exact) followed by a correctly rounded division by 7 with one FMA
@@ -45,14 +49,34 @@ namespace fp8blk {
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kThreads = 256;
-// Shared memory of the transposed paths (no padding needed: see the access patterns below).
-constexpr int kXsBytes = kTile * kTile * 2;       // bf16 tile, 256-byte rows
+constexpr int kConsumers = 256;                   // 8 warps
+constexpr int kThreads = kConsumers;              // thread 0 also issues the TMA loads
+constexpr uint32_t kTileBytes = kTile * kTile * 2;  // one bf16 tile as TMA writes it: 128 rows of 256 bytes
+
+// Stages of the input ring: the transposed paths also keep a code tile, so
+// they take two stages to stay at two CTAs per SM.
+template <int MODE>
+__host__ __device__ constexpr int stages_for() { return (MODE & (Q_COLT | Q_BLKT)) ? 2 : 3; }
+
+// Shared memory: input stages, then (transposed paths) the transposed code
+// tile, then the small per-tile arrays and the barriers.
+struct QCtrl {
+  uint64_t full[3], empty[3];
+  uint64_t never;            // completed by nothing: the stall test waits on it
+  int abort;
+  float warpmax[2][8];                   // per-warp block maxima, double-buffered by tile parity
+  alignas(16) float2 qs[kTile];          // per-column {s, -1/s}
+  alignas(16) float2 rq[8][2][8];        // per half-warp: {s, -1/s} of its 8 rows
+  alignas(16) uint32_t cpart[8 * 64];    // per-warp packed column maxima (16-byte stores)
+};
+static_assert(sizeof(QCtrl) % 16 == 0, "QCtrl keeps 16-byte alignment");
 constexpr int kCsBytes = kTile * kTile;           // transposed codes, 128-byte rows, 16-B chunks swizzled
-constexpr int kCpartBytes = 8 * 64 * 4;           // per-warp packed column maxima
-constexpr int kQsBytes = kTile * 8;               // per-column {s, -1/s}
-constexpr int kSmallBytes = 64;                   // per-warp block maxima
-constexpr int kSmemBytes = kSmallBytes + kQsBytes + kCpartBytes + kXsBytes + kCsBytes;
+
+template <int MODE>
+__host__ __device__ constexpr int smem_bytes_for() {
+  return stages_for<MODE>() * static_cast<int>(kTileBytes) + ((MODE & (Q_COLT | Q_BLKT)) ? kCsBytes : 0) +
+         static_cast<int>(sizeof(QCtrl)) + 1024;  // + alignment slack for the 1024-byte aligned base
+}
 
 struct QScale {
   float s;    // the group's scale
@@ -78,6 +102,13 @@ __device__ __forceinline__ uint32_t cvt4(float x0, float x1, float x2, float x3)
       "mov.b32 %0, {l, h};\n\t}"
       : "=r"(r)
       : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
+  return r;
+}
+
+// Two values -> two E4M3 codes in the low 16 bits (x0 in the low byte).
+__device__ __forceinline__ uint32_t cvt2(float x0, float x1) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(x0), "f"(x1));
   return r;
 }
 
@@ -110,63 +141,172 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
 // |bf16| maxima on raw bits: clearing the sign keeps the order of finite magnitudes.
 constexpr uint32_t kAbs2 = 0x7FFF7FFFu;
 
-__device__ __forceinline__ float absmax8(const uint4& v) {
-  uint32_t a = __vmaxu2(__vmaxu2(v.x & kAbs2, v.y & kAbs2), __vmaxu2(v.z & kAbs2, v.w & kAbs2));
-  a = max(a & 0xFFFFu, a >> 16);
-  return __uint_as_float(a << 16);
+
+// Consumer-only barrier (named barrier 1, the 256 consumer threads).
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Consumer-only barrier that also returns the AND of `v` over the consumers.
+__device__ __forceinline__ bool consumers_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, 256, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
 }
 
 }  // namespace
 
+// Persistent, two CTAs per SM.  The CTA's 128x128 bf16 tiles stream from HBM
+// into a ring of S shared-memory stages with TMA; each warp copies its rows of
+// a stage into registers and hands the stage back at once, and thread 0 then
+// refills that stage with the tile S steps ahead, so the next tiles are in
+// flight while the current one is quantised.  Every wait is bounded: on a
+// timeout the threads agree (one barrier reduction) to leave together, thread
+// 0 first waits for its copies in flight, and the error word records the
+// timeout.
 template <int MODE>
-__global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_constant__ CUtensorMap tm_x, QuantArgs a) {
   constexpr bool kRow = MODE & Q_ROW;
   constexpr bool kColT = MODE & Q_COLT;
   constexpr bool kBlk = MODE & Q_BLK;
   constexpr bool kBlkT = MODE & Q_BLKT;
   constexpr bool kTileSmem = kColT || kBlkT;
   constexpr bool kBlockScale = kBlk || kBlkT;
+  constexpr int S = stages_for<MODE>();
 
-  extern __shared__ __align__(16) uint8_t smem[];
-  float* warpmax = reinterpret_cast<float*>(smem);                                      // [8]
-  float2* qs = reinterpret_cast<float2*>(smem + kSmallBytes);                           // [128] column scales
-  uint32_t* cpart = reinterpret_cast<uint32_t*>(smem + kSmallBytes + kQsBytes);         // [8][64]
-  uint8_t* xs = smem + kSmallBytes + kQsBytes + kCpartBytes;                            // [128][256 B]
-  uint8_t* cs = xs + kXsBytes;                                                          // [128][128 B]
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* cs = smem + S * kTileBytes;                                      // [128][128 B] (transposed paths)
+  QCtrl* ctrl = reinterpret_cast<QCtrl*>(cs + (kTileSmem ? kCsBytes : 0));
 
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
-  const int chunk = t & 15;      // this thread's 16-byte column chunk of the tile
-  const int rbase = t >> 4;      // rows rbase + 16 i, i = 0..7
   const int64_t tiles = a.tiles_r * a.tiles_c;
-  const uint32_t ldx = static_cast<uint32_t>(a.ldx);
+  auto load_tile = [&](int stage, int64_t tile) {
+    const int64_t tr = tile % a.tiles_r, tc = tile / a.tiles_r;
+    mbar_arrive_expect_tx(&ctrl->full[stage], kTileBytes);
+    tma_load_2d(smem + stage * kTileBytes, &tm_x, &ctrl->full[stage], static_cast<int>(tc * kTile),
+                static_cast<int>(tr * kTile));
+  };
+
+  int64_t issued = 0;   // loads issued (thread 0 only)
+  if (t == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&ctrl->full[s], 1);
+      mbar_init(&ctrl->empty[s], kConsumers / 32);
+    }
+    mbar_init(&ctrl->never, 1);
+    ctrl->abort = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&tm_x);
+    for (int64_t tile = blockIdx.x; issued < S && tile < tiles; tile += gridDim.x) load_tile(issued++, tile);
+  }
+  __syncthreads();
+  volatile int* abort = &ctrl->abort;
+
+  // -------------------------------------------------------------- consumers
+  // Thread layout: each consumer owns an 8 x 8 sub-block of the tile, rows
+  // 8 bi .. 8 bi + 7 and the 16-byte column chunk bj (columns 8 bj .. 8 bj + 7),
+  // and makes both the in-place and the transposed codes of it from registers.
+  // A 1x128 row group spans the 16 lanes of a half-warp; a 128-token column
+  // group spans all 16 row blocks (two per warp).
+  const int bj = lane & 15;
+  const int bi = 2 * warp + (lane >> 4);
   const uint32_t cols = static_cast<uint32_t>(a.cols);
   const uint32_t rows = static_cast<uint32_t>(a.rows);
+  float2* rq = ctrl->rq[warp][lane >> 4];
 
-  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+  int64_t it = 0;
+  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+    const int s = static_cast<int>(it % S);
+    const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+    bool ok = a.inject_stall ? mbar_wait_bounded(&ctrl->never, 0, abort, a.timeout_ns, a.err)
+                             : mbar_wait_bounded(&ctrl->full[s], ph, abort, a.timeout_ns, a.err);
+    if (!consumers_all(ok)) break;
+
     const int64_t tr = tile % a.tiles_r, tc = tile / a.tiles_r;
     const int64_t row0 = tr * kTile, col0 = tc * kTile;
-
     uint4 v[8];
     {
-      const uint16_t* src = a.x + row0 * a.ldx + col0 + rbase * ldx + chunk * 8;
+      const uint8_t* xs = smem + s * kTileBytes + (8 * bi) * 256 + bj * 16;   // conflict-free: 2 rows per warp
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = ld_nc_v4(src + 16u * i * ldx);
+      for (int r = 0; r < 8; ++r) v[r] = *reinterpret_cast<const uint4*>(xs + r * 256);
+    }
+    __syncwarp();                                // everything else comes from registers: hand the stage back
+    if (lane == 0) mbar_arrive(&ctrl->empty[s]);
+    if (t == 0) {                                // and refill it with the tile S steps ahead
+      const int64_t next = tile + static_cast<int64_t>(S) * gridDim.x;
+      if (next < tiles && mbar_wait_bounded(&ctrl->empty[s], ph, abort, a.timeout_ns, a.err)) {
+        load_tile(s, next);
+        ++issued;
+      }
     }
 
-    // ---------------------------------------------------------------- from registers
+    // Maxima of |x| on raw bf16 bits (clearing the sign keeps the order of
+    // finite magnitudes), two columns per word.
+    [[maybe_unused]] uint32_t cm[4] = {0, 0, 0, 0};   // column maxima over this thread's 8 rows
+    [[maybe_unused]] uint32_t rm[4];                  // row maxima, rows 2p (low half) and 2p+1 (high half)
+    [[maybe_unused]] uint32_t bm = 0;                 // block maximum
+    {
+      [[maybe_unused]] uint32_t even = 0;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const uint32_t a0 = v[r].x & kAbs2, a1 = v[r].y & kAbs2, a2 = v[r].z & kAbs2, a3 = v[r].w & kAbs2;
+        if constexpr (kColT) {
+          cm[0] = __vmaxu2(cm[0], a0);
+          cm[1] = __vmaxu2(cm[1], a1);
+          cm[2] = __vmaxu2(cm[2], a2);
+          cm[3] = __vmaxu2(cm[3], a3);
+        }
+        if constexpr (kRow || kBlockScale) {
+          const uint32_t m = __vmaxu2(__vmaxu2(a0, a1), __vmaxu2(a2, a3));
+          if constexpr (kBlockScale) bm = __vmaxu2(bm, m);
+          if constexpr (kRow) {
+            if (r & 1) rm[r >> 1] = __vmaxu2(__byte_perm(even, m, 0x5410), __byte_perm(even, m, 0x7632));
+            else even = m;
+          }
+        }
+      }
+    }
+
+    if constexpr (kRow) {
+      // Reduce-scatter of the 8 row maxima over the half-warp's 16 lanes: after
+      // the exchanges at distance 8 and 4 each lane holds one row pair, the
+      // exchanges at 2 and 1 finish its maximum; lane bits 3..1 name the row.
+      const bool b = lane & 8, c = lane & 4, d = lane & 2;
+      uint32_t k0 = b ? rm[2] : rm[0], k1 = b ? rm[3] : rm[1];
+      const uint32_t s0 = b ? rm[0] : rm[2], s1 = b ? rm[1] : rm[3];
+      k0 = __vmaxu2(k0, __shfl_xor_sync(0xFFFFFFFFu, s0, 8));
+      k1 = __vmaxu2(k1, __shfl_xor_sync(0xFFFFFFFFu, s1, 8));
+      uint32_t k = c ? k1 : k0;
+      k = __vmaxu2(k, __shfl_xor_sync(0xFFFFFFFFu, c ? k0 : k1, 4));
+      k = __vmaxu2(k, __shfl_xor_sync(0xFFFFFFFFu, k, 2));
+      k = __vmaxu2(k, __shfl_xor_sync(0xFFFFFFFFu, k, 1));
+      const int rho = (lane >> 1) & 7;             // = 4 b + 2 c + d
+      const QScale q = make_qscale(__uint_as_float(d ? (k & 0xFFFF0000u) : (k << 16)));
+      if ((lane & 1) == 0) {
+        rq[rho] = make_float2(q.s, q.nr);
+        a.s_row[tc * a.rows + row0 + 8 * bi + rho] = q.s;
+      }
+      __syncwarp();
+    }
+
     QScale qblk{};
     if constexpr (kBlockScale) {
-      float amax = 0.0f;
+      uint32_t m = max(bm & 0xFFFFu, bm >> 16);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, absmax8(v[i]));
+      for (int o = 16; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      float* wm = ctrl->warpmax[it & 1];
+      if (lane == 0) wm[warp] = __uint_as_float(m << 16);
+      consumers_sync();
+      float amax = wm[0];
 #pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-      if (lane == 0) warpmax[warp] = amax;
-      __syncthreads();
-      amax = warpmax[0];
-#pragma unroll
-      for (int w = 1; w < kThreads / 32; ++w) amax = fmaxf(amax, warpmax[w]);
+      for (int w = 1; w < kConsumers / 32; ++w) amax = fmaxf(amax, wm[w]);
       qblk = make_qscale(amax);
       if (t == 0) {
         if constexpr (kBlk) a.s_row[tr * a.tiles_c + tc] = qblk.s;
@@ -174,141 +314,128 @@ __global__ void __launch_bounds__(kThreads) quant_tile_kernel(QuantArgs a) {
       }
     }
 
-    // Row groups (or the whole block) in place: chunk i of this thread is rows
-    // rbase + 16 i, columns chunk*8 .. +7 of the tile.
-    auto quant_in_place = [&](auto chunk_of) {
-      uint8_t* qdst = a.q_row + row0 * a.cols + col0 + rbase * cols + chunk * 8;
-      [[maybe_unused]] float* sdst = kRow ? a.s_row + tc * a.rows + row0 + rbase : nullptr;
-      auto scale_of = [&](const uint4& vi) {
-        if constexpr (kRow) {
-          float amax = absmax8(vi);
+    [[maybe_unused]] QScale cq[8];                   // scales of this thread's 8 columns
+    if constexpr (kColT) {
 #pragma unroll
-          for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-          return make_qscale(amax);
-        } else {
-          return qblk;
+      for (int j = 0; j < 4; ++j) cm[j] = __vmaxu2(cm[j], __shfl_xor_sync(0xFFFFFFFFu, cm[j], 16));
+      if (lane < 16) *reinterpret_cast<uint4*>(ctrl->cpart + warp * 64 + bj * 4) = make_uint4(cm[0], cm[1], cm[2], cm[3]);
+      consumers_sync();                          // every warp's column maxima are in
+      if (t < kTile) {                           // one column per thread
+        uint32_t mx = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) mx = __vmaxu2(mx, ctrl->cpart[w * 64 + (t >> 1)]);
+        const QScale q = make_qscale(__uint_as_float((t & 1) ? (mx & 0xFFFF0000u) : (mx << 16)));
+        ctrl->qs[t] = make_float2(q.s, q.nr);
+        a.s_t[tr * a.cols + col0 + t] = q.s;
+      }
+      consumers_sync();                          // the column scales are in
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 f = *reinterpret_cast<const float4*>(&ctrl->qs[8 * bj + 2 * j]);
+        cq[2 * j] = QScale{f.x, f.y};
+        cq[2 * j + 1] = QScale{f.z, f.w};
+      }
+    }
+
+    // Codes, two rows at a time.  In place: one 8-byte store per row (a warp
+    // writes two 128-byte row segments).  Transposed: column c of the tile
+    // collects the codes of rows 8 bi .. 8 bi + 7 in the 8-byte unit bi ^ bj of
+    // its 128-byte line in cs (the XOR spreads a half-warp over all 32 banks).
+    [[maybe_unused]] uint8_t* qdst = kRow || kBlk ? a.q_row + (row0 + 8 * bi) * a.cols + col0 + 8 * bj : nullptr;
+    [[maybe_unused]] uint32_t pend[8];             // transposed: codes of the previous row pair, per column
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      float f0[8], f1[8];
+      unpack8(v[2 * p], f0);
+      unpack8(v[2 * p + 1], f1);
+      if constexpr (kRow || kBlk) {
+        QScale q0 = qblk, q1 = qblk;
+        if constexpr (kRow) {
+          const float4 f = *reinterpret_cast<const float4*>(&rq[2 * p]);
+          q0 = QScale{f.x, f.y};
+          q1 = QScale{f.z, f.w};
         }
-      };
+        *reinterpret_cast<uint2*>(qdst + (2 * p) * cols) = quant8(f0, q0);
+        *reinterpret_cast<uint2*>(qdst + (2 * p + 1) * cols) = quant8(f1, q1);
+      }
+      if constexpr (kTileSmem) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint4 vi = chunk_of(i);
-        const QScale q = scale_of(vi);
-        float f[8];
-        unpack8(vi, f);
-        *reinterpret_cast<uint2*>(qdst + 16u * i * cols) = quant8(f, q);
-        if constexpr (kRow) {
-          if (chunk == 0) sdst[16 * i] = q.s;
+        for (int c = 0; c < 8; ++c) {
+          const QScale q = kColT ? cq[c] : qblk;
+          float w0, w1;
+          neg_quotient2(w0, w1, f0[c], f1[c], q.s, q.nr);
+          const uint32_t h = cvt2(w0, w1);
+          if (p & 1) {
+            const uint32_t word = __byte_perm(pend[c], h, 0x5410) ^ 0x80808080u;
+            *reinterpret_cast<uint32_t*>(cs + (8 * bj + c) * 128 + ((bi ^ bj) * 8) + (p >> 1) * 4) = word;
+          } else {
+            pend[c] = h;
+          }
         }
       }
-    };
-    if constexpr ((kRow || kBlk) && !kTileSmem) {
-      quant_in_place([&](int i) { return v[i]; });
     }
 
     if constexpr (kTileSmem) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4*>(xs + (rbase + 16 * i) * 256 + chunk * 16) = v[i];
-      if constexpr (kColT) {
-        // Column maxima of this thread's 8 rows, packed two columns per word,
-        // then across the two row sets of the warp.
-        uint32_t m[4] = {0, 0, 0, 0};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          m[0] = __vmaxu2(m[0], v[i].x & kAbs2);
-          m[1] = __vmaxu2(m[1], v[i].y & kAbs2);
-          m[2] = __vmaxu2(m[2], v[i].z & kAbs2);
-          m[3] = __vmaxu2(m[3], v[i].w & kAbs2);
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) m[j] = __vmaxu2(m[j], __shfl_xor_sync(0xFFFFFFFFu, m[j], 16));
-        if (lane < 16) *reinterpret_cast<uint4*>(cpart + warp * 64 + chunk * 4) = make_uint4(m[0], m[1], m[2], m[3]);
-      }
-      __syncthreads();
-      // With the tile in shared memory the in-place codes are made from there,
-      // so the input registers are free for the transposed pass.
-      if constexpr (kRow || kBlk) {
-        auto from_smem = [&](int i) { return *reinterpret_cast<const uint4*>(xs + (rbase + 16 * i) * 256 + chunk * 16); };
-        quant_in_place(from_smem);
-      }
-      if constexpr (kColT) {
-        if (t < kTile) {  // one column per thread
-          uint32_t mx = 0;
-#pragma unroll
-          for (int w = 0; w < 8; ++w) mx = __vmaxu2(mx, cpart[w * 64 + (t >> 1)]);
-          const float am = __uint_as_float((t & 1) ? (mx & 0xFFFF0000u) : (mx << 16));
-          const QScale q = make_qscale(am);
-          qs[t] = make_float2(q.s, q.nr);
-          a.s_t[tr * a.cols + col0 + t] = q.s;
-        }
-        __syncthreads();
-      }
-      // Transposed codes.  Item = (column pair cp, 16-row chunk rc); the 32 lanes
-      // of a warp read consecutive words of the same smem rows (conflict-free) and
-      // write 16-byte chunks whose position is XOR-swizzled by cp (conflict-free).
-      const uint32_t* xs32 = reinterpret_cast<const uint32_t*>(xs);
-      auto col_scale = [&](int c) {
-        if constexpr (kColT) {
-          const float2 fq = qs[c];
-          return QScale{fq.x, fq.y};
-        } else {
-          return qblk;
-        }
-      };
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int item = t + kThreads * j;
-        const int cp = item & 63, rc = item >> 6;
-        const QScale qa = col_scale(2 * cp), qb = col_scale(2 * cp + 1);
-        float lo[16], hi[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint32_t w = xs32[(rc * 16 + i) * 64 + cp];
-          lo[i] = bf16lo(w);
-          hi[i] = bf16hi(w);
-        }
-        const uint2 a0 = quant8(*reinterpret_cast<const float(*)[8]>(lo), qa);
-        const uint2 a1 = quant8(*reinterpret_cast<const float(*)[8]>(lo + 8), qa);
-        const uint2 b0 = quant8(*reinterpret_cast<const float(*)[8]>(hi), qb);
-        const uint2 b1 = quant8(*reinterpret_cast<const float(*)[8]>(hi + 8), qb);
-        const int phys = (rc ^ (cp & 7)) * 16;
-        *reinterpret_cast<uint4*>(cs + (2 * cp) * 128 + phys) = make_uint4(a0.x, a0.y, a1.x, a1.y);
-        *reinterpret_cast<uint4*>(cs + (2 * cp + 1) * 128 + phys) = make_uint4(b0.x, b0.y, b1.x, b1.y);
-      }
-      __syncthreads();
+      consumers_sync();                          // the transposed code tile is complete
+      // Column cc's logical 16-byte part m (tokens 16 m .. 16 m + 15) holds units
+      // 2m and 2m + 1, stored at units (2m) ^ x and (2m + 1) ^ x, x = cc / 8: the
+      // same 16-byte chunk m ^ (x / 2), halves swapped when x is odd.
       uint8_t* tdst = a.q_t + col0 * a.rows + row0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int k = t + kThreads * j;
-        const int c = k >> 3, part = k & 7;
-        const uint4 codes = *reinterpret_cast<const uint4*>(cs + c * 128 + ((part ^ ((c >> 1) & 7)) * 16));
-        *reinterpret_cast<uint4*>(tdst + c * rows + part * 16) = codes;
+        const int k = t + kConsumers * j;
+        const int cc = k >> 3, m = k & 7, x = cc >> 3;
+        uint4 w = *reinterpret_cast<const uint4*>(cs + cc * 128 + ((m ^ (x >> 1)) * 16));
+        if (x & 1) w = make_uint4(w.z, w.w, w.x, w.y);
+        *reinterpret_cast<uint4*>(tdst + cc * rows + m * 16) = w;
       }
+      // The next tile rewrites cs, qs, cpart and rq only after its first
+      // consumer barrier, which every thread reaches after these reads.
     }
-    if constexpr (kTileSmem || kBlockScale) __syncthreads();  // shared memory is reused by the next tile
+  }
+  // Thread 0 lets its copies still in flight land before the CTA's shared
+  // memory goes away (on the normal path every load has been consumed).
+  if (t == 0) {
+    for (int64_t j = it; j < issued; ++j)
+      mbar_wait_bounded(&ctrl->full[j % S], static_cast<uint32_t>((j / S) & 1), nullptr, a.timeout_ns, a.err);
   }
 }
 
 namespace {
 
+// 2-D map over the bf16 input [rows][ldx], box = one 128 x 128 tile, no swizzle
+// (the kernel's shared-memory access patterns are conflict-free on plain rows).
+bool make_input_map(CUtensorMap* map, const QuantArgs& a) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.cols), static_cast<cuuint64_t>(a.rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.ldx) * 2};
+  const cuuint32_t box[2] = {kTile, kTile};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int MODE>
 cudaError_t launch_mode(const QuantArgs& a, cudaStream_t stream) {
   static int grid_cap = 0;  // resident CTAs on this device (set on first use)
-  constexpr bool kSmem = (MODE & (Q_COLT | Q_BLKT)) != 0;
-  const int smem = kSmem ? kSmemBytes : kSmallBytes;
+  constexpr int kSmem = smem_bytes_for<MODE>();
   if (grid_cap == 0) {
-    cudaError_t e = cudaFuncSetAttribute(quant_tile_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(quant_tile_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_tile_kernel<MODE>, kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_tile_kernel<MODE>, kThreads, kSmem);
     if (e != cudaSuccess) return e;
     grid_cap = sms * (per_sm > 0 ? per_sm : 1);
   }
+  CUtensorMap map;
+  if (!make_input_map(&map, a)) return cudaErrorInvalidValue;
   const int64_t tiles = a.tiles_r * a.tiles_c;
   const int grid = static_cast<int>(tiles < grid_cap ? tiles : grid_cap);
-  quant_tile_kernel<MODE><<<grid, kThreads, smem, stream>>>(a);
+  quant_tile_kernel<MODE><<<grid, kThreads, kSmem, stream>>>(map, a);
   return cudaGetLastError();
 }
 

@@ -1,10 +1,10 @@
-"""Failure detection on the GPU without a fault: the GEMM's bounded waits.
+"""Failure detection on the GPU without a fault: the kernels' bounded waits.
 
-A test hook makes the MMA issuer wait on a barrier that nothing completes.
-With a 200 ms bound every role of the kernel must give up, drain its own
-copies, free its tensor memory and return; the host then reads
-FP8BLK_ERR_TIMEOUT from the device error word, and the context must still
-run a normal GEMM correctly."""
+A test hook makes the GEMM's MMA issuer (or the quantiser's consumer warps)
+wait on a barrier that nothing completes.  With a 200 ms bound every role of
+the kernel must give up, drain its own copies, free its tensor memory and
+return; the host then reads FP8BLK_ERR_TIMEOUT from the device error word,
+and the context must still run a normal launch correctly."""
 import numpy as np
 import pytest
 import torch
@@ -52,3 +52,30 @@ def test_stalled_gemm_reports_timeout_and_recovers(layout, monkeypatch):
     assert fb.fp8blk_get_device_error() == 0
     ref = oracle.gemm(layout, qa, sa, qb, sb)
     assert_gemm_close(d.float().cpu().numpy(), ref, "after timeout")
+
+
+@pytest.mark.parametrize("kind", ["act_row", "act_both", "weight"])
+def test_stalled_quantiser_reports_timeout_and_recovers(kind, monkeypatch):
+    require_cuda()
+    rng = np.random.default_rng(12)
+    x = workloads.activation(rng, 384, 640)
+    X = torch.from_numpy(x).view(torch.bfloat16).cuda()
+
+    def run():
+        if kind == "weight":
+            return fb.fp8blk_quantize_weight_128x128(X)
+        q, s, qT, sT = fb.fp8blk_quantize_act_1x128(X, fb.ROWWISE if kind == "act_row" else fb.BOTH)
+        return q, s
+
+    assert fb.fp8blk_get_device_error() == 0
+    monkeypatch.setenv("FP8BLK_TEST_INJECT_STALL", "1")
+    monkeypatch.setenv("FP8BLK_WAIT_TIMEOUT_MS", "200")
+    run()
+    assert fb.fp8blk_get_device_error() == TIMEOUT_STATUS
+    assert fb.fp8blk_get_device_error() == 0
+    monkeypatch.delenv("FP8BLK_TEST_INJECT_STALL")
+    q, s = run()
+    assert fb.fp8blk_get_device_error() == 0
+    oq, os_ = oracle.quantize_weight(x) if kind == "weight" else oracle.quantize_act_rowwise(x)
+    assert np.array_equal(q.view(torch.uint8).cpu().numpy(), oq)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
