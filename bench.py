@@ -4,12 +4,11 @@
 One step = the four linear GEMMs of a Qwen2-1.5B-shaped decoder layer (QKV
 2048x1536, O 1536x1536, gate+up 17920x1536, down 1536x8960), each run
 forward, data-gradient and weight-gradient at 16384 tokens per GPU, with
-every quantisation the pass needs inside the step (28 kernels):
+every quantisation the pass needs inside the step (24 kernels):
 
     per linear layer (X [T,K], W [N,K], dY [T,N]):
       quantize_act_1x128(X, BOTH)          row-wise for FWD, along tokens for WGRAD
-      quantize_weight_128x128(W)           FWD operand
-      quantize_weight_128x128_t(W)         DGRAD operand
+      quantize_weight_128x128_both(W)      FWD operand and (transposed) DGRAD operand
       gemm FWD    Y  = X . W^T
       quantize_act_1x128(dY, BOTH)
       gemm DGRAD  dX = dY . W
@@ -118,10 +117,15 @@ class Program:
                      lambda x=x, m=mode, a=qx, b=sx, c=qxT, d=sxT: fb.fp8blk_quantize_act_1x128(x, m, a, b, c, d))
             if "fwd" in passes:
                 qw, sw = f(N, K), f(N // 128, K // 128, dt=torch.float32)
-                self._op(f"{g}.quant_w", "quant", N * K * (3 + 4 / 16384),
-                         lambda w=w, q=qw, s=sw: fb.fp8blk_quantize_weight_128x128(w, q, s))
             if "dgrad" in passes:
                 qwT, swT = f(K, N), f(K // 128, N // 128, dt=torch.float32)
+            if "fwd" in passes and "dgrad" in passes:     # both block layouts from one read of W
+                self._op(f"{g}.quant_w", "quant", N * K * (2 + 2 * (1 + 4 / 16384)),
+                         lambda w=w, q=qw, s=sw, qT=qwT, sT=swT: fb.fp8blk_quantize_weight_128x128_both(w, q, s, qT, sT))
+            elif "fwd" in passes:
+                self._op(f"{g}.quant_w", "quant", N * K * (3 + 4 / 16384),
+                         lambda w=w, q=qw, s=sw: fb.fp8blk_quantize_weight_128x128(w, q, s))
+            elif "dgrad" in passes:
                 self._op(f"{g}.quant_wt", "quant", N * K * (3 + 4 / 16384),
                          lambda w=w, q=qwT, s=swT: fb.fp8blk_quantize_weight_128x128_t(w, q, s))
             if "fwd" in passes:

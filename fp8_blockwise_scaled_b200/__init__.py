@@ -16,6 +16,7 @@ Layouts (row-major, dimensions multiples of 128):
       BOTH      -> all four
   fp8blk_quantize_weight_128x128(w[N,K])   -> q[N,K],  s[N/128,K/128]
   fp8blk_quantize_weight_128x128_t(w[N,K]) -> qT[K,N], sT[K/128,N/128]
+  fp8blk_quantize_weight_128x128_both(w[N,K]) -> q, s, qT, sT from one read of w
   fp8blk_gemm(layout, a[M,K], sa[K/128,M], b[N,K], sb) -> d[M,N] bfloat16
       sb = [N/128,K/128] for FWD/DGRAD, [K/128,N] for WGRAD
 """
@@ -30,6 +31,7 @@ from ._lib import (BOTH, COLWISE_T, DGRAD, FWD, ROWWISE, WGRAD, Fp8BlkError, LIB
 
 __all__ = [
     "fp8blk_quantize_act_1x128", "fp8blk_quantize_weight_128x128", "fp8blk_quantize_weight_128x128_t",
+    "fp8blk_quantize_weight_128x128_both",
     "fp8blk_gemm", "fp8blk_get_device_error", "fp8blk_version", "linear_forward", "linear_backward",
     "ROWWISE", "COLWISE_T", "BOTH", "FWD", "DGRAD", "WGRAD", "Fp8BlkError", "LIB_PATH", "status_string",
 ]
@@ -110,6 +112,20 @@ def fp8blk_quantize_weight_128x128_t(w, qT=None, sT=None, stream=None):
     check(lib.fp8blk_quantize_weight_128x128_t(_ptr(w), n, k, w.stride(0), _ptr(qT), _ptr(sT),
                                                _stream_handle(stream)))
     return qT, sT
+
+
+def fp8blk_quantize_weight_128x128_both(w, q=None, s=None, qT=None, sT=None, stream=None):
+    """Both block layouts from one read of w.  Returns (q[N,K], s[N/128,K/128], qT[K,N], sT[K/128,N/128])."""
+    w = _bf16_2d(w)
+    _need_cuda(w)
+    n, k = w.shape
+    q = _out(q, (n, k), E4M3, w.device)
+    s = _out(s, (n // 128, k // 128), torch.float32, w.device)
+    qT = _out(qT, (k, n), E4M3, w.device)
+    sT = _out(sT, (k // 128, n // 128), torch.float32, w.device)
+    check(lib.fp8blk_quantize_weight_128x128_both(_ptr(w), n, k, w.stride(0), _ptr(q), _ptr(s), _ptr(qT), _ptr(sT),
+                                                  _stream_handle(stream)))
+    return q, s, qT, sT
 
 
 def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None):

@@ -37,6 +37,7 @@ def _load() -> ctypes.CDLL:
         "fp8blk_quantize_act_1x128": [P, I64, I64, I64, I, P, P, P, P, P],
         "fp8blk_quantize_weight_128x128": [P, I64, I64, I64, P, P, P],
         "fp8blk_quantize_weight_128x128_t": [P, I64, I64, I64, P, P, P],
+        "fp8blk_quantize_weight_128x128_both": [P, I64, I64, I64, P, P, P, P, P],
         "fp8blk_gemm": [I, I64, I64, I64, P, P, P, P, P, I64, P],
         "fp8blk_get_device_error": [P],
         "fp8blk_status_string": [I],

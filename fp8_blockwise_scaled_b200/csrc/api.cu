@@ -1,6 +1,7 @@
 // C-ABI entry points of libfp8blk (declared in include/fp8blk.h): argument
 // checks, device check, dispatch to the kernels on the caller's stream.
 #include <cstdlib>
+#include <tuple>
 #include <cstring>
 
 #include "../../include/fp8blk.h"
@@ -115,36 +116,42 @@ fp8blk_status fp8blk_quantize_act_1x128(const void* x, int64_t rows, int64_t col
   return launch_status(fp8blk::launch_quant(kmode, a, static_cast<cudaStream_t>(stream)));
 }
 
+// Weight quantisation in 128x128 blocks: (q, s) in place and/or (qT, sT)
+// transposed; a null pair is not written.
 static fp8blk_status quantize_weight(const void* w, int64_t n, int64_t k, int64_t ldw, uint8_t* q, float* s,
-                                     bool transposed, void* stream) {
+                                     uint8_t* qT, float* sT, void* stream) {
   fp8blk_status st = check_quant_common(w, n, k, ldw);
   if (st != FP8BLK_OK) return st;
-  if (!q || !s) return FP8BLK_ERR_INVALID_ARG;
-  if (!aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u)) return FP8BLK_ERR_ALIGN;
-  if ((st = check_device()) != FP8BLK_OK) return st;
-  QuantArgs a{static_cast<const uint16_t*>(w), n, k, ldw, nullptr, nullptr, nullptr, nullptr, n / 128, k / 128};
-  if ((st = set_quant_waits(a)) != FP8BLK_OK) return st;
-  int kmode;
-  if (transposed) {
-    a.q_t = q;
-    a.s_t = s;
-    kmode = fp8blk::Q_BLKT;
-  } else {
-    a.q_row = q;
-    a.s_row = s;
-    kmode = fp8blk::Q_BLK;
+  int kmode = 0;
+  for (auto [codes, scales, bit] : {std::tuple{q, s, int(fp8blk::Q_BLK)}, std::tuple{qT, sT, int(fp8blk::Q_BLKT)}}) {
+    if (!codes && !scales) continue;
+    if (!codes || !scales) return FP8BLK_ERR_INVALID_ARG;
+    if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return FP8BLK_ERR_ALIGN;
+    kmode |= bit;
   }
+  if (!kmode) return FP8BLK_ERR_INVALID_ARG;
+  if ((st = check_device()) != FP8BLK_OK) return st;
+  QuantArgs a{static_cast<const uint16_t*>(w), n, k, ldw, q, s, qT, sT, n / 128, k / 128};
+  if ((st = set_quant_waits(a)) != FP8BLK_OK) return st;
   return launch_status(fp8blk::launch_quant(kmode, a, static_cast<cudaStream_t>(stream)));
 }
 
 fp8blk_status fp8blk_quantize_weight_128x128(const void* w, int64_t n, int64_t k, int64_t ldw, uint8_t* q,
                                              float* s, void* stream) {
-  return quantize_weight(w, n, k, ldw, q, s, false, stream);
+  if (!q || !s) return FP8BLK_ERR_INVALID_ARG;
+  return quantize_weight(w, n, k, ldw, q, s, nullptr, nullptr, stream);
 }
 
 fp8blk_status fp8blk_quantize_weight_128x128_t(const void* w, int64_t n, int64_t k, int64_t ldw, uint8_t* qT,
                                                float* sT, void* stream) {
-  return quantize_weight(w, n, k, ldw, qT, sT, true, stream);
+  if (!qT || !sT) return FP8BLK_ERR_INVALID_ARG;
+  return quantize_weight(w, n, k, ldw, nullptr, nullptr, qT, sT, stream);
+}
+
+fp8blk_status fp8blk_quantize_weight_128x128_both(const void* w, int64_t n, int64_t k, int64_t ldw, uint8_t* q,
+                                                  float* s, uint8_t* qT, float* sT, void* stream) {
+  if (!q || !s || !qT || !sT) return FP8BLK_ERR_INVALID_ARG;
+  return quantize_weight(w, n, k, ldw, q, s, qT, sT, stream);
 }
 
 fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uint8_t* a, const float* sa,

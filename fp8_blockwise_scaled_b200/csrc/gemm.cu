@@ -58,18 +58,23 @@ constexpr int BM = 128;
 constexpr int BK = 128;
 constexpr int kEpiWarps = 8;
 constexpr int kSRing = 8;        // scale ring depth (K-blocks)
-// Two thread layouts.  Plain: 320 threads (producer, MMA issuer, 8 promotion
-// warps), 168 registers each.  Split: 384 threads; warpgroup 0 (producer, MMA
-// issuer, two idle warps) hands registers to the two promotion warpgroups
-// with setmaxnreg, which pays for double-buffered TMEM reads.  The launch
-// allocates 168 per thread (ptxas pins it when setmaxnreg is used).
+// Two thread layouts.  Plain: 352 threads (operand producer, MMA issuer, 8
+// promotion warps, scale producer).  Split: 384 threads; warpgroup 0 (operand
+// producer, MMA issuer, scale producer, one idle warp) hands registers to the
+// two promotion warpgroups with setmaxnreg, which pays for double-buffered
+// TMEM reads.  The launch allocates 168 per thread (ptxas pins it when
+// setmaxnreg is used).  The scale producer runs ahead of the operand ring by
+// up to the scale ring's depth: the scales' small loads queue behind the
+// operand traffic in L2, and issued in step with the operand stages they
+// arrived late for the promotion.
 constexpr int kLowRegs = 56;
 constexpr int kHighRegs = 224;
 static_assert(128 * kLowRegs + 256 * kHighRegs == 384 * 168, "register split must match the launch allocation");
 template <bool kSplit>
 struct Layout {
-  static constexpr int kThreads = kSplit ? 384 : 320;
+  static constexpr int kThreads = kSplit ? 384 : 352;
   static constexpr int kEpiWarp0 = kSplit ? 4 : 2;
+  static constexpr int kScaleWarp = kSplit ? 2 : 10;
 };
 
 template <int BN>
@@ -126,19 +131,6 @@ struct GemmParams {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
-}
-
-__device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(smem_dst)), "l"(gsrc) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gsrc) : "memory");
-}
-
-// The mbarrier receives one arrival from this thread once all its earlier cp.async copies have landed.
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 // tcgen05.wait::ld, tied to the registers it makes valid so that the
@@ -218,6 +210,67 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&v)[8]) {
 
 }  // namespace
 
+// Scale producer (one warp): fills the scale ring, up to kSRing K-blocks ahead
+// of the promotion.  The per-row A scales (and the per-column B scales of
+// WGRAD) come by TMA bulk copies, so they travel the same path as the operand
+// tiles instead of queueing behind them as small loads; the two per-block B
+// scales of FWD/DGRAD are read 32 K-blocks at a time, one per lane, and handed
+// out by shuffle.  Returns after its last copies have landed.
+template <int BN, bool kWgrad, typename Coords>
+__device__ __forceinline__ void scale_feed(Ctrl* ctrl, const GemmParams& p, int first_tile, int tile_step, int tiles,
+                                           int kblocks, Coords coords, volatile int* abort, int lane) {
+  int slot = 0;
+  uint32_t sphase = 0;
+  int64_t issued = 0;
+  bool ok = true;
+  [[maybe_unused]] float sb0 = 0.0f, sb1 = 0.0f;   // FWD/DGRAD: B scales of K-blocks (kb & ~31) + lane
+  for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
+    int64_t m0, n0;
+    coords(tile, m0, n0);
+    for (int kb = 0; kb < kblocks; ++kb) {
+      if constexpr (!kWgrad) {
+        if ((kb & 31) == 0) {
+          const int k = kb + lane;
+          const float* row = p.sb + (n0 / 128) * kblocks;
+          sb0 = k < kblocks ? __ldg(row + k) : 0.0f;
+          if constexpr (BN == 256) sb1 = k < kblocks ? __ldg(row + kblocks + k) : 0.0f;
+        }
+      }
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&ctrl->sempty[slot], sphase ^ 1u, abort, p.timeout_ns, p.err))) {
+        ok = false;
+        break;
+      }
+      ScaleSlot& ss = ctrl->slots[slot];
+      if constexpr (!kWgrad) {
+        const float v0 = __shfl_sync(0xFFFFFFFFu, sb0, kb & 31);
+        const float v1 = __shfl_sync(0xFFFFFFFFu, sb1, kb & 31);
+        if (lane == 0) {
+          ss.sb[0] = v0;
+          if constexpr (BN == 256) ss.sb[1] = v1;
+        }
+      }
+      if (lane == 0) {
+        constexpr uint32_t kBytes = BM * 4 + (kWgrad ? BN * 4 : 0);
+        mbar_arrive_expect_tx(&ctrl->sfull[slot], kBytes);   // releases the sb stores above
+        bulk_load(ss.sa, p.sa + static_cast<int64_t>(kb) * p.M + m0, BM * 4, &ctrl->sfull[slot]);
+        if constexpr (kWgrad) bulk_load(ss.sb, p.sb + static_cast<int64_t>(kb) * p.N + n0, BN * 4, &ctrl->sfull[slot]);
+      }
+      ++issued;
+      if (++slot == kSRing) {
+        slot = 0;
+        sphase ^= 1u;
+      }
+    }
+  }
+  // Let the copies still in flight land before the CTA's smem goes away (on
+  // the normal path the promotion has consumed them all: no wait).
+  if (lane == 0) {
+    for (int64_t j = issued > kSRing ? issued - kSRing : 0; j < issued; ++j)
+      mbar_wait_bounded(&ctrl->sfull[j % kSRing], static_cast<uint32_t>((j / kSRing) & 1), nullptr, p.timeout_ns,
+                        p.err);
+  }
+}
+
 // Tile order: groups of `group_m` M-blocks, N-blocks inside a group, M-blocks
 // fastest inside that.  The CTAs running at the same time then share each A tile
 // among ~#SMs/group_m CTAs and each B tile among group_m CTAs, instead of all
@@ -259,7 +312,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
       mbar_init(&ctrl->tempty[b], kEpiWarps);
     }
     for (int s = 0; s < kSRing; ++s) {
-      mbar_init(&ctrl->sfull[s], 32);   // one cp.async arrival per producer lane
+      mbar_init(&ctrl->sfull[s], 1);    // the scale producer's arrive + the bytes of its copies
       mbar_init(&ctrl->sempty[s], kEpiWarps);
     }
     mbar_init(&ctrl->mma_done, 1);
@@ -281,65 +334,51 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
   const uint32_t tmem_base = ctrl->tmem_base;
   volatile int* abort = &ctrl->abort;
 
-  if (warp < kEpiWarp0) {
+  if (warp < kEpiWarp0 || warp >= kEpiWarp0 + kEpiWarps) {
   if constexpr (kSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
   if (warp == 0) {
-    // ------------------------------------------------------------ producer (whole warp)
-    int stage = 0, slot = 0;
-    uint32_t phase = 0, sphase = 0;
-    int64_t issued = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-      int mb, nb;
-      tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
-      const int64_t m0 = static_cast<int64_t>(mb) * BM, n0 = static_cast<int64_t>(nb) * BN;
-      for (int kb = 0; kb < kblocks; ++kb) {
-        // Scales of this K-block into the scale ring.
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&ctrl->sempty[slot], sphase ^ 1u, abort, p.timeout_ns, p.err))) {
-          ok = false;
-          break;
-        }
-        ScaleSlot& ss = ctrl->slots[slot];
-        cp_async_16(&ss.sa[lane * 4], p.sa + static_cast<int64_t>(kb) * p.M + m0 + lane * 4);
-        if constexpr (kWgrad) {
-          for (int c = lane * 4; c < BN; c += 128)
-            cp_async_16(&ss.sb[c], p.sb + static_cast<int64_t>(kb) * p.N + n0 + c);
-        } else {
-          if (lane < BN / 128) cp_async_4(&ss.sb[lane], p.sb + (n0 / 128 + lane) * kblocks + kb);
-        }
-        cp_async_arrive(&ctrl->sfull[slot]);
-        if (++slot == kSRing) {
-          slot = 0;
-          sphase ^= 1u;
-        }
-        // Operand tiles of this K-block into the stage ring.
-        if (lane == 0) {
-          ok = mbar_wait_bounded(&ctrl->empty[stage], phase ^ 1u, abort, p.timeout_ns, p.err);
-          if (ok) {
-            uint8_t* sa_tile = smem + stage * C::kStageBytes;
-            mbar_arrive_expect_tx(&ctrl->full[stage], C::kStageBytes);
-            tma_load_2d(sa_tile, &tm_a, &ctrl->full[stage], kb * BK, static_cast<int>(m0));
-            tma_load_2d(sa_tile + C::kABytes, &tm_b, &ctrl->full[stage], kb * BK, static_cast<int>(n0));
+    // ------------------------------------------------------------ operand producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(&ctrl->empty[stage], phase ^ 1u, abort, p.timeout_ns, p.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa_tile = smem + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(&ctrl->full[stage], C::kStageBytes);
+          tma_load_2d(sa_tile, &tm_a, &ctrl->full[stage], kb * BK, mb * BM);
+          tma_load_2d(sa_tile + C::kABytes, &tm_b, &ctrl->full[stage], kb * BK, nb * BN);
+          ++issued;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
           }
         }
-        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-        if (!ok) break;
-        ++issued;
-        if (++stage == C::kStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
       }
-    }
-    // Let the copies still in flight land before the CTA's smem goes away
-    // (on the normal path they have all been consumed: no wait).
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    if (lane == 0) {
+      // Let the copies still in flight land before the CTA's smem goes away
+      // (on the normal path they have all been consumed: no wait).
       const int64_t first = issued > C::kStages ? issued - C::kStages : 0;
       for (int64_t j = first; j < issued; ++j)
         mbar_wait_bounded(&ctrl->full[j % C::kStages], static_cast<uint32_t>((j / C::kStages) & 1), nullptr,
                           p.timeout_ns, p.err);
     }
+  } else if (warp == Layout<kSplit>::kScaleWarp) {
+    // ------------------------------------------------------------ scale producer (whole warp)
+    scale_feed<BN, kWgrad>(ctrl, p, blockIdx.x, gridDim.x, tiles, kblocks,
+                           [&](int tile, int64_t& m0, int64_t& n0) {
+                             int mb, nb;
+                             tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
+                             m0 = static_cast<int64_t>(mb) * BM;
+                             n0 = static_cast<int64_t>(nb) * BN;
+                           },
+                           abort, lane);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -552,7 +591,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
       mbar_init(&ctrl->tempty[b], 2 * kEpiWarps);   // promotion warps of both CTAs
     }
     for (int s = 0; s < kSRing; ++s) {
-      mbar_init(&ctrl->sfull[s], 32);
+      mbar_init(&ctrl->sfull[s], 1);
       mbar_init(&ctrl->sempty[s], kEpiWarps);
     }
     mbar_init(&ctrl->mma_done, 1);
@@ -576,64 +615,53 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
   volatile int* abort = &ctrl->abort;
   const uint32_t peer_abort = mapa_shared(smem_addr(&ctrl->abort), rank ^ 1u);
 
-  if (warp < kEpiWarp0) {
+  if (warp < kEpiWarp0 || warp >= kEpiWarp0 + kEpiWarps) {
   if constexpr (kSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
   if (warp == 0) {
-    // ------------------------------------------------------------ producer (whole warp)
-    int stage = 0, slot = 0;
-    uint32_t phase = 0, sphase = 0;
-    int64_t issued = 0;
-    bool ok = true;
-    for (int tile = pair; ok && tile < tiles; tile += npairs) {
-      const int mp = tile % num_mp, nb = tile / num_mp;
-      const int64_t m0 = static_cast<int64_t>(mp) * 2 * BM + rank * BM, n0 = static_cast<int64_t>(nb) * BN;
-      for (int kb = 0; kb < kblocks; ++kb) {
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded_pair(&ctrl->sempty[slot], sphase ^ 1u, abort, peer_abort,
-                                                            p.timeout_ns, p.err, false))) {
-          ok = false;
-          break;
-        }
-        ScaleSlot& ss = ctrl->slots[slot];
-        cp_async_16(&ss.sa[lane * 4], p.sa + static_cast<int64_t>(kb) * p.M + m0 + lane * 4);
-        if constexpr (kWgrad) {
-          for (int c = lane * 4; c < BN; c += 128)
-            cp_async_16(&ss.sb[c], p.sb + static_cast<int64_t>(kb) * p.N + n0 + c);
-        } else {
-          if (lane < BN / 128) cp_async_4(&ss.sb[lane], p.sb + (n0 / 128 + lane) * kblocks + kb);
-        }
-        cp_async_arrive(&ctrl->sfull[slot]);
-        if (++slot == kSRing) {
-          slot = 0;
-          sphase ^= 1u;
-        }
-        if (lane == 0) {
-          ok = mbar_wait_bounded_pair(&ctrl->empty[stage], phase ^ 1u, abort, peer_abort, p.timeout_ns, p.err, true);
-          if (ok) {
-            uint8_t* st = smem + stage * kPairStageBytes;
-            const uint32_t full_leader = mapa_shared(smem_addr(&ctrl->full[stage]), 0);
-            if (leader) mbar_arrive_expect_tx(&ctrl->full[stage], 2 * kPairStageBytes);
-            tma_load_2d_pair(st, &tm_a, full_leader, kb * BK, static_cast<int>(m0));
-            tma_load_2d_pair(st + kPairHalfBytes, &tm_b, full_leader, kb * BK, static_cast<int>(n0 + rank * BM));
+    // ------------------------------------------------------------ operand producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < tiles; tile += npairs) {
+        const int mp = tile % num_mp, nb = tile / num_mp;
+        const int64_t m0 = static_cast<int64_t>(mp) * 2 * BM + rank * BM, n0 = static_cast<int64_t>(nb) * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded_pair(&ctrl->empty[stage], phase ^ 1u, abort, peer_abort, p.timeout_ns, p.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + stage * kPairStageBytes;
+          const uint32_t full_leader = mapa_shared(smem_addr(&ctrl->full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&ctrl->full[stage], 2 * kPairStageBytes);
+          tma_load_2d_pair(st, &tm_a, full_leader, kb * BK, static_cast<int>(m0));
+          tma_load_2d_pair(st + kPairHalfBytes, &tm_b, full_leader, kb * BK, static_cast<int>(n0 + rank * BM));
+          ++issued;
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1u;
           }
         }
-        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-        if (!ok) break;
-        ++issued;
-        if (++stage == kPairStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
+      }
+      if (leader) {
+        // The leader's full barriers count the bytes of both CTAs: once the last
+        // stages it armed are complete, no load of the pair is in flight.
+        const int64_t first = issued > kPairStages ? issued - kPairStages : 0;
+        for (int64_t j = first; j < issued; ++j)
+          mbar_wait_bounded(&ctrl->full[j % kPairStages], static_cast<uint32_t>((j / kPairStages) & 1), nullptr,
+                            p.timeout_ns, p.err);
       }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    if (leader && lane == 0) {
-      // The leader's full barriers count the bytes of both CTAs: once the last
-      // stages it armed are complete, no load of the pair is in flight.
-      const int64_t first = issued > kPairStages ? issued - kPairStages : 0;
-      for (int64_t j = first; j < issued; ++j)
-        mbar_wait_bounded(&ctrl->full[j % kPairStages], static_cast<uint32_t>((j / kPairStages) & 1), nullptr,
-                          p.timeout_ns, p.err);
-    }
+  } else if (warp == Layout<kSplit>::kScaleWarp) {
+    // ------------------------------------------------------------ scale producer (whole warp)
+    scale_feed<BN, kWgrad>(ctrl, p, pair, npairs, tiles, kblocks,
+                           [&](int tile, int64_t& m0, int64_t& n0) {
+                             const int mp = tile % num_mp, nb = tile / num_mp;
+                             m0 = static_cast<int64_t>(mp) * 2 * BM + rank * BM;
+                             n0 = static_cast<int64_t>(nb) * BN;
+                           },
+                           abort, lane);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader CTA only)
     if (leader && lane == 0) {
@@ -642,12 +670,11 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
       uint32_t phase = 0, abuf = 0, aphase = 0;
       bool ok = true;
       if (p.inject_stall)
-        ok = mbar_wait_bounded_pair(&ctrl->never, 0, abort, peer_abort, p.timeout_ns, p.err, false);
+        ok = mbar_wait_bounded_pair(&ctrl->never, 0, abort, peer_abort, p.timeout_ns, p.err);
       for (int tile = pair; ok && tile < tiles; tile += npairs) {
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded_pair(&ctrl->full[stage], phase, abort, peer_abort, p.timeout_ns, p.err, true) ||
-              !mbar_wait_bounded_pair(&ctrl->tempty[abuf], aphase ^ 1u, abort, peer_abort, p.timeout_ns, p.err,
-                                      true)) {
+          if (!mbar_wait_bounded_pair(&ctrl->full[stage], phase, abort, peer_abort, p.timeout_ns, p.err) ||
+              !mbar_wait_bounded_pair(&ctrl->tempty[abuf], aphase ^ 1u, abort, peer_abort, p.timeout_ns, p.err)) {
             ok = false;
             break;
           }
@@ -696,8 +723,8 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
 
       for (int kb = 0; kb < kblocks; ++kb) {
         const bool got =
-            mbar_wait_bounded_pair(&ctrl->sfull[slot], sphase, abort, peer_abort, p.timeout_ns, p.err, false) &&
-            mbar_wait_bounded_pair(&ctrl->tfull[abuf], aphase, abort, peer_abort, p.timeout_ns, p.err, true);
+            mbar_wait_bounded_pair(&ctrl->sfull[slot], sphase, abort, peer_abort, p.timeout_ns, p.err) &&
+            mbar_wait_bounded_pair(&ctrl->tfull[abuf], aphase, abort, peer_abort, p.timeout_ns, p.err);
         if (!__all_sync(0xFFFFFFFFu, got)) {
           ok = false;
           break;

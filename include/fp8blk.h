@@ -110,6 +110,16 @@ fp8blk_status fp8blk_quantize_weight_128x128_t(const void* w, int64_t n, int64_t
                                                uint8_t* qT, float* sT, void* stream);
 
 /*
+ * Both of the above from one read of w (a training step needs both layouts:
+ * (q, s) for the forward GEMM, (qT, sT) for the data-gradient GEMM).  The
+ * outputs are bitwise those of the two separate calls.  Alignment and
+ * argument errors as for the separate calls; all four outputs are required.
+ */
+fp8blk_status fp8blk_quantize_weight_128x128_both(const void* w, int64_t n, int64_t k, int64_t ldw,
+                                                  uint8_t* q, float* s, uint8_t* qT, float* sT,
+                                                  void* stream);
+
+/*
  * Blockwise-scaled FP8 GEMM with bf16 output ([EXPL] "核心挑战：Scale Factor
  * 管理": the output is linear(x_fp8 * x_scale, w_fp8 * w_scale); [DIGEST]
  * "方法关键点": the linear-layer GEMMs run in E4M3):

@@ -22,7 +22,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for want in ("fp8blk_quantize_act_1x128", "fp8blk_quantize_weight_128x128",
-                 "fp8blk_quantize_weight_128x128_t", "fp8blk_gemm", "fp8blk_get_device_error",
+                 "fp8blk_quantize_weight_128x128_t", "fp8blk_quantize_weight_128x128_both",
+                 "fp8blk_gemm", "fp8blk_get_device_error",
                  "fp8blk_status_string"):
         assert want in names
 
@@ -76,6 +77,19 @@ def test_quantize_weight_argument_errors(fn):
     assert f(NULL, 128, 128, 128, ALIGNED, ALIGNED, S) == 1
     assert f(ALIGNED, 128, 128, 128, NULL, ALIGNED, S) == 1
     assert f(ALIGNED, 128, 128, 128, MISALIGNED, ALIGNED, S) == 3
+
+
+def test_quantize_weight_both_argument_errors():
+    f = _lib.lib.fp8blk_quantize_weight_128x128_both
+    A = ALIGNED
+    assert f(A, 128, 200, 256, A, A, A, A, S) == 2
+    assert f(NULL, 128, 128, 128, A, A, A, A, S) == 1
+    for i in range(4):                      # every output is required
+        outs = [A, A, A, A]
+        outs[i] = NULL
+        assert f(A, 128, 128, 128, *outs, S) == 1
+    assert f(A, 128, 128, 128, A, A, MISALIGNED, A, S) == 3
+    assert f(A, 128, 128, 132, A, A, A, A, S) == 3          # ldw % 8
 
 
 @pytest.mark.parametrize("args,code", [

@@ -45,6 +45,9 @@ def _check_weight(w_bits, what):
     assert_bits_equal(f32(s), os_, f"{what} weight scales")
     assert_bits_equal(u8(qT), oqT, f"{what} weight^T codes")
     assert_bits_equal(f32(sT), osT, f"{what} weight^T scales")
+    q2, s2, qT2, sT2 = fb.fp8blk_quantize_weight_128x128_both(w)
+    for got, want, name in ((q2, oq, "codes"), (s2, os_, "scales"), (qT2, oqT, "^T codes"), (sT2, osT, "^T scales")):
+        assert_bits_equal(u8(got) if "codes" in name else f32(got), want, f"{what} weight (both) {name}")
     assert fb.fp8blk_get_device_error() == 0
 
 
