@@ -167,14 +167,19 @@ class Program:
     def _op(self, label, kind, units, fn):
         self.ops.append((label, kind, units, fn))
 
-    def run(self, events=None):
-        """One step.  events: list of (start, end) CUDA event pairs, one per op, or None."""
+    def run(self, events=None, reduce=True):
+        """One step.  events: list of (start, end) CUDA event pairs, one per op, or None.
+        reduce: sum the weight gradients over ranks (data parallel) at the end."""
         for i, (_, _, _, fn) in enumerate(self.ops):
             if events is not None:
                 events[i][0].record()
             fn()
             if events is not None:
                 events[i][1].record()
+        if reduce:
+            self.reduce()
+
+    def reduce(self):
         if self.world > 1:
             from fp8_blockwise_scaled_b200.dp import allreduce_weight_grads
             allreduce_weight_grads(self.grads)
@@ -332,19 +337,37 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nops)]
           for _ in range(args.steps)]
     st = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # Per-op device times: eager launches, one event pair around each op.
+    for i in range(args.steps):
+        flush.zero_()
+        prog.run(ev[i], reduce=False)
+    barrier()
+    per_op_ms = [[a.elapsed_time(b) for a, b in ev[i]] for i in range(args.steps)]
+    # The timed steps: the step's kernels as one CUDA graph (consecutive kernels
+    # linked by programmatic dependent launch), replayed once per step.
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            prog.run(reduce=False)
+        graph.replay()                         # one untimed replay
+    barrier()
     sampler = ClockSampler(local_rank)
     time.sleep(0.3)
     barrier()
     for i in range(args.steps):
         flush.zero_()                          # L2 flush, outside the timed events
         st[i][0].record(stream)
-        prog.run(ev[i])
+        if graph is not None:
+            graph.replay()
+        else:
+            prog.run(reduce=False)
+        prog.reduce()
         st[i][1].record(stream)
     barrier()
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in st]
     total_ms = sum(step_ms)
-    per_op_ms = [[a.elapsed_time(b) for a, b in ev[i]] for i in range(args.steps)]
     gemm_ms = sum(per_op_ms[i][j] for i in range(args.steps) for j in range(nops) if prog.ops[j][1] == "gemm")
     quant_ms = sum(per_op_ms[i][j] for i in range(args.steps) for j in range(nops) if prog.ops[j][1] == "quant")
     if world > 1:
@@ -394,6 +417,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "config": {"workload": WORKLOAD_DESC[args.workload], "tokens_per_gpu": tokens,
                    "l2": "flushed between steps (256 MiB write outside the timed events)",
                    "streams": 1, "seed": {"layer": 4, "qkv_fwd": 1, "mlp_fwd": 2, "down_bwd": 3}[args.workload],
+                   "launch": "eager" if graph is None else
+                             "one CUDA graph per step, programmatic dependent launch between kernels",
                    "parallelism": f"dp{world}" if world > 1 else "single-gpu"},
         "frac_of_spec_fp8_peak": value / SPEC_FP8_TFLOPS,
         "roofline": {"bound": "tensor", "kernel": "gemm_blockwise_kernel", "achieved": gemm_tflops,
@@ -461,6 +486,7 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=0, help="tokens per GPU (default 16384 for layer, else 8192)")
     ap.add_argument("--sweep", action="store_true", help="token sweep of the layer GEMMs (one JSON line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of the step's CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -70,6 +70,14 @@ fp8blk_status launch_status(cudaError_t e) {
   return FP8BLK_ERR_LAUNCH;
 }
 
+// Programmatic dependent launch of every kernel: off unless FP8BLK_PDL=1.
+// Measured on the decoder-layer step (one CUDA graph per step) it cost ~2%:
+// dependents launched early occupy the SMs that free up while they wait.
+int pdl_enabled() {
+  const char* e = std::getenv("FP8BLK_PDL");
+  return e ? std::atoi(e) != 0 : 0;
+}
+
 // Bounded device waits of a quantiser launch (and the stall test hook).
 fp8blk_status set_quant_waits(QuantArgs& a) {
   a.timeout_ns = wait_timeout_ns();
@@ -77,6 +85,7 @@ fp8blk_status set_quant_waits(QuantArgs& a) {
   if (!a.err) return FP8BLK_ERR_CUDA;
   a.inject_stall = 0;
   if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) a.inject_stall = std::atoi(e) != 0;
+  a.pdl = pdl_enabled();
   return FP8BLK_OK;
 }
 
@@ -185,6 +194,7 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   g.tmem_db = -1;
   g.pair = 0;   // pair tiles measured slower (cross-SM hand-offs per K-block); opt in with FP8BLK_GEMM_PAIR=1
   g.group_m = 0;
+  g.pdl = pdl_enabled();
   if (const char* e = std::getenv("FP8BLK_GEMM_PAIR")) g.pair = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_GROUP_M")) g.group_m = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);

@@ -291,6 +291,19 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
       : "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Blocks until the grid this one depends on (the previous kernel of the
+// stream, when this one was launched with programmatic stream serialization)
+// has completed and its memory is visible; returns at once otherwise.  Every
+// thread that touches global memory produced or read by earlier kernels
+// calls it first.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next kernel of the stream, if launched with programmatic stream
+// serialization, start its prologue once every CTA of this grid has called it
+// (or exited); that kernel still waits in griddep_wait for this one to finish.
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // ------------------------------------------------------------------ misc
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   uint4 v;

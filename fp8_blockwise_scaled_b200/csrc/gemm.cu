@@ -331,6 +331,10 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
+  // The prologue above touched no global memory; from here on the previous
+  // kernel's outputs are read and this kernel's outputs written.
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
   const uint32_t tmem_base = ctrl->tmem_base;
   volatile int* abort = &ctrl->abort;
 
@@ -611,6 +615,8 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
   __syncthreads();
   cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after_sync();
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
   const uint32_t tmem_base = ctrl->tmem_base;
   volatile int* abort = &ctrl->abort;
   const uint32_t peer_abort = mapa_shared(smem_addr(&ctrl->abort), rank ^ 1u);
@@ -851,7 +857,16 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, group_m};
   const int64_t tiles = (g.M / BM) * (g.N / BN);
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-  gemm_blockwise_kernel<BN, kWgrad, kSplit><<<grid, Layout<kSplit>::kThreads, kSmem, stream>>>(ta, tb, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(Layout<kSplit>::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  cfg.numAttrs = set_pdl_attr(attr, g.pdl);
+  cfg.attrs = attr;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<BN, kWgrad, kSplit>, ta, tb, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -876,13 +891,13 @@ cudaError_t launch_pair(const GemmArgs& g, cudaStream_t stream) {
   cfg.blockDim = dim3(Layout<kSplit>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1 + set_pdl_attr(attr + 1, g.pdl);
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kWgrad, kSplit>, ta, tb, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -21,6 +21,7 @@ struct QuantArgs {
   uint64_t timeout_ns;   // bound on every device-side wait
   int inject_stall;      // test hook: the consumers wait on a barrier nothing completes
   unsigned int* err;     // device error word
+  int pdl;               // 1 = launch with programmatic stream serialization
 };
 
 cudaError_t launch_quant(int mode, const QuantArgs& a, cudaStream_t stream);
@@ -40,10 +41,21 @@ struct GemmArgs {
   int tmem_db;                // -1 = choose, 0/1 = single/double-buffered TMEM reads
   int pair;                   // 1 = use 256 x 256 pair tiles when the shape allows, 0 = never
   int group_m;                // tile order: M-blocks per group (0 = default)
+  int pdl;                    // 1 = launch with programmatic stream serialization
   unsigned int* err;          // device error word
 };
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream);
+
+// Fills attr[0] with programmatic stream serialization when `enable` (the
+// kernel may start its prologue while the previous kernel of the stream
+// finishes; it waits for it in griddep_wait) and returns the attribute count.
+inline unsigned int set_pdl_attr(cudaLaunchAttribute* attr, int enable) {
+  if (!enable) return 0;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  return 1;
+}
 
 // The driver's cuTensorMapEncodeTiled (looked up once), or null if unavailable.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();

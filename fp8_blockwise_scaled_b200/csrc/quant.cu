@@ -204,9 +204,12 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
     ctrl->abort = 0;
     fence_mbar_init();
     tma_prefetch_map(&tm_x);
+    griddep_wait();                              // the input may come from the previous kernel
     for (int64_t tile = blockIdx.x; issued < S && tile < tiles; tile += gridDim.x) load_tile(issued++, tile);
   }
   __syncthreads();
+  griddep_wait();                                // before any global write
+  if (t == 0) griddep_launch_dependents();
   volatile int* abort = &ctrl->abort;
 
   // -------------------------------------------------------------- consumers
@@ -435,7 +438,16 @@ cudaError_t launch_mode(const QuantArgs& a, cudaStream_t stream) {
   if (!make_input_map(&map, a)) return cudaErrorInvalidValue;
   const int64_t tiles = a.tiles_r * a.tiles_c;
   const int grid = static_cast<int>(tiles < grid_cap ? tiles : grid_cap);
-  quant_tile_kernel<MODE><<<grid, kThreads, kSmem, stream>>>(map, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  cfg.numAttrs = set_pdl_attr(attr, a.pdl);
+  cfg.attrs = attr;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, quant_tile_kernel<MODE>, map, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
