@@ -58,23 +58,26 @@ constexpr int BM = 128;
 constexpr int BK = 128;
 constexpr int kEpiWarps = 8;
 constexpr int kSRing = 8;        // scale ring depth (K-blocks)
-// Two thread layouts.  Plain: 352 threads (operand producer, MMA issuer, 8
-// promotion warps, scale producer).  Split: 384 threads; warpgroup 0 (operand
-// producer, MMA issuer, scale producer, one idle warp) hands registers to the
-// two promotion warpgroups with setmaxnreg, which pays for double-buffered
-// TMEM reads.  The launch allocates 168 per thread (ptxas pins it when
-// setmaxnreg is used).  The scale producer runs ahead of the operand ring by
-// up to the scale ring's depth: the scales' small loads queue behind the
-// operand traffic in L2, and issued in step with the operand stages they
-// arrived late for the promotion.
+// Two thread layouts, 384 threads each.  Plain: A-operand producer, MMA
+// issuer, 8 promotion warps, scale producer, B-operand producer.  Split:
+// warpgroup 0 (A producer, MMA issuer, scale producer, B producer) hands
+// registers to the two promotion warpgroups with setmaxnreg, which pays for
+// double-buffered TMEM reads.  The launch allocates 168 per thread (ptxas
+// pins it when setmaxnreg is used).
+// Two operand producers: one thread's stream of TMA box loads completes
+// about one box per ~350 cycles whatever the box size (measured on B200:
+// 16 KB boxes 46 B/clk per issuing thread, two issuing warps 76 B/clk), so
+// A and B tiles are issued by different warps.  The scale producer runs
+// ahead of the operand ring by up to the scale ring's depth.
 constexpr int kLowRegs = 56;
 constexpr int kHighRegs = 224;
 static_assert(128 * kLowRegs + 256 * kHighRegs == 384 * 168, "register split must match the launch allocation");
 template <bool kSplit>
 struct Layout {
-  static constexpr int kThreads = kSplit ? 384 : 352;
+  static constexpr int kThreads = 384;
   static constexpr int kEpiWarp0 = kSplit ? 4 : 2;
   static constexpr int kScaleWarp = kSplit ? 2 : 10;
+  static constexpr int kBWarp = kSplit ? 3 : 11;
 };
 
 template <int BN>
@@ -320,10 +323,6 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     ctrl->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_map(&tm_a);
-    tma_prefetch_map(&tm_b);
-  }
   if (warp == 1) {
     tmem_alloc(&ctrl->tmem_base, C::kTmemCols);
     tmem_relinquish();
@@ -340,9 +339,14 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
 
   if (warp < kEpiWarp0 || warp >= kEpiWarp0 + kEpiWarps) {
   if constexpr (kSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
-  if (warp == 0) {
-    // ------------------------------------------------------------ operand producer
+  if (warp == 0 || warp == Layout<kSplit>::kBWarp) {
+    // ------------------------------------------------------------ operand producers (A: warp 0, B: kBWarp)
+    // Both wait for the same free stage; the A producer arms the stage's full
+    // barrier with the bytes of both tiles (the B bytes may land first: the
+    // transaction count may go negative until the arrival).
+    const bool is_a = warp == 0;
     if (lane == 0) {
+      tma_prefetch_map(is_a ? &tm_a : &tm_b);
       int stage = 0;
       uint32_t phase = 0;
       int64_t issued = 0;
@@ -355,10 +359,13 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
             ok = false;
             break;
           }
-          uint8_t* sa_tile = smem + stage * C::kStageBytes;
-          mbar_arrive_expect_tx(&ctrl->full[stage], C::kStageBytes);
-          tma_load_2d(sa_tile, &tm_a, &ctrl->full[stage], kb * BK, mb * BM);
-          tma_load_2d(sa_tile + C::kABytes, &tm_b, &ctrl->full[stage], kb * BK, nb * BN);
+          uint8_t* st = smem + stage * C::kStageBytes;
+          if (is_a) {
+            mbar_arrive_expect_tx(&ctrl->full[stage], C::kStageBytes);
+            tma_load_2d(st, &tm_a, &ctrl->full[stage], kb * BK, mb * BM);
+          } else {
+            tma_load_2d(st + C::kABytes, &tm_b, &ctrl->full[stage], kb * BK, nb * BN);
+          }
           ++issued;
           if (++stage == C::kStages) {
             stage = 0;
@@ -603,10 +610,6 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     ctrl->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_map(&tm_a);
-    tma_prefetch_map(&tm_b);
-  }
   if (warp == 1) {
     tmem_alloc_pair(&ctrl->tmem_base, kAccBufs * BN);
     tmem_relinquish_pair();
@@ -623,9 +626,11 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
 
   if (warp < kEpiWarp0 || warp >= kEpiWarp0 + kEpiWarps) {
   if constexpr (kSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
-  if (warp == 0) {
-    // ------------------------------------------------------------ operand producer
+  if (warp == 0 || warp == Layout<kSplit>::kBWarp) {
+    // ------------------------------------------------------------ operand producers (A: warp 0, B half: kBWarp)
+    const bool is_a = warp == 0;
     if (lane == 0) {
+      tma_prefetch_map(is_a ? &tm_a : &tm_b);
       int stage = 0;
       uint32_t phase = 0;
       int64_t issued = 0;
@@ -640,9 +645,12 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
           }
           uint8_t* st = smem + stage * kPairStageBytes;
           const uint32_t full_leader = mapa_shared(smem_addr(&ctrl->full[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(&ctrl->full[stage], 2 * kPairStageBytes);
-          tma_load_2d_pair(st, &tm_a, full_leader, kb * BK, static_cast<int>(m0));
-          tma_load_2d_pair(st + kPairHalfBytes, &tm_b, full_leader, kb * BK, static_cast<int>(n0 + rank * BM));
+          if (is_a) {
+            if (leader) mbar_arrive_expect_tx(&ctrl->full[stage], 2 * kPairStageBytes);
+            tma_load_2d_pair(st, &tm_a, full_leader, kb * BK, static_cast<int>(m0));
+          } else {
+            tma_load_2d_pair(st + kPairHalfBytes, &tm_b, full_leader, kb * BK, static_cast<int>(n0 + rank * BM));
+          }
           ++issued;
           if (++stage == kPairStages) {
             stage = 0;
