@@ -417,8 +417,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "config": {"workload": WORKLOAD_DESC[args.workload], "tokens_per_gpu": tokens,
                    "l2": "flushed between steps (256 MiB write outside the timed events)",
                    "streams": 1, "seed": {"layer": 4, "qkv_fwd": 1, "mlp_fwd": 2, "down_bwd": 3}[args.workload],
-                   "launch": "eager" if graph is None else
-                             "one CUDA graph per step, programmatic dependent launch between kernels",
+                   "launch": ("eager" if graph is None else "one CUDA graph per step")
+                             + (", programmatic dependent launch" if os.environ.get("FP8BLK_PDL") == "1" else ""),
                    "parallelism": f"dp{world}" if world > 1 else "single-gpu"},
         "frac_of_spec_fp8_peak": value / SPEC_FP8_TFLOPS,
         "roofline": {"bound": "tensor", "kernel": "gemm_blockwise_kernel", "achieved": gemm_tflops,
