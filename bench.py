@@ -47,6 +47,11 @@ SPEC_FP8_TFLOPS = 4500.0          # B200 dense FP8, NVIDIA's published figure
 FP8_PER_BF16 = 2.0                # nominal dense FP8 / BF16 tensor throughput ratio
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
+# DRAM traffic of the 12 GEMM launches of one decoder-layer step at 16384 tokens
+# (dram__bytes_read.sum + dram__bytes_write.sum, one ncu pass over the launches of
+# one step; profiles/gemm_dram_layer_16384.md), for the GEMM kernel of commit
+# a7b876c; algorithmic minimum 2.59 GB (codes read once, bf16 outputs written once).
+GEMM_STEP_DRAM_BYTES_16384 = 2.94e9
 
 WORKLOAD_DESC = {
     "layer": "qwen2-1.5b-shaped decoder layer linears (qkv 2048x1536, o 1536x1536, gate_up 17920x1536, "
@@ -422,7 +427,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "parallelism": f"dp{world}" if world > 1 else "single-gpu"},
         "frac_of_spec_fp8_peak": value / SPEC_FP8_TFLOPS,
         "roofline": {"bound": "tensor", "kernel": "gemm_blockwise_kernel", "achieved": gemm_tflops,
-                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak, "traffic": None,
+                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
+                     "traffic": GEMM_STEP_DRAM_BYTES_16384 if (args.workload == "layer" and tokens == 16384) else None,
+                     "traffic_scope": "bytes per step, the 12 GEMM launches together (achieved is over the same launches)",
                      "peak_source": f"{peak_src} bf16 sustained x {FP8_PER_BF16:g} (nominal fp8/bf16 ratio)",
                      "frac_of_spec_fp8": gemm_tflops / SPEC_FP8_TFLOPS},
         "quant": {"kernel": "quant_tile_kernel", "achieved_gbs": quant_gbs, "peak_gbs": peaks["hbm_gbs"],
