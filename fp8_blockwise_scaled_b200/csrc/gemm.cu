@@ -253,6 +253,9 @@ __device__ __forceinline__ void scale_feed(Ctrl* ctrl, const GemmParams& p, int 
         }
       }
       if (lane == 0) {
+        // The promotion warps read this slot through the generic proxy; the
+        // bulk copies below write it through the async proxy: order them.
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         constexpr uint32_t kBytes = BM * 4 + (kWgrad ? BN * 4 : 0);
         mbar_arrive_expect_tx(&ctrl->sfull[slot], kBytes);   // releases the sb stores above
         bulk_load(ss.sa, p.sa + static_cast<int64_t>(kb) * p.M + m0, BM * 4, &ctrl->sfull[slot]);

@@ -245,6 +245,9 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
     if (t == 0) {                                // and refill it with the tile S steps ahead
       const int64_t next = tile + static_cast<int64_t>(S) * gridDim.x;
       if (next < tiles && mbar_wait_bounded(&ctrl->empty[s], ph, abort, a.timeout_ns, a.err)) {
+        // The warps read the stage through the generic proxy; the TMA load
+        // rewrites it through the async proxy: order the two.
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         load_tile(s, next);
         ++issued;
       }
