@@ -16,6 +16,9 @@ Layouts (all row-major, dimensions multiples of 128):
 * ``quantize_weight(w[N,K])``        -> q[N,K] uint8, s[N/128,K/128] float32
 * ``quantize_weight_t(w[N,K])``      -> qT[K,N] uint8, sT[K/128,N/128] float32
 * ``gemm(layout, qa, sa, qb, sb)``   -> D[M,N] float64 (layout 0 FWD, 1 DGRAD, 2 WGRAD)
+
+The activation quantisers and the GEMM take a code format (``E4M3`` or
+``E5M2``; E4M3 by default); weights are always E4M3.
 """
 from __future__ import annotations
 
@@ -30,6 +33,7 @@ _SRC = os.path.join(_HERE, "oracle.cpp")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 FWD, DGRAD, WGRAD = 0, 1, 2
+E4M3, E5M2 = 0, 1
 
 _lib = None
 
@@ -59,6 +63,13 @@ def _load():
         lib.orc_quantize_act_colwise_t.argtypes = [P, I64, I64, P, P]
         lib.orc_quantize_weight.argtypes = [P, I64, I64, ctypes.c_int, P, P]
         lib.orc_gemm.argtypes = [ctypes.c_int, I64, I64, I64, P, P, P, P, P, I64, P]
+        lib.orc_e5m2_encode.argtypes = [P, I64, P]
+        lib.orc_e5m2_decode.argtypes = [P, I64, P]
+        lib.orc_group_scale_fmt.argtypes = [ctypes.c_float, ctypes.c_int]
+        lib.orc_group_scale_fmt.restype = ctypes.c_float
+        lib.orc_quantize_act_rowwise_fmt.argtypes = [P, I64, I64, ctypes.c_int, P, P]
+        lib.orc_quantize_act_colwise_t_fmt.argtypes = [P, I64, I64, ctypes.c_int, P, P]
+        lib.orc_gemm_fmt.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, I64, I64, I64, P, P, P, P, P, I64, P]
         _lib = lib
     return _lib
 
@@ -89,8 +100,22 @@ def e4m3_decode(c) -> np.ndarray:
     return out
 
 
-def group_scale(amax: float) -> np.float32:
-    return np.float32(_load().orc_group_scale(float(amax)))
+def e5m2_encode(v) -> np.ndarray:
+    v = _c(v, np.float32)
+    out = np.empty(v.shape, np.uint8)
+    _load().orc_e5m2_encode(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def e5m2_decode(c) -> np.ndarray:
+    c = _c(c, np.uint8)
+    out = np.empty(c.shape, np.float64)
+    _load().orc_e5m2_decode(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+def group_scale(amax: float, fmt: int = E4M3) -> np.float32:
+    return np.float32(_load().orc_group_scale_fmt(float(amax), int(fmt)))
 
 
 def _check_dims(*dims):
@@ -99,23 +124,23 @@ def _check_dims(*dims):
             raise ValueError(f"dimension {d} is not a positive multiple of 128")
 
 
-def quantize_act_rowwise(x):
+def quantize_act_rowwise(x, fmt: int = E4M3):
     x = _c(x, np.uint16)
     r, c = x.shape
     _check_dims(r, c)
     q = np.empty((r, c), np.uint8)
     s = np.empty((c // 128, r), np.float32)
-    _load().orc_quantize_act_rowwise(_ptr(x), r, c, _ptr(q), _ptr(s))
+    _load().orc_quantize_act_rowwise_fmt(_ptr(x), r, c, int(fmt), _ptr(q), _ptr(s))
     return q, s
 
 
-def quantize_act_colwise_t(x):
+def quantize_act_colwise_t(x, fmt: int = E4M3):
     x = _c(x, np.uint16)
     r, c = x.shape
     _check_dims(r, c)
     qt = np.empty((c, r), np.uint8)
     s = np.empty((r // 128, c), np.float32)
-    _load().orc_quantize_act_colwise_t(_ptr(x), r, c, _ptr(qt), _ptr(s))
+    _load().orc_quantize_act_colwise_t_fmt(_ptr(x), r, c, int(fmt), _ptr(qt), _ptr(s))
     return qt, s
 
 
@@ -139,7 +164,7 @@ def quantize_weight_t(w):
     return qt, st
 
 
-def gemm(layout: int, qa, sa, qb, sb, rows=None) -> np.ndarray:
+def gemm(layout: int, qa, sa, qb, sb, rows=None, a_fmt: int = E4M3, b_fmt: int = E4M3) -> np.ndarray:
     """D = dequant(A) . dequant(B)^T in fp64; ``rows`` selects output rows (default all)."""
     qa = _c(qa, np.uint8)
     qb = _c(qb, np.uint8)
@@ -163,5 +188,6 @@ def gemm(layout: int, qa, sa, qb, sb, rows=None) -> np.ndarray:
             raise ValueError("row index out of range")
         nrows, rp = rows_arr.size, _ptr(rows_arr)
     d = np.empty((nrows, n), np.float64)
-    _load().orc_gemm(layout, m, n, k, _ptr(qa), _ptr(sa), _ptr(qb), _ptr(sb), rp, nrows, _ptr(d))
+    _load().orc_gemm_fmt(layout, int(a_fmt), int(b_fmt), m, n, k, _ptr(qa), _ptr(sa), _ptr(qb), _ptr(sb), rp,
+                         nrows, _ptr(d))
     return d

@@ -22,11 +22,13 @@
 // (R3, R4); the sign of zero is kept (R5); NaN/Inf inputs are outside the
 // contract (R6); every dimension is a multiple of 128 (R11); per-row scales
 // are stored block-major S[kb][row] and block scales row-major S[nb][kb]
-// (R12).
+// (R12); E5M2 codes (for gradients) follow the same rule with that format's
+// largest value, 57344, in place of 448 (R15).
 //
 // Parity pins: every function here is pinned by tests/test_oracle_*.py
 // against the pages' constants, closed forms, invariants, torch's CPU
-// float8_e4m3fn cast (a library routine) and brute-force fp64 matmuls.
+// float8_e4m3fn and float8_e5m2 casts (library routines) and brute-force
+// fp64 matmuls.
 
 #include <algorithm>
 #include <atomic>
@@ -127,6 +129,57 @@ uint8_t e4m3_encode(float v) {
   return sign | code;
 }
 
+// ---------------------------------------------------------------- E5M2 codec
+// [EXPL] "Blackwell 的 FP8 Tensor Core", list "FP8 有两种格式": E5M2
+// (float8_e5m2) has 5 exponent bits and 2 mantissa bits, largest value 57344,
+// wide range and low precision, meant for gradients.  57344 = 1.75 * 2^15
+// forces exponent bias 15 with the top exponent field (31) reserved for
+// infinities and NaN, as in IEEE binary formats.  Byte layout: s eeeee mm.
+//   normal     (e = 1..30):  (-1)^s * 2^(e-15) * (1 + m/4)
+//   subnormal  (e = 0)    :  (-1)^s * 2^(-14) * (m/4)
+//   e = 31: m = 0 infinity, m != 0 NaN (never produced: the quantiser clamps).
+constexpr double kE5M2Max = 57344.0;
+
+double e5m2_decode(uint8_t c) {
+  const int s = c >> 7, e = (c >> 2) & 0x1F, m = c & 3;
+  double mag;
+  if (e == 31) mag = (m == 0) ? HUGE_VAL : std::nan("");
+  else mag = (e == 0) ? std::ldexp(m / 4.0, -14) : std::ldexp(1.0 + m / 4.0, e - 15);
+  return s ? -mag : mag;
+}
+
+// fp32 -> E5M2, round to nearest with ties to the even mantissa, sign kept on
+// zero results; magnitudes above 57344 saturate to 57344 (as for E4M3, only
+// direct codec calls reach that branch).
+uint8_t e5m2_encode(float v) {
+  const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+  const double a = std::fabs(static_cast<double>(v));
+  if (!(a <= kE5M2Max)) return sign | 0x7B;
+  // The representable magnitudes in [2^e, 2^(e+1)) are k * 2^(e-2), k = 4..7;
+  // below 2^-14 they are k * 2^-16, k = 0..3 (subnormals).
+  int e;
+  std::frexp(a, &e);
+  int exp2 = e - 1;
+  if (a == 0.0 || exp2 < -14) {
+    // Subnormal grid, spacing 2^-16; k = 4 lands on 2^-14, the first normal code 0x04.
+    double k = round_half_even(std::ldexp(a, 16));
+    return sign | static_cast<uint8_t>(k);
+  }
+  double k = round_half_even(std::ldexp(a, 2 - exp2));  // in [4, 8]
+  if (k == 8.0) {
+    k = 4.0;
+    exp2 += 1;
+  }
+  uint8_t code = static_cast<uint8_t>(((exp2 + 15) << 2) | (static_cast<int>(k) - 4));
+  if (code > 0x7B) code = 0x7B;  // 61440 and above would be infinity
+  return sign | code;
+}
+
+// The two formats, selected by `fmt`: 0 = E4M3, 1 = E5M2.
+double fmt_max(int fmt) { return fmt ? kE5M2Max : kE4M3Max; }
+double fmt_decode(int fmt, uint8_t c) { return fmt ? e5m2_decode(c) : e4m3_decode(c); }
+uint8_t fmt_encode(int fmt, float v) { return fmt ? e5m2_encode(v) : e4m3_encode(v); }
+
 // ---------------------------------------------------------------- one group
 // [EXPL] "核心挑战：Scale Factor 管理" (_quantize) and "常见错误：直接转换而不加
 // Scale": scale = amax / 448, floored at 1e-12; the value cast to E4M3 is
@@ -135,16 +188,20 @@ uint8_t e4m3_encode(float v) {
 // scaling of the block itself, with no history.
 constexpr float kScaleFloor = 1e-12f;  // fl32(1e-12) = 0x2B8CBCCC
 
-float group_scale(float amax) {
-  float s = amax / 448.0f;  // IEEE binary32 division, round to nearest even
+// For E5M2 the same rule divides by that format's largest value, 57344 (the
+// pages give the rule with E4M3's 448 and name E5M2's maximum; reading R15).
+float group_scale(float amax, int fmt = 0) {
+  const float fmax = static_cast<float>(fmt_max(fmt));
+  float s = amax / fmax;  // IEEE binary32 division, round to nearest even
   return s < kScaleFloor ? kScaleFloor : s;
 }
 
-uint8_t quantize_value(float x, float s) {
+uint8_t quantize_value(float x, float s, int fmt = 0) {
+  const float fmax = static_cast<float>(fmt_max(fmt));
   float v = x / s;  // IEEE binary32 division
-  if (v > 448.0f) v = 448.0f;
-  if (v < -448.0f) v = -448.0f;
-  return e4m3_encode(v);
+  if (v > fmax) v = fmax;
+  if (v < -fmax) v = -fmax;
+  return fmt_encode(fmt, v);
 }
 
 constexpr int64_t kBlock = 128;
@@ -169,42 +226,66 @@ void orc_e4m3_decode(const uint8_t* c, int64_t n, double* out) {
 
 float orc_group_scale(float amax) { return group_scale(amax); }
 
-// Activations, 1x128 groups along the contiguous (feature) dimension.
-//   x [rows][cols] bf16  ->  q [rows][cols] E4M3,  s [cols/128][rows] fp32.
-void orc_quantize_act_rowwise(const uint16_t* x, int64_t rows, int64_t cols,
-                              uint8_t* q, float* s) {
+void orc_e5m2_encode(const float* v, int64_t n, uint8_t* out) {
+  const int64_t chunk = 1 << 20;
+  parallel_for((n + chunk - 1) / chunk, [&](int64_t c) {
+    int64_t lo = c * chunk, hi = std::min(n, lo + chunk);
+    for (int64_t i = lo; i < hi; ++i) out[i] = e5m2_encode(v[i]);
+  });
+}
+
+void orc_e5m2_decode(const uint8_t* c, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e5m2_decode(c[i]);
+}
+
+float orc_group_scale_fmt(float amax, int fmt) { return group_scale(amax, fmt); }
+
+// Activations, 1x128 groups along the contiguous (feature) dimension, codes in
+// format fmt (0 E4M3, 1 E5M2).
+//   x [rows][cols] bf16  ->  q [rows][cols],  s [cols/128][rows] fp32.
+void orc_quantize_act_rowwise_fmt(const uint16_t* x, int64_t rows, int64_t cols, int fmt,
+                                  uint8_t* q, float* s) {
   const int64_t groups = cols / kBlock;
   parallel_for(rows, [&](int64_t r) {
     for (int64_t g = 0; g < groups; ++g) {
       const uint16_t* xg = x + r * cols + g * kBlock;
       float amax = 0.0f;
       for (int64_t j = 0; j < kBlock; ++j) amax = std::max(amax, std::fabs(bf16_to_float(xg[j])));
-      const float sc = group_scale(amax);
+      const float sc = group_scale(amax, fmt);
       s[g * rows + r] = sc;
-      for (int64_t j = 0; j < kBlock; ++j) q[r * cols + g * kBlock + j] = quantize_value(bf16_to_float(xg[j]), sc);
+      for (int64_t j = 0; j < kBlock; ++j)
+        q[r * cols + g * kBlock + j] = quantize_value(bf16_to_float(xg[j]), sc, fmt);
     }
   });
 }
 
-// Activations, 1x128 groups along the token (row) dimension, codes written
-// transposed so that tokens are contiguous:
-//   x [rows][cols] bf16  ->  qT [cols][rows] E4M3,  s [rows/128][cols] fp32.
-void orc_quantize_act_colwise_t(const uint16_t* x, int64_t rows, int64_t cols,
-                                uint8_t* qT, float* s) {
+void orc_quantize_act_rowwise(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q, float* s) {
+  orc_quantize_act_rowwise_fmt(x, rows, cols, 0, q, s);
+}
+
+// Activations, 1x128 groups along the token (row) dimension, codes (format
+// fmt) written transposed so that tokens are contiguous:
+//   x [rows][cols] bf16  ->  qT [cols][rows],  s [rows/128][cols] fp32.
+void orc_quantize_act_colwise_t_fmt(const uint16_t* x, int64_t rows, int64_t cols, int fmt,
+                                    uint8_t* qT, float* s) {
   const int64_t groups = rows / kBlock;
   parallel_for(cols, [&](int64_t c) {
     for (int64_t g = 0; g < groups; ++g) {
       float amax = 0.0f;
       for (int64_t j = 0; j < kBlock; ++j)
         amax = std::max(amax, std::fabs(bf16_to_float(x[(g * kBlock + j) * cols + c])));
-      const float sc = group_scale(amax);
+      const float sc = group_scale(amax, fmt);
       s[g * cols + c] = sc;
       for (int64_t j = 0; j < kBlock; ++j) {
         const int64_t r = g * kBlock + j;
-        qT[c * rows + r] = quantize_value(bf16_to_float(x[r * cols + c]), sc);
+        qT[c * rows + r] = quantize_value(bf16_to_float(x[r * cols + c]), sc, fmt);
       }
     }
   });
+}
+
+void orc_quantize_act_colwise_t(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* qT, float* s) {
+  orc_quantize_act_colwise_t_fmt(x, rows, cols, 0, qT, s);
 }
 
 // Weights, 128x128 blocks.  transposed = 0:  q [n][k], s [n/128][k/128];
@@ -241,9 +322,10 @@ void orc_quantize_weight(const uint16_t* w, int64_t n, int64_t k, int transposed
 //   layout 2   (weight gradient):         sb(n, k) = sb[(k/128) * N + n]
 // rows: indices of the output rows to compute (nullptr = all M rows);
 // d receives nrows x N values in that order.
-void orc_gemm(int layout, int64_t M, int64_t N, int64_t K,
-              const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb,
-              const int64_t* rows, int64_t nrows, double* d) {
+// a_fmt / b_fmt: the code format of each operand (0 E4M3, 1 E5M2).
+void orc_gemm_fmt(int layout, int a_fmt, int b_fmt, int64_t M, int64_t N, int64_t K,
+                  const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb,
+                  const int64_t* rows, int64_t nrows, double* d) {
   const int64_t kblocks = K / kBlock;
   if (!rows) nrows = M;
   // Dequantised B, one row of K values per output column n.
@@ -252,13 +334,13 @@ void orc_gemm(int layout, int64_t M, int64_t N, int64_t K,
     for (int64_t k = 0; k < K; ++k) {
       const double scale = (layout == 2) ? sb[(k / kBlock) * N + n]
                                          : sb[(n / kBlock) * kblocks + k / kBlock];
-      bdq[n * K + k] = e4m3_decode(qb[n * K + k]) * scale;  // exact in fp64
+      bdq[n * K + k] = fmt_decode(b_fmt, qb[n * K + k]) * scale;  // exact in fp64
     }
   });
   parallel_for(nrows, [&](int64_t i) {
     const int64_t m = rows ? rows[i] : i;
     std::vector<double> adq(K);
-    for (int64_t k = 0; k < K; ++k) adq[k] = e4m3_decode(qa[m * K + k]) * sa[(k / kBlock) * M + m];
+    for (int64_t k = 0; k < K; ++k) adq[k] = fmt_decode(a_fmt, qa[m * K + k]) * sa[(k / kBlock) * M + m];
     for (int64_t n = 0; n < N; ++n) {
       const double* bn = &bdq[n * K];
       double acc = 0.0;
@@ -266,6 +348,11 @@ void orc_gemm(int layout, int64_t M, int64_t N, int64_t K,
       d[i * N + n] = acc;
     }
   });
+}
+
+void orc_gemm(int layout, int64_t M, int64_t N, int64_t K, const uint8_t* qa, const float* sa,
+              const uint8_t* qb, const float* sb, const int64_t* rows, int64_t nrows, double* d) {
+  orc_gemm_fmt(layout, 0, 0, M, N, K, qa, sa, qb, sb, rows, nrows, d);
 }
 
 }  // extern "C"
