@@ -93,7 +93,7 @@ def workload_tensors(name: str, tokens: int) -> list[dict]:
 class Program:
     """Device buffers and the ordered kernel launches of one step."""
 
-    def __init__(self, specs, device, world):
+    def __init__(self, specs, device, world, grad_e5m2=False):
         import torch
         import fp8_blockwise_scaled_b200 as fb
         self.fb, self.torch, self.world = fb, torch, world
@@ -143,11 +143,13 @@ class Program:
                 dy = self._dev(sp["dY"], device)
                 need_row_d = "dgrad" in passes
                 need_colt_d = "wgrad" in passes
-                qd = f(T, N) if need_row_d else None
+                gdt = torch.float8_e5m2 if grad_e5m2 else E4      # E5M2 gradients: the DGRAD/WGRAD A operand
+                qd = f(T, N, dt=gdt) if need_row_d else None
                 sd = f(N // 128, T, dt=torch.float32) if need_row_d else None
-                qdT = f(N, T) if need_colt_d else None
+                qdT = f(N, T, dt=gdt) if need_colt_d else None
                 sdT = f(T // 128, N, dt=torch.float32) if need_colt_d else None
-                mode_d = (fb.ROWWISE if need_row_d else 0) | (fb.COLWISE_T if need_colt_d else 0)
+                mode_d = ((fb.ROWWISE if need_row_d else 0) | (fb.COLWISE_T if need_colt_d else 0)
+                          | (fb.E5M2 if grad_e5m2 else 0))
                 self._op(f"{g}.quant_dy", "quant", T * N * (2 + (1 + 4 / 128) * (int(need_row_d) + int(need_colt_d))),
                          lambda x=dy, m=mode_d, a=qd, b=sd, c=qdT, d=sdT:
                          fb.fp8blk_quantize_act_1x128(x, m, a, b, c, d))
@@ -355,7 +357,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     tokens = args.tokens or (16384 if args.workload == "layer" else 8192)
     specs = workload_tensors(args.workload, tokens)
-    prog = Program(specs, dev, world)
+    prog = Program(specs, dev, world, grad_e5m2=args.grad_format == "e5m2")
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -472,10 +474,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if args.grad_format == "e4m3" else "e4m3+e5m2",
+        "data": "synthetic",
         "config": {"workload": WORKLOAD_DESC[args.workload], "tokens_per_gpu": tokens,
                    "l2": "flushed between steps (256 MiB write outside the timed events)",
                    "streams": 1, "seed": {"layer": 4, "qkv_fwd": 1, "mlp_fwd": 2, "down_bwd": 3}[args.workload],
+                   "grad_format": args.grad_format,
                    "launch": ("eager" if graph is None else "one CUDA graph per step")
                              + (", programmatic dependent launch" if os.environ.get("FP8BLK_PDL") == "1" else ""),
                    "parallelism": f"dp{world}" if world > 1 else "single-gpu"},
@@ -552,6 +556,8 @@ def main(argv=None):
     ap.add_argument("--sweep", action="store_true", help="token sweep of the layer GEMMs (one JSON line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of the step's CUDA graph")
+    ap.add_argument("--grad-format", choices=["e4m3", "e5m2"], default="e4m3",
+                    help="code format of the output gradient dY (the DGRAD/WGRAD A operand)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

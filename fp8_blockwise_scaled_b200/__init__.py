@@ -26,17 +26,19 @@ import ctypes
 
 import torch
 
-from ._lib import (BOTH, COLWISE_T, DGRAD, FWD, ROWWISE, WGRAD, Fp8BlkError, LIB_PATH, check,
-                   lib, status_string)
+from ._lib import (A_E5M2, B_E5M2, BOTH, COLWISE_T, DGRAD, E5M2, FWD, ROWWISE, WGRAD, Fp8BlkError, LIB_PATH,
+                   check, lib, status_string)
 
 __all__ = [
     "fp8blk_quantize_act_1x128", "fp8blk_quantize_weight_128x128", "fp8blk_quantize_weight_128x128_t",
     "fp8blk_quantize_weight_128x128_both",
     "fp8blk_gemm", "fp8blk_get_device_error", "fp8blk_version", "linear_forward", "linear_backward",
-    "ROWWISE", "COLWISE_T", "BOTH", "FWD", "DGRAD", "WGRAD", "Fp8BlkError", "LIB_PATH", "status_string",
+    "ROWWISE", "COLWISE_T", "BOTH", "E5M2", "FWD", "DGRAD", "WGRAD", "A_E5M2", "B_E5M2", "Fp8BlkError",
+    "LIB_PATH", "status_string",
 ]
 
 E4M3 = torch.float8_e4m3fn
+E5M2_DTYPE = torch.float8_e5m2
 
 
 def _stream_handle(stream) -> ctypes.c_void_p:
@@ -71,18 +73,20 @@ def _bf16_2d(x):
 
 def fp8blk_quantize_act_1x128(x, mode=ROWWISE, q_row=None, s_row=None, q_colT=None, s_colT=None,
                               stream=None):
-    """Activation quantisation in 1x128 groups.  Returns (q_row, s_row, q_colT, s_colT); unused are None."""
+    """Activation quantisation in 1x128 groups.  Returns (q_row, s_row, q_colT, s_colT); unused are None.
+    ``mode`` may include E5M2 (codes as torch.float8_e5m2, for gradients)."""
     x = _bf16_2d(x)
     _need_cuda(x)
     rows, cols = x.shape
     dev = x.device
+    code_dtype = E5M2_DTYPE if mode & E5M2 else E4M3
     if mode & ROWWISE:
-        q_row = _out(q_row, (rows, cols), E4M3, dev)
+        q_row = _out(q_row, (rows, cols), code_dtype, dev)
         s_row = _out(s_row, (cols // 128, rows), torch.float32, dev)
     else:
         q_row = s_row = None
     if mode & COLWISE_T:
-        q_colT = _out(q_colT, (cols, rows), E4M3, dev)
+        q_colT = _out(q_colT, (cols, rows), code_dtype, dev)
         s_colT = _out(s_colT, (rows // 128, cols), torch.float32, dev)
     else:
         q_colT = s_colT = None
@@ -135,8 +139,8 @@ def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None):
     n = b.shape[0]
     if b.shape[1] != k:
         raise ValueError("A and B disagree on K")
-    if a.dtype != E4M3 or b.dtype != E4M3:
-        raise ValueError("A and B must be float8_e4m3fn")
+    if a.dtype not in (E4M3, E5M2_DTYPE) or b.dtype not in (E4M3, E5M2_DTYPE):
+        raise ValueError("A and B must be float8_e4m3fn or float8_e5m2")
     want_sb = (k // 128, n) if layout == WGRAD else (n // 128, k // 128)
     if tuple(sa.shape) != (k // 128, m) or tuple(sb.shape) != want_sb:
         raise ValueError(f"scale shapes {tuple(sa.shape)}, {tuple(sb.shape)} do not match layout {layout}")
@@ -146,7 +150,8 @@ def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None):
         d = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
     elif d.dtype != torch.bfloat16 or d.dim() != 2 or d.stride(1) != 1 or tuple(d.shape) != (m, n):
         raise ValueError("d must be a bfloat16 [M,N] tensor with unit column stride")
-    check(lib.fp8blk_gemm(int(layout), m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d), d.stride(0),
+    flags = (A_E5M2 if a.dtype == E5M2_DTYPE else 0) | (B_E5M2 if b.dtype == E5M2_DTYPE else 0)
+    check(lib.fp8blk_gemm(int(layout) | flags, m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d), d.stride(0),
                           _stream_handle(stream)))
     return d
 

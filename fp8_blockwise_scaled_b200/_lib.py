@@ -11,6 +11,8 @@ LIB_PATH = _build.LIB
 
 # fp8blk_act_mode / fp8blk_layout
 ROWWISE, COLWISE_T, BOTH = 1, 2, 3
+E5M2 = 4                       # OR into an activation mode: E5M2 codes
+A_E5M2, B_E5M2 = 8, 16         # OR into a GEMM layout: that operand holds E5M2 codes
 FWD, DGRAD, WGRAD = 0, 1, 2
 
 STATUS_NAMES = {

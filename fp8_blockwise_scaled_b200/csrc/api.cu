@@ -106,8 +106,9 @@ fp8blk_status fp8blk_quantize_act_1x128(const void* x, int64_t rows, int64_t col
                                         void* stream) {
   fp8blk_status st = check_quant_common(x, rows, cols, ldx);
   if (st != FP8BLK_OK) return st;
-  if (mode != FP8BLK_ROWWISE && mode != FP8BLK_COLWISE_T && mode != FP8BLK_BOTH) return FP8BLK_ERR_INVALID_ARG;
-  int kmode = 0;
+  const int base = mode & ~FP8BLK_E5M2;
+  if (base != FP8BLK_ROWWISE && base != FP8BLK_COLWISE_T && base != FP8BLK_BOTH) return FP8BLK_ERR_INVALID_ARG;
+  int kmode = (mode & FP8BLK_E5M2) ? fp8blk::Q_E5M2 : 0;
   if (mode & FP8BLK_ROWWISE) {
     if (!q_row || !s_row) return FP8BLK_ERR_INVALID_ARG;
     if (!aligned16(q_row) || !aligned16(s_row)) return FP8BLK_ERR_ALIGN;
@@ -165,6 +166,8 @@ fp8blk_status fp8blk_quantize_weight_128x128_both(const void* w, int64_t n, int6
 
 fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uint8_t* a, const float* sa,
                           const uint8_t* b, const float* sb, void* d, int64_t ldd, void* stream) {
+  const int formats = layout & (FP8BLK_A_E5M2 | FP8BLK_B_E5M2);
+  layout &= ~(FP8BLK_A_E5M2 | FP8BLK_B_E5M2);
   if (layout != FP8BLK_FWD && layout != FP8BLK_DGRAD && layout != FP8BLK_WGRAD) return FP8BLK_ERR_INVALID_ARG;
   if (!a || !sa || !b || !sb || !d) return FP8BLK_ERR_INVALID_ARG;
   if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K)) return FP8BLK_ERR_SHAPE;
@@ -195,6 +198,8 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   g.pair = 0;   // pair tiles measured slower (cross-SM hand-offs per K-block); opt in with FP8BLK_GEMM_PAIR=1
   g.group_m = 0;
   g.pdl = pdl_enabled();
+  g.a_e5m2 = (formats & FP8BLK_A_E5M2) != 0;
+  g.b_e5m2 = (formats & FP8BLK_B_E5M2) != 0;
   if (const char* e = std::getenv("FP8BLK_GEMM_PAIR")) g.pair = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_GROUP_M")) g.group_m = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);

@@ -129,6 +129,7 @@ struct GemmParams {
   unsigned int* err;
   int inject_stall;
   int group_m;
+  uint32_t fmt_bits;      // operand formats for the instruction descriptor (A: bits 7-9, B: bits 10-12; 1 = E5M2)
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -396,7 +397,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      const uint32_t idesc = idesc_e4m3_f32(BM, BN) | p.fmt_bits;
       int stage = 0;
       uint32_t phase = 0, abuf = 0, aphase = 0;
       bool ok = true;
@@ -682,7 +683,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader CTA only)
     if (leader && lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(2 * BM, BN);
+      const uint32_t idesc = idesc_e4m3_f32(2 * BM, BN) | p.fmt_bits;
       int stage = 0;
       uint32_t phase = 0, abuf = 0, aphase = 0;
       bool ok = true;
@@ -839,6 +840,11 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, in
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Instruction-descriptor bits of the operand formats (kind::f8f6f4: E4M3 = 0, E5M2 = 1).
+uint32_t fmt_bits(const GemmArgs& g) {
+  return (static_cast<uint32_t>(g.a_e5m2 != 0) << 7) | (static_cast<uint32_t>(g.b_e5m2 != 0) << 10);
+}
+
 int num_sms() {
   static int sms = 0;
   if (!sms) {
@@ -865,7 +871,7 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   const int num_mb = static_cast<int>(g.M / BM);
   int group_m = g.group_m > 0 ? g.group_m : 8;
   if (group_m > num_mb) group_m = num_mb;
-  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, group_m};
+  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, group_m, fmt_bits(g)};
   const int64_t tiles = (g.M / BM) * (g.N / BN);
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
   cudaLaunchConfig_t cfg = {};
@@ -893,7 +899,7 @@ cudaError_t launch_pair(const GemmArgs& g, cudaStream_t stream) {
   }
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BM)) return cudaErrorInvalidValue;
-  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, 0};
+  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, 0, fmt_bits(g)};
   const int64_t tiles = (g.M / (2 * BM)) * (g.N / kPairBN);
   const int64_t max_pairs = num_sms() / 2;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);

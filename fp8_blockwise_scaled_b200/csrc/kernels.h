@@ -8,7 +8,8 @@
 namespace fp8blk {
 
 // Which outputs a quantiser launch writes (may be OR-ed: ROW|COLT, BLK|BLKT).
-enum QuantMode : int { Q_ROW = 1, Q_COLT = 2, Q_BLK = 4, Q_BLKT = 8 };
+// Q_E5M2 selects E5M2 codes (gradients) for the activation modes.
+enum QuantMode : int { Q_ROW = 1, Q_COLT = 2, Q_BLK = 4, Q_BLKT = 8, Q_E5M2 = 16 };
 
 struct QuantArgs {
   const uint16_t* x;  // [rows][ldx] bf16
@@ -42,6 +43,7 @@ struct GemmArgs {
   int pair;                   // 1 = use 256 x 256 pair tiles when the shape allows, 0 = never
   int group_m;                // tile order: M-blocks per group (0 = default)
   int pdl;                    // 1 = launch with programmatic stream serialization
+  int a_e5m2, b_e5m2;         // 1 = that operand holds E5M2 codes (else E4M3)
   unsigned int* err;          // device error word
 };
 

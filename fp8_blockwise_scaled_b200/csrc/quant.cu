@@ -83,32 +83,51 @@ struct QScale {
   float nr;   // -RN(1/s)
 };
 
+// kE5: E5M2 codes, scale amax / 57344 = (amax * 2^-13) / 7; otherwise E4M3,
+// amax / 448 = (amax * 2^-6) / 7.  The same FMA-corrected division by 7 is
+// correctly rounded for every bfloat16 amax in both cases (checked exhaustively).
+template <bool kE5>
 __device__ __forceinline__ QScale make_qscale(float amax) {
   const float c7 = 0x1.24924ap-3f;  // fl32(1/7)
-  const float y = amax * 0.015625f;
+  const float y = amax * (kE5 ? 0x1p-13f : 0x1p-6f);
   const float q0 = y * c7;
   const float r = fmaf(-7.0f, q0, y);
   const float s = fmaxf(fmaf(r, c7, q0), 1e-12f);
   return {s, -__frcp_rn(s)};
 }
 
-// Four values -> four E4M3 codes packed little-endian (x0 in the lowest byte):
-// two paired conversions (the second source goes to the low byte) and one move.
+// Four values -> four codes packed little-endian (x0 in the lowest byte): two
+// paired conversions (the second source goes to the low byte) and one move.
+// Saturating conversion equals the pages' clamp-then-cast for both formats:
+// every value above the format's maximum rounds or saturates to it.
+template <bool kE5>
 __device__ __forceinline__ uint32_t cvt4(float x0, float x1, float x2, float x3) {
   uint32_t r;
-  asm("{\n\t.reg .b16 l, h;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 l, %2, %1;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 h, %4, %3;\n\t"
-      "mov.b32 %0, {l, h};\n\t}"
-      : "=r"(r)
-      : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
+  if constexpr (kE5)
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "cvt.rn.satfinite.e5m2x2.f32 l, %2, %1;\n\t"
+        "cvt.rn.satfinite.e5m2x2.f32 h, %4, %3;\n\t"
+        "mov.b32 %0, {l, h};\n\t}"
+        : "=r"(r)
+        : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
+  else
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 l, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h, %4, %3;\n\t"
+        "mov.b32 %0, {l, h};\n\t}"
+        : "=r"(r)
+        : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
   return r;
 }
 
-// Two values -> two E4M3 codes in the low 16 bits (x0 in the low byte).
+// Two values -> two codes in the low 16 bits (x0 in the low byte).
+template <bool kE5>
 __device__ __forceinline__ uint32_t cvt2(float x0, float x1) {
   uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(x0), "f"(x1));
+  if constexpr (kE5)
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %2, %1;" : "=h"(r) : "f"(x0), "f"(x1));
+  else
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(x0), "f"(x1));
   return r;
 }
 
@@ -124,11 +143,13 @@ __device__ __forceinline__ void neg_quotient2(float& w0, float& w1, float x0, fl
 }
 
 // Eight values -> eight codes packed little-endian (x[0] in the lowest byte).
+template <bool kE5>
 __device__ __forceinline__ uint2 quant8(const float (&x)[8], const QScale& q) {
   float w[8];
 #pragma unroll
   for (int j = 0; j < 8; j += 2) neg_quotient2(w[j], w[j + 1], x[j], x[j + 1], q.s, q.nr);
-  return make_uint2(cvt4(w[0], w[1], w[2], w[3]) ^ 0x80808080u, cvt4(w[4], w[5], w[6], w[7]) ^ 0x80808080u);
+  return make_uint2(cvt4<kE5>(w[0], w[1], w[2], w[3]) ^ 0x80808080u,
+                    cvt4<kE5>(w[4], w[5], w[6], w[7]) ^ 0x80808080u);
 }
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
@@ -177,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
   constexpr bool kBlkT = MODE & Q_BLKT;
   constexpr bool kTileSmem = kColT || kBlkT;
   constexpr bool kBlockScale = kBlk || kBlkT;
+  constexpr bool kE5 = MODE & Q_E5M2;        // E5M2 codes (activation modes only)
   constexpr int S = stages_for<MODE>();
 
   extern __shared__ uint8_t smem_raw[];
@@ -294,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
       k = __vmaxu2(k, __shfl_xor_sync(0xFFFFFFFFu, k, 2));
       k = __vmaxu2(k, __shfl_xor_sync(0xFFFFFFFFu, k, 1));
       const int rho = (lane >> 1) & 7;             // = 4 b + 2 c + d
-      const QScale q = make_qscale(__uint_as_float(d ? (k & 0xFFFF0000u) : (k << 16)));
+      const QScale q = make_qscale<kE5>(__uint_as_float(d ? (k & 0xFFFF0000u) : (k << 16)));
       if ((lane & 1) == 0) {
         rq[rho] = make_float2(q.s, q.nr);
         a.s_row[tc * a.rows + row0 + 8 * bi + rho] = q.s;
@@ -313,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
       float amax = wm[0];
 #pragma unroll
       for (int w = 1; w < kConsumers / 32; ++w) amax = fmaxf(amax, wm[w]);
-      qblk = make_qscale(amax);
+      qblk = make_qscale<kE5>(amax);
       if (t == 0) {
         if constexpr (kBlk) a.s_row[tr * a.tiles_c + tc] = qblk.s;
         if constexpr (kBlkT) a.s_t[tc * a.tiles_r + tr] = qblk.s;
@@ -330,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
         uint32_t mx = 0;
 #pragma unroll
         for (int w = 0; w < 8; ++w) mx = __vmaxu2(mx, ctrl->cpart[w * 64 + (t >> 1)]);
-        const QScale q = make_qscale(__uint_as_float((t & 1) ? (mx & 0xFFFF0000u) : (mx << 16)));
+        const QScale q = make_qscale<kE5>(__uint_as_float((t & 1) ? (mx & 0xFFFF0000u) : (mx << 16)));
         ctrl->qs[t] = make_float2(q.s, q.nr);
         a.s_t[tr * a.cols + col0 + t] = q.s;
       }
@@ -361,8 +383,8 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
           q0 = QScale{f.x, f.y};
           q1 = QScale{f.z, f.w};
         }
-        *reinterpret_cast<uint2*>(qdst + (2 * p) * cols) = quant8(f0, q0);
-        *reinterpret_cast<uint2*>(qdst + (2 * p + 1) * cols) = quant8(f1, q1);
+        *reinterpret_cast<uint2*>(qdst + (2 * p) * cols) = quant8<kE5>(f0, q0);
+        *reinterpret_cast<uint2*>(qdst + (2 * p + 1) * cols) = quant8<kE5>(f1, q1);
       }
       if constexpr (kTileSmem) {
 #pragma unroll
@@ -370,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
           const QScale q = kColT ? cq[c] : qblk;
           float w0, w1;
           neg_quotient2(w0, w1, f0[c], f1[c], q.s, q.nr);
-          const uint32_t h = cvt2(w0, w1);
+          const uint32_t h = cvt2<kE5>(w0, w1);
           if (p & 1) {
             const uint32_t word = __byte_perm(pend[c], h, 0x5410) ^ 0x80808080u;
             *reinterpret_cast<uint32_t*>(cs + (8 * bj + c) * 128 + ((bi ^ bj) * 8) + (p >> 1) * 4) = word;
@@ -464,6 +486,9 @@ cudaError_t launch_quant(int mode, const QuantArgs& a, cudaStream_t stream) {
     case Q_BLK: return launch_mode<Q_BLK>(a, stream);
     case Q_BLKT: return launch_mode<Q_BLKT>(a, stream);
     case Q_BLK | Q_BLKT: return launch_mode<Q_BLK | Q_BLKT>(a, stream);
+    case Q_ROW | Q_E5M2: return launch_mode<Q_ROW | Q_E5M2>(a, stream);
+    case Q_COLT | Q_E5M2: return launch_mode<Q_COLT | Q_E5M2>(a, stream);
+    case Q_ROW | Q_COLT | Q_E5M2: return launch_mode<Q_ROW | Q_COLT | Q_E5M2>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -61,7 +61,8 @@ typedef enum {
 typedef enum {
   FP8BLK_ROWWISE = 1,   /* 1x128 groups along the contiguous (feature) dimension */
   FP8BLK_COLWISE_T = 2, /* 1x128 groups along rows (tokens); codes written transposed */
-  FP8BLK_BOTH = 3       /* both of the above from one read of the input */
+  FP8BLK_BOTH = 3,      /* both of the above from one read of the input */
+  FP8BLK_E5M2 = 4       /* OR-ed into a mode: E5M2 codes instead of E4M3 (gradients) */
 } fp8blk_act_mode;
 
 typedef enum {
@@ -70,12 +71,22 @@ typedef enum {
   FP8BLK_WGRAD = 2  /* B scales per row and K-block: sb[K/128][N] */
 } fp8blk_layout;
 
+/* OR-ed into a layout: operand A (or B) holds E5M2 codes instead of E4M3. */
+typedef enum {
+  FP8BLK_A_E5M2 = 8,
+  FP8BLK_B_E5M2 = 16
+} fp8blk_operand_format;
+
 /*
  * Activation quantisation, 1x128 groups ([DIGEST] "激活 1D 128"; scale and
  * cast rule from [EXPL] "核心挑战：Scale Factor 管理").
  *
  *   x      [rows][ldx] bf16, the first `cols` columns of each row are used.
- *   mode   FP8BLK_ROWWISE, FP8BLK_COLWISE_T or FP8BLK_BOTH.
+ *   mode   FP8BLK_ROWWISE, FP8BLK_COLWISE_T or FP8BLK_BOTH, optionally OR-ed
+ *          with FP8BLK_E5M2: E5M2 codes ([EXPL] "Blackwell 的 FP8 Tensor
+ *          Core": 5 exponent bits, 2 mantissa bits, max 57344, the format for
+ *          gradients) with scale = max(fl32(amax / 57344), fl32(1e-12)) and the
+ *          value clamped to +-57344 before the cast; otherwise E4M3 as below.
  *   ROWWISE outputs (required for ROWWISE and BOTH, else ignored):
  *     q_row  [rows][cols] E4M3 codes, group = 128 consecutive columns of a row
  *     s_row  [cols/128][rows] fp32, s_row[g][r] = scale of row r, group g
@@ -129,6 +140,8 @@ fp8blk_status fp8blk_quantize_weight_128x128_both(const void* w, int64_t n, int6
  *
  *   a   [M][K] E4M3 codes (K contiguous),  sa [K/128][M] fp32 (per row, per K-block)
  *   b   [N][K] E4M3 codes (K contiguous)
+ *   layout may be OR-ed with FP8BLK_A_E5M2 and/or FP8BLK_B_E5M2 when that
+ *   operand holds E5M2 codes (E5M2 gradients: DGRAD and WGRAD take dY as A).
  *   sb  FWD / DGRAD: [N/128][K/128] fp32 (per 128x128 block)
  *       WGRAD      : [K/128][N] fp32     (per row of b, per K-block)
  *   d   [M][ldd] bf16 output, ldd >= N, ldd % 8 == 0.

@@ -61,7 +61,10 @@ S = NULL                  # stream
     ((ALIGNED, 128, 128, 64, 1, ALIGNED, ALIGNED, NULL, NULL, S), 1),       # ldx < cols
     ((ALIGNED, 128, 128, 132, 1, ALIGNED, ALIGNED, NULL, NULL, S), 3),      # row stride not 16-B
     ((MISALIGNED, 128, 128, 128, 1, ALIGNED, ALIGNED, NULL, NULL, S), 3),   # input pointer
-    ((ALIGNED, 128, 128, 128, 4, ALIGNED, ALIGNED, NULL, NULL, S), 1),      # bad mode
+    ((ALIGNED, 128, 128, 128, 4, ALIGNED, ALIGNED, NULL, NULL, S), 1),      # E5M2 flag without a layout
+    ((ALIGNED, 128, 128, 128, 8, ALIGNED, ALIGNED, NULL, NULL, S), 1),      # unknown flag
+    ((ALIGNED, 128, 128, 128, 1 | 4, NULL, ALIGNED, NULL, NULL, S), 1),     # E5M2 row-wise, missing q_row
+    ((ALIGNED, 128, 128, 128, 3 | 4, ALIGNED, ALIGNED, MISALIGNED, ALIGNED, S), 3),
     ((ALIGNED, 128, 128, 128, 1, NULL, ALIGNED, NULL, NULL, S), 1),         # missing q_row
     ((ALIGNED, 128, 128, 128, 2, ALIGNED, ALIGNED, NULL, NULL, S), 1),      # missing q_colT
     ((ALIGNED, 128, 128, 128, 3, ALIGNED, ALIGNED, MISALIGNED, ALIGNED, S), 3),
@@ -94,6 +97,9 @@ def test_quantize_weight_both_argument_errors():
 
 @pytest.mark.parametrize("args,code", [
     ((3, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 1),   # bad layout
+    ((3 | 8, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 1),   # bad layout, E5M2 A
+    ((1 | 32, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 1),  # unknown flag
+    ((2 | 8, 100, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 2),   # E5M2 A, bad shape
     ((0, 100, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 2),
     ((0, 128, 128, 96, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 2),
     ((0, 128, 128, 128, NULL, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 1),
