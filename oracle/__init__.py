@@ -70,6 +70,12 @@ def _load():
         lib.orc_quantize_act_rowwise_fmt.argtypes = [P, I64, I64, ctypes.c_int, P, P]
         lib.orc_quantize_act_colwise_t_fmt.argtypes = [P, I64, I64, ctypes.c_int, P, P]
         lib.orc_gemm_fmt.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, I64, I64, I64, P, P, P, P, P, I64, P]
+        lib.orc_amax_ema.argtypes = [P, I64, I64, ctypes.c_float, ctypes.c_double]
+        lib.orc_amax_ema.restype = ctypes.c_float
+        lib.orc_tensor_scale.argtypes = [ctypes.c_float]
+        lib.orc_tensor_scale.restype = ctypes.c_float
+        lib.orc_quantize_tensor.argtypes = [P, I64, I64, ctypes.c_float, P]
+        lib.orc_gemm_tensor.argtypes = [I64, I64, I64, P, ctypes.c_float, P, ctypes.c_float, P, I64, P]
         _lib = lib
     return _lib
 
@@ -190,4 +196,47 @@ def gemm(layout: int, qa, sa, qb, sb, rows=None, a_fmt: int = E4M3, b_fmt: int =
     d = np.empty((nrows, n), np.float64)
     _load().orc_gemm_fmt(layout, int(a_fmt), int(b_fmt), m, n, k, _ptr(qa), _ptr(sa), _ptr(qb), _ptr(sb), rp,
                          nrows, _ptr(d))
+    return d
+
+
+# ---------------------------------------------------------------- per-tensor delayed scaling
+EMA_BETA = 0.99
+
+
+def amax_ema(x, amax: float, beta: float = EMA_BETA) -> np.float32:
+    """Updated amax buffer: RN(RN(amax * RN32(beta)) + RN(max|x| * RN32(1 - beta)))."""
+    x = _c(x, np.uint16)
+    r, c = x.shape
+    return np.float32(_load().orc_amax_ema(_ptr(x), r, c, float(np.float32(amax)), float(beta)))
+
+
+def tensor_scale(amax: float) -> np.float32:
+    return np.float32(_load().orc_tensor_scale(float(np.float32(amax))))
+
+
+def quantize_tensor(x, scale: float) -> np.ndarray:
+    """The whole tensor with one scale: E4M3(clamp(x / scale, -448, 448))."""
+    x = _c(x, np.uint16)
+    r, c = x.shape
+    q = np.empty((r, c), np.uint8)
+    _load().orc_quantize_tensor(_ptr(x), r, c, float(np.float32(scale)), _ptr(q))
+    return q
+
+
+def gemm_tensor(qa, sa: float, qb, sb: float, rows=None) -> np.ndarray:
+    """D = (qa * sa) . (qb * sb)^T in fp64 over dequantised E4M3 operands (both K-major)."""
+    qa = _c(qa, np.uint8)
+    qb = _c(qb, np.uint8)
+    m, k = qa.shape
+    n, k2 = qb.shape
+    if k != k2:
+        raise ValueError("A and B disagree on K")
+    if rows is None:
+        rows_arr, nrows, rp = None, m, None
+    else:
+        rows_arr = _c(rows, np.int64)
+        nrows, rp = rows_arr.size, _ptr(rows_arr)
+    d = np.empty((nrows, n), np.float64)
+    _load().orc_gemm_tensor(m, n, k, _ptr(qa), float(np.float32(sa)), _ptr(qb), float(np.float32(sb)), rp, nrows,
+                            _ptr(d))
     return d

@@ -355,4 +355,66 @@ void orc_gemm(int layout, int64_t M, int64_t N, int64_t K, const uint8_t* qa, co
   orc_gemm_fmt(layout, 0, 0, M, N, K, qa, sa, qb, sb, rows, nrows, d);
 }
 
+// ---------------------------------------------------------------- per-tensor delayed scaling
+// [EXPL] "核心挑战：Scale Factor 管理", FP8Linear (the pages' "delayed scaling"
+// recipe): each tensor keeps an amax buffer, initialised to 1 and updated by
+// an exponential moving average with beta = 0.99 from the tensor's current
+// max |x| before it is quantised; the whole tensor then shares one scale,
+// max(amax / 448, 1e-12), and is quantised as above (divide, clamp to +-448,
+// cast to E4M3).  The forward product is the matmul of the dequantised
+// operands.  The EMA is evaluated in binary32 as written there:
+//   amax <- RN(RN(amax * b) + RN(cur * c)),  b = RN32(0.99), c = RN32(1 - 0.99)  (reading R16)
+
+// cur = max |x| over the whole [rows][cols] bf16 tensor (exact); returns the
+// updated amax.  beta is the decimal constant (0.99) as a double; the binary32
+// operands are RN32(beta) and RN32(1 - beta), as when the page's Python
+// constants meet its binary32 buffers.
+float orc_amax_ema(const uint16_t* x, int64_t rows, int64_t cols, float amax, double beta) {
+  std::vector<float> part(static_cast<size_t>(rows), 0.0f);
+  parallel_for(rows, [&](int64_t r) {
+    float m = 0.0f;
+    for (int64_t c = 0; c < cols; ++c) m = std::max(m, std::fabs(bf16_to_float(x[r * cols + c])));
+    part[r] = m;
+  });
+  float cur = 0.0f;
+  for (float m : part) cur = std::max(cur, m);
+  const float b = static_cast<float>(beta);
+  const float c = static_cast<float>(1.0 - beta);
+  const float keep = amax * b;                                   // binary32 products and sum
+  const float add = cur * c;
+  return keep + add;
+}
+
+// One scale for the whole tensor: max(amax / 448, 1e-12) (binary32 division).
+float orc_tensor_scale(float amax) { return group_scale(amax, 0); }
+
+// Quantise the whole [rows][cols] bf16 tensor with the single scale s.
+void orc_quantize_tensor(const uint16_t* x, int64_t rows, int64_t cols, float s, uint8_t* q) {
+  parallel_for(rows, [&](int64_t r) {
+    for (int64_t c = 0; c < cols; ++c) q[r * cols + c] = quantize_value(bf16_to_float(x[r * cols + c]), s, 0);
+  });
+}
+
+// D[m][n] = sum_k (qa[m][k] * sa) * (qb[n][k] * sb) in fp64 over the dequantised
+// operands (both K-major E4M3), rows as in orc_gemm.
+void orc_gemm_tensor(int64_t M, int64_t N, int64_t K, const uint8_t* qa, float sa, const uint8_t* qb, float sb,
+                     const int64_t* rows, int64_t nrows, double* d) {
+  if (!rows) nrows = M;
+  std::vector<double> bdq(static_cast<size_t>(N) * K);
+  parallel_for(N, [&](int64_t n) {
+    for (int64_t k = 0; k < K; ++k) bdq[n * K + k] = e4m3_decode(qb[n * K + k]) * static_cast<double>(sb);
+  });
+  parallel_for(nrows, [&](int64_t i) {
+    const int64_t m = rows ? rows[i] : i;
+    std::vector<double> adq(K);
+    for (int64_t k = 0; k < K; ++k) adq[k] = e4m3_decode(qa[m * K + k]) * static_cast<double>(sa);
+    for (int64_t n = 0; n < N; ++n) {
+      const double* bn = &bdq[n * K];
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += adq[k] * bn[k];
+      d[i * N + n] = acc;
+    }
+  });
+}
+
 }  // extern "C"
