@@ -93,7 +93,7 @@ def workload_tensors(name: str, tokens: int) -> list[dict]:
 class Program:
     """Device buffers and the ordered kernel launches of one step."""
 
-    def __init__(self, specs, device, world, grad_e5m2=False):
+    def __init__(self, specs, device, world, grad_e5m2=False, recipe="blockwise"):
         import torch
         import fp8_blockwise_scaled_b200 as fb
         self.fb, self.torch, self.world = fb, torch, world
@@ -103,6 +103,9 @@ class Program:
         self.grads = []        # weight gradients all-reduced across ranks
         self.gemm_flops = 0
         E4 = torch.float8_e4m3fn
+        if recipe == "delayed":
+            self._build_delayed(specs, device)
+            specs = []
         for sp in specs:
             x = self._dev(sp["X"], device)
             w = self._dev(sp["W"], device)
@@ -166,6 +169,32 @@ class Program:
                     self.grads.append(dw)
         self.gemm_flops = sum(u for _, k, u, _ in self.ops if k == "gemm")
         self.quant_bytes = sum(u for _, k, u, _ in self.ops if k == "quant")
+
+    def _build_delayed(self, specs, device):
+        """The pages' per-tensor delayed-scaling FP8Linear forward for every linear: amax EMA of X and
+        of W (buffers persist across steps), both tensors quantised with their one scale, one GEMM."""
+        torch, fb = self.torch, self.fb
+        for sp in specs:
+            x, w = self._dev(sp["X"], device), self._dev(sp["W"], device)
+            T, K = x.shape
+            N = w.shape[0]
+            g = sp["name"]
+            amax = {k: torch.ones(1, dtype=torch.float32, device=device) for k in "xw"}
+            scale = {k: torch.empty(1, dtype=torch.float32, device=device) for k in "xw"}
+            ws = {k: torch.empty(max(16, fb.fp8blk_amax_ema_workspace_bytes(r)), dtype=torch.uint8, device=device)
+                  for k, r in (("x", T), ("w", N))}
+            qx = torch.empty(T, K, dtype=torch.float8_e4m3fn, device=device)
+            qw = torch.empty(N, K, dtype=torch.float8_e4m3fn, device=device)
+            y = torch.empty(T, N, dtype=torch.bfloat16, device=device)
+            self._op(f"{g}.amax_x", "quant", T * K * 2,
+                     lambda x=x, a=amax["x"], s=scale["x"], w=ws["x"]: fb.fp8blk_amax_ema(x, a, s, w))
+            self._op(f"{g}.amax_w", "quant", N * K * 2,
+                     lambda x=w, a=amax["w"], s=scale["w"], w=ws["w"]: fb.fp8blk_amax_ema(x, a, s, w))
+            self._op(f"{g}.quant_x", "quant", T * K * 3, lambda x=x, s=scale["x"], q=qx: fb.fp8blk_quantize_tensor(x, s, q))
+            self._op(f"{g}.quant_w", "quant", N * K * 3, lambda x=w, s=scale["w"], q=qw: fb.fp8blk_quantize_tensor(x, s, q))
+            self._op(f"{g}.gemm_fwd", "gemm", 2 * T * N * K,
+                     lambda a=qx, sa=scale["x"], b=qw, sb=scale["w"], d=y: fb.fp8blk_gemm_tensor_scaled(a, sa, b, sb, d))
+            self.outputs.append(y)
 
     def _dev(self, host, device):
         t = self.torch.from_numpy(np.ascontiguousarray(host)).view(self.torch.bfloat16).to(device)
@@ -357,7 +386,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     tokens = args.tokens or (16384 if args.workload == "layer" else 8192)
     specs = workload_tensors(args.workload, tokens)
-    prog = Program(specs, dev, world, grad_e5m2=args.grad_format == "e5m2")
+    prog = Program(specs, dev, world, grad_e5m2=args.grad_format == "e5m2", recipe=args.recipe)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -480,6 +509,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "l2": "flushed between steps (256 MiB write outside the timed events)",
                    "streams": 1, "seed": {"layer": 4, "qkv_fwd": 1, "mlp_fwd": 2, "down_bwd": 3}[args.workload],
                    "grad_format": args.grad_format,
+                   "recipe": args.recipe if args.recipe == "blockwise" else
+                             "delayed: per-tensor scales from an amax EMA, forward GEMMs only",
                    "launch": ("eager" if graph is None else "one CUDA graph per step")
                              + (", programmatic dependent launch" if os.environ.get("FP8BLK_PDL") == "1" else ""),
                    "parallelism": f"dp{world}" if world > 1 else "single-gpu"},
@@ -556,6 +587,9 @@ def main(argv=None):
     ap.add_argument("--sweep", action="store_true", help="token sweep of the layer GEMMs (one JSON line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of the step's CUDA graph")
+    ap.add_argument("--recipe", choices=["blockwise", "delayed"], default="blockwise",
+                    help="blockwise 1x128 / 128x128 scaling (fwd+dgrad+wgrad), or the per-tensor delayed-scaling "
+                         "forward")
     ap.add_argument("--grad-format", choices=["e4m3", "e5m2"], default="e4m3",
                     help="code format of the output gradient dY (the DGRAD/WGRAD A operand)")
     args = ap.parse_args(argv)

@@ -31,7 +31,8 @@ from ._lib import (A_E5M2, B_E5M2, BOTH, COLWISE_T, DGRAD, E5M2, FWD, ROWWISE, W
 
 __all__ = [
     "fp8blk_quantize_act_1x128", "fp8blk_quantize_weight_128x128", "fp8blk_quantize_weight_128x128_t",
-    "fp8blk_quantize_weight_128x128_both",
+    "fp8blk_quantize_weight_128x128_both", "fp8blk_amax_ema", "fp8blk_amax_ema_workspace_bytes",
+    "fp8blk_quantize_tensor", "fp8blk_gemm_tensor_scaled", "fp8_linear_delayed_forward",
     "fp8blk_gemm", "fp8blk_get_device_error", "fp8blk_version", "linear_forward", "linear_backward",
     "ROWWISE", "COLWISE_T", "BOTH", "E5M2", "FWD", "DGRAD", "WGRAD", "A_E5M2", "B_E5M2", "Fp8BlkError",
     "LIB_PATH", "status_string",
@@ -154,6 +155,61 @@ def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None):
     check(lib.fp8blk_gemm(int(layout) | flags, m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d), d.stride(0),
                           _stream_handle(stream)))
     return d
+
+
+def fp8blk_amax_ema_workspace_bytes(rows: int) -> int:
+    return int(lib.fp8blk_amax_ema_workspace_bytes(int(rows)))
+
+
+def fp8blk_amax_ema(x, amax, scale=None, workspace=None, stream=None):
+    """Per-tensor delayed scaling: update the amax buffer (float32 [1], in place) from max|x| by the
+    EMA and write the tensor's scale.  Returns (amax, scale)."""
+    x = _bf16_2d(x)
+    _need_cuda(x, amax)
+    rows, cols = x.shape
+    if amax.dtype != torch.float32 or amax.numel() != 1:
+        raise ValueError("amax must be a float32 tensor with one element")
+    scale = _out(scale, (1,), torch.float32, x.device)
+    need = fp8blk_amax_ema_workspace_bytes(rows)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    check(lib.fp8blk_amax_ema(_ptr(x), rows, cols, x.stride(0), _ptr(amax), _ptr(scale), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream_handle(stream)))
+    return amax, scale
+
+
+def fp8blk_quantize_tensor(x, scale, q=None, stream=None):
+    """The whole tensor with its one scale (device float32 [1]).  Returns q [rows, cols] E4M3."""
+    x = _bf16_2d(x)
+    _need_cuda(x, scale)
+    rows, cols = x.shape
+    q = _out(q, (rows, cols), E4M3, x.device)
+    check(lib.fp8blk_quantize_tensor(_ptr(x), rows, cols, x.stride(0), _ptr(scale), _ptr(q), _stream_handle(stream)))
+    return q
+
+
+def fp8blk_gemm_tensor_scaled(a, sa, b, sb, d=None, stream=None):
+    """D[M,N] = bf16(sa * sb * A . B^T) with one scale per E4M3 operand (device float32 [1] each)."""
+    _need_cuda(a, sa, b, sb, d)
+    m, k = a.shape
+    n = b.shape[0]
+    if b.shape[1] != k or a.dtype != E4M3 or b.dtype != E4M3:
+        raise ValueError("A [M,K] and B [N,K] must be float8_e4m3fn")
+    if d is None:
+        d = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
+    check(lib.fp8blk_gemm_tensor_scaled(m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d), d.stride(0),
+                                        _stream_handle(stream)))
+    return d
+
+
+def fp8_linear_delayed_forward(x, w, x_amax, w_amax, stream=None):
+    """Y = X . W^T with per-tensor delayed scaling: both amax buffers updated by the EMA, both
+    tensors quantised with their one scale, one GEMM.  Returns Y (bf16)."""
+    _, sx = fp8blk_amax_ema(x, x_amax, stream=stream)
+    _, sw = fp8blk_amax_ema(w, w_amax, stream=stream)
+    qx = fp8blk_quantize_tensor(x, sx, stream=stream)
+    qw = fp8blk_quantize_tensor(w, sw, stream=stream)
+    return fp8blk_gemm_tensor_scaled(qx, sx, qw, sw, stream=stream)
 
 
 def fp8blk_get_device_error(stream=None) -> int:

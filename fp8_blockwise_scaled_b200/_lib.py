@@ -40,6 +40,10 @@ def _load() -> ctypes.CDLL:
         "fp8blk_quantize_weight_128x128": [P, I64, I64, I64, P, P, P],
         "fp8blk_quantize_weight_128x128_t": [P, I64, I64, I64, P, P, P],
         "fp8blk_quantize_weight_128x128_both": [P, I64, I64, I64, P, P, P, P, P],
+        "fp8blk_amax_ema": [P, I64, I64, I64, P, P, P, I64, P],
+        "fp8blk_amax_ema_workspace_bytes": [I64],
+        "fp8blk_quantize_tensor": [P, I64, I64, I64, P, P, P],
+        "fp8blk_gemm_tensor_scaled": [I64, I64, I64, P, P, P, P, P, I64, P],
         "fp8blk_gemm": [I, I64, I64, I64, P, P, P, P, P, I64, P],
         "fp8blk_get_device_error": [P],
         "fp8blk_status_string": [I],
@@ -48,7 +52,8 @@ def _load() -> ctypes.CDLL:
     for name, args in sigs.items():
         fn = getattr(so, name)
         fn.argtypes = args
-        fn.restype = ctypes.c_char_p if name == "fp8blk_status_string" else ctypes.c_int
+        fn.restype = {"fp8blk_status_string": ctypes.c_char_p,
+                      "fp8blk_amax_ema_workspace_bytes": ctypes.c_int64}.get(name, ctypes.c_int)
     return so
 
 

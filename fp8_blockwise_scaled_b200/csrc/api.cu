@@ -174,7 +174,9 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   // One CTA row/column of tiles is addressed with 32-bit TMA coordinates.
   if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return FP8BLK_ERR_SHAPE;
   if (ldd < N) return FP8BLK_ERR_INVALID_ARG;
-  if (!aligned16(a) || !aligned16(b) || !aligned16(d) || ldd % 8 != 0) return FP8BLK_ERR_ALIGN;
+  // The epilogue writes 32-byte vectors: d and every output row start on a 32-byte boundary.
+  if (!aligned16(a) || !aligned16(b) || (reinterpret_cast<uintptr_t>(d) & 31u) || ldd % 16 != 0)
+    return FP8BLK_ERR_ALIGN;
   if (!aligned16(sa) || !aligned16(sb)) return FP8BLK_ERR_ALIGN;
   fp8blk_status st = check_device();
   if (st != FP8BLK_OK) return st;
@@ -204,6 +206,69 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   if (const char* e = std::getenv("FP8BLK_GEMM_GROUP_M")) g.group_m = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_TMEM_DB")) g.tmem_db = std::atoi(e);
+  if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) g.inject_stall = std::atoi(e) != 0;
+  return launch_status(fp8blk::launch_gemm(g, static_cast<cudaStream_t>(stream)));
+}
+
+int64_t fp8blk_amax_ema_workspace_bytes(int64_t rows) {
+  if (rows <= 0) return 0;
+  return ((rows + fp8blk::kTensorRowsPerPartial - 1) / fp8blk::kTensorRowsPerPartial) * 4;
+}
+
+fp8blk_status fp8blk_amax_ema(const void* x, int64_t rows, int64_t cols, int64_t ldx, float* amax, float* scale,
+                              void* workspace, int64_t workspace_bytes, void* stream) {
+  fp8blk_status st = check_quant_common(x, rows, cols, ldx);
+  if (st != FP8BLK_OK) return st;
+  if (!amax || !scale || !workspace) return FP8BLK_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(amax) & 3u) || (reinterpret_cast<uintptr_t>(scale) & 3u) || !aligned16(workspace))
+    return FP8BLK_ERR_ALIGN;
+  if (workspace_bytes < fp8blk_amax_ema_workspace_bytes(rows)) return FP8BLK_ERR_INVALID_ARG;
+  if ((st = check_device()) != FP8BLK_OK) return st;
+  fp8blk::TensorArgs t{static_cast<const uint16_t*>(x), rows, cols, ldx, amax, scale, pdl_enabled()};
+  return launch_status(fp8blk::launch_amax_ema(t, static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream)));
+}
+
+fp8blk_status fp8blk_quantize_tensor(const void* x, int64_t rows, int64_t cols, int64_t ldx, const float* scale,
+                                     uint8_t* q, void* stream) {
+  fp8blk_status st = check_quant_common(x, rows, cols, ldx);
+  if (st != FP8BLK_OK) return st;
+  if (!scale || !q) return FP8BLK_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(scale) & 3u) || !aligned16(q)) return FP8BLK_ERR_ALIGN;
+  if ((st = check_device()) != FP8BLK_OK) return st;
+  fp8blk::TensorArgs t{static_cast<const uint16_t*>(x), rows, cols, ldx, nullptr, const_cast<float*>(scale),
+                       pdl_enabled()};
+  return launch_status(fp8blk::launch_quant_tensor(t, q, static_cast<cudaStream_t>(stream)));
+}
+
+fp8blk_status fp8blk_gemm_tensor_scaled(int64_t M, int64_t N, int64_t K, const uint8_t* a, const float* sa,
+                                        const uint8_t* b, const float* sb, void* d, int64_t ldd, void* stream) {
+  if (!a || !sa || !b || !sb || !d) return FP8BLK_ERR_INVALID_ARG;
+  if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K)) return FP8BLK_ERR_SHAPE;
+  if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return FP8BLK_ERR_SHAPE;
+  if (ldd < N) return FP8BLK_ERR_INVALID_ARG;
+  // The epilogue writes 32-byte vectors: d and every output row start on a 32-byte boundary.
+  if (!aligned16(a) || !aligned16(b) || (reinterpret_cast<uintptr_t>(d) & 31u) || ldd % 16 != 0)
+    return FP8BLK_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(sa) & 3u) || (reinterpret_cast<uintptr_t>(sb) & 3u)) return FP8BLK_ERR_ALIGN;
+  fp8blk_status st = check_device();
+  if (st != FP8BLK_OK) return st;
+  fp8blk::GemmArgs g{};
+  g.layout = 0;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.a = a;
+  g.b = b;
+  g.d = static_cast<uint16_t*>(d);
+  g.ldd = ldd;
+  g.timeout_ns = wait_timeout_ns();
+  g.err = error_word();
+  if (!g.err) return FP8BLK_ERR_CUDA;
+  g.tmem_db = -1;
+  g.pdl = pdl_enabled();
+  g.tensor_sa = sa;
+  g.tensor_sb = sb;
+  if (const char* e = std::getenv("FP8BLK_GEMM_GROUP_M")) g.group_m = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) g.inject_stall = std::atoi(e) != 0;
   return launch_status(fp8blk::launch_gemm(g, static_cast<cudaStream_t>(stream)));
 }

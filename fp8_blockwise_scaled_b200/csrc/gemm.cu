@@ -130,6 +130,8 @@ struct GemmParams {
   int inject_stall;
   int group_m;
   uint32_t fmt_bits;      // operand formats for the instruction descriptor (A: bits 7-9, B: bits 10-12; 1 = E5M2)
+  const float* tsa;       // per-tensor scales (kTensor variant), device scalars
+  const float* tsb;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -290,7 +292,10 @@ __device__ __forceinline__ void tile_coords(int tile, int num_mb, int num_nb, in
   nb = r / gm;
 }
 
-template <int BN, bool kWgrad, bool kSplit>
+// kTensor: one scale per operand (per-tensor scaling).  No per-K-block
+// promotion: the MMAs accumulate the whole K loop of a tile in TMEM and the
+// promotion warps only apply sa * sb, round to bf16 and store, once per tile.
+template <int BN, bool kWgrad, bool kSplit, bool kTensor = false>
 __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     gemm_blockwise_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const GemmParams p) {
@@ -386,7 +391,8 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     }
   } else if (warp == Layout<kSplit>::kScaleWarp) {
     // ------------------------------------------------------------ scale producer (whole warp)
-    scale_feed<BN, kWgrad>(ctrl, p, blockIdx.x, gridDim.x, tiles, kblocks,
+    if constexpr (!kTensor)
+      scale_feed<BN, kWgrad>(ctrl, p, blockIdx.x, gridDim.x, tiles, kblocks,
                            [&](int tile, int64_t& m0, int64_t& n0) {
                              int mb, nb;
                              tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
@@ -403,9 +409,15 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
       bool ok = true;
       if (p.inject_stall) ok = mbar_wait_bounded(&ctrl->never, 0, abort, p.timeout_ns, p.err);
       for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+        if constexpr (kTensor) {   // one accumulator buffer per tile
+          if (!mbar_wait_bounded(&ctrl->tempty[abuf], aphase ^ 1u, abort, p.timeout_ns, p.err)) {
+            ok = false;
+            break;
+          }
+        }
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait_bounded(&ctrl->full[stage], phase, abort, p.timeout_ns, p.err) ||
-              !mbar_wait_bounded(&ctrl->tempty[abuf], aphase ^ 1u, abort, p.timeout_ns, p.err)) {
+              (!kTensor && !mbar_wait_bounded(&ctrl->tempty[abuf], aphase ^ 1u, abort, p.timeout_ns, p.err))) {
             ok = false;
             break;
           }
@@ -416,13 +428,23 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
           const uint32_t d_tmem = tmem_base + abuf * BN;
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k)  // 32 E4M3 values = 32 bytes = 2 x 16 B per step
-            umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+            umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (k > 0 || (kTensor && kb > 0)) ? 1u : 0u);
           umma_commit(&ctrl->empty[stage]);
-          umma_commit(&ctrl->tfull[abuf]);
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
           }
+          if constexpr (!kTensor) {
+            umma_commit(&ctrl->tfull[abuf]);
+            if (++abuf == C::kAccBufs) {
+              abuf = 0;
+              aphase ^= 1u;
+            }
+          }
+        }
+        if constexpr (kTensor) {
+          if (!ok) break;
+          umma_commit(&ctrl->tfull[abuf]);   // the tile's whole K loop is in this buffer
           if (++abuf == C::kAccBufs) {
             abuf = 0;
             aphase ^= 1u;
@@ -444,8 +466,40 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     const int col0 = wg * C::kHalf;
     uint32_t abuf = 0, aphase = 0, sphase = 0;
     int slot = 0;
-    float2 acc[C::kHalf / 2];
     bool ok = true;
+    if constexpr (kTensor) {
+      // ---------------------------------------------------------- per-tensor epilogue
+      const float f = *p.tsa * *p.tsb;
+      for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&ctrl->tfull[abuf], aphase, abort, p.timeout_ns, p.err)))
+          break;
+        tc_fence_after_sync();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * BN + col0;
+        uint16_t* drow = p.d + (static_cast<int64_t>(mb) * BM + row) * p.ldd + static_cast<int64_t>(nb) * BN + col0;
+#pragma unroll
+        for (int c = 0; c < C::kHalf; c += 16) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(taddr + c, r);
+          tmem_wait_ld16(r);
+          uint32_t v[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            v[q] = pack_bf16x2(__uint_as_float(r[2 * q]) * f, __uint_as_float(r[2 * q + 1]) * f);
+          st_global_v8(drow + c, v);
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->tempty[abuf]);
+        if (++abuf == C::kAccBufs) {
+          abuf = 0;
+          aphase ^= 1u;
+        }
+      }
+      ok = false;   // skip the blockwise loop below
+    }
+    float2 acc[C::kHalf / 2];
     for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
       int mb, nb;
       tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
@@ -856,12 +910,12 @@ int num_sms() {
   return sms;
 }
 
-template <int BN, bool kWgrad, bool kSplit>
+template <int BN, bool kWgrad, bool kSplit, bool kTensor = false>
 cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   static bool attr_set = false;
   constexpr int kSmem = smem_bytes<BN>();
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_blockwise_kernel<BN, kWgrad, kSplit>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_blockwise_kernel<BN, kWgrad, kSplit, kTensor>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -871,7 +925,8 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   const int num_mb = static_cast<int>(g.M / BM);
   int group_m = g.group_m > 0 ? g.group_m : 8;
   if (group_m > num_mb) group_m = num_mb;
-  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, group_m, fmt_bits(g)};
+  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, group_m, fmt_bits(g),
+               g.tensor_sa, g.tensor_sb};
   const int64_t tiles = (g.M / BM) * (g.N / BN);
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
   cudaLaunchConfig_t cfg = {};
@@ -882,7 +937,7 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   cudaLaunchAttribute attr[1];
   cfg.numAttrs = set_pdl_attr(attr, g.pdl);
   cfg.attrs = attr;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<BN, kWgrad, kSplit>, ta, tb, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<BN, kWgrad, kSplit, kTensor>, ta, tb, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -899,7 +954,8 @@ cudaError_t launch_pair(const GemmArgs& g, cudaStream_t stream) {
   }
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BM)) return cudaErrorInvalidValue;
-  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, 0, fmt_bits(g)};
+  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, 0, fmt_bits(g), nullptr,
+               nullptr};
   const int64_t tiles = (g.M / (2 * BM)) * (g.N / kPairBN);
   const int64_t max_pairs = num_sms() / 2;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
@@ -947,6 +1003,11 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream) {
     }
   }
   if (bn == 256 && g.N % 256 != 0) return cudaErrorInvalidValue;
+  if (g.tensor_sa) {   // per-tensor scales: plain layout, no per-K-block promotion
+    if (g.layout != 0) return cudaErrorInvalidValue;
+    return bn == 256 ? launch_variant<256, false, false, true>(g, stream)
+                     : launch_variant<128, false, false, true>(g, stream);
+  }
   // The register split with double-buffered TMEM reads pays off where the
   // promotion does more work per column (WGRAD); measured on B200, the plain
   // layout is faster for the forward/data-gradient promotion.

@@ -27,6 +27,19 @@ struct QuantArgs {
 
 cudaError_t launch_quant(int mode, const QuantArgs& a, cudaStream_t stream);
 
+// Per-tensor delayed scaling (tensor.cu).
+constexpr int kTensorRowsPerPartial = 16;   // rows reduced by one CTA of the amax reduction
+struct TensorArgs {
+  const uint16_t* x;  // [rows][ldx] bf16
+  int64_t rows, cols, ldx;
+  float* amax;        // the tensor's amax buffer (in: previous value, out: after the EMA)
+  float* scale;       // out (amax_ema) or in (quantize): max(amax / 448, 1e-12)
+  int pdl;
+};
+// partials: ceil(rows / kTensorRowsPerPartial) words of scratch, fully rewritten.
+cudaError_t launch_amax_ema(const TensorArgs& t, uint32_t* partials, cudaStream_t stream);
+cudaError_t launch_quant_tensor(const TensorArgs& t, uint8_t* q, cudaStream_t stream);
+
 struct GemmArgs {
   int layout;                 // 0 FWD, 1 DGRAD, 2 WGRAD
   int64_t M, N, K;
@@ -44,6 +57,8 @@ struct GemmArgs {
   int group_m;                // tile order: M-blocks per group (0 = default)
   int pdl;                    // 1 = launch with programmatic stream serialization
   int a_e5m2, b_e5m2;         // 1 = that operand holds E5M2 codes (else E4M3)
+  const float* tensor_sa;     // non-null: one scale per operand (device scalars), no per-block scales
+  const float* tensor_sb;
   unsigned int* err;          // device error word
 };
 

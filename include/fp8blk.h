@@ -144,7 +144,7 @@ fp8blk_status fp8blk_quantize_weight_128x128_both(const void* w, int64_t n, int6
  *   operand holds E5M2 codes (E5M2 gradients: DGRAD and WGRAD take dY as A).
  *   sb  FWD / DGRAD: [N/128][K/128] fp32 (per 128x128 block)
  *       WGRAD      : [K/128][N] fp32     (per row of b, per K-block)
- *   d   [M][ldd] bf16 output, ldd >= N, ldd % 8 == 0.
+ *   d   [M][ldd] bf16 output, ldd >= N, ldd % 16 == 0, d 32-byte aligned.
  *
  * Operands per pass of a linear layer Y = X . W^T (X [T][in], W [out][in]):
  *   FWD   : a = X rowwise,      b = W (128x128),           d = Y  [T][out]
@@ -156,6 +156,45 @@ fp8blk_status fp8blk_quantize_weight_128x128_both(const void* w, int64_t n, int6
 fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K,
                           const uint8_t* a, const float* sa, const uint8_t* b, const float* sb,
                           void* d, int64_t ldd, void* stream);
+
+/*
+ * Per-tensor delayed scaling ([EXPL] "核心挑战：Scale Factor 管理", FP8Linear):
+ * one amax buffer per tensor (the caller initialises it to 1), updated from
+ * the tensor's current max |x| by an exponential moving average before the
+ * tensor is quantised with one scale.
+ *
+ * fp8blk_amax_ema: amax <- RN(RN(amax * RN32(0.99)) + RN(max|x| * RN32(1 - 0.99)))
+ *   (binary32), then scale <- max(amax / 448, 1e-12) (correctly rounded).
+ *   x          [rows][ldx] bf16, the first cols columns of each row are used.
+ *   amax       device float, read and written (the EMA state).
+ *   scale      device float, written.
+ *   workspace  device scratch of at least fp8blk_amax_ema_workspace_bytes(rows)
+ *              bytes (16-byte aligned), fully rewritten by every call, owned by
+ *              the caller; two calls may share it only if they are ordered on
+ *              one stream.  Too small: FP8BLK_ERR_INVALID_ARG.
+ */
+fp8blk_status fp8blk_amax_ema(const void* x, int64_t rows, int64_t cols, int64_t ldx, float* amax, float* scale,
+                              void* workspace, int64_t workspace_bytes, void* stream);
+int64_t fp8blk_amax_ema_workspace_bytes(int64_t rows);
+
+/*
+ * Quantise a whole tensor with the one scale *scale (device float, e.g. from
+ * fp8blk_amax_ema): q = E4M3(RN(clamp(x / scale, -448, 448))).  A stale amax
+ * may put |x / scale| far above 448: those values saturate to +-448.
+ *   x [rows][ldx] bf16 -> q [rows][cols] E4M3.
+ */
+fp8blk_status fp8blk_quantize_tensor(const void* x, int64_t rows, int64_t cols, int64_t ldx, const float* scale,
+                                     uint8_t* q, void* stream);
+
+/*
+ * GEMM with one scale per operand ([EXPL] FP8Linear.forward: the product of
+ * the dequantised operands):  D[m][n] = bf16( *sa * *sb * sum_k a[m][k] b[n][k] ),
+ * the sum accumulated in fp32 on the tensor cores over the whole K loop.
+ *   a [M][K] E4M3, b [N][K] E4M3 (both K-major), sa / sb device floats,
+ *   d [M][ldd] bf16 (ldd % 16 == 0, d 32-byte aligned).  Errors as for fp8blk_gemm.
+ */
+fp8blk_status fp8blk_gemm_tensor_scaled(int64_t M, int64_t N, int64_t K, const uint8_t* a, const float* sa,
+                                        const uint8_t* b, const float* sb, void* d, int64_t ldd, void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device error word of the

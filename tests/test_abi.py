@@ -106,6 +106,8 @@ def test_quantize_weight_both_argument_errors():
     ((2, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, NULL, ALIGNED, 128, S), 1),
     ((0, 128, 256, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 1),   # ldd < N
     ((0, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 132, S), 3),   # ldd % 8
+    ((0, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 136, S), 3),   # rows not 32-byte aligned
+    ((0, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, P(0x10010), 128, S), 3),  # d not 32-byte aligned
     ((0, 128, 128, 128, MISALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 3),
     ((1, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, MISALIGNED, 128, S), 3),
 ])
@@ -126,3 +128,18 @@ def test_binding_refuses_cpu_tensors():
 def test_valid_call_without_a_gpu_reports_a_cuda_error():
     st = _lib.lib.fp8blk_quantize_act_1x128(ALIGNED, 128, 128, 128, 1, ALIGNED, ALIGNED, NULL, NULL, S)
     assert st in (4, 7)
+
+
+def test_delayed_scaling_argument_errors():
+    L = _lib.lib
+    A = ALIGNED
+    assert L.fp8blk_amax_ema_workspace_bytes(128) == 32 and L.fp8blk_amax_ema_workspace_bytes(0) == 0
+    assert L.fp8blk_amax_ema(A, 128, 128, 128, A, A, A, 31, S) == 1          # workspace too small
+    assert L.fp8blk_amax_ema(A, 128, 128, 128, NULL, A, A, 64, S) == 1       # no amax buffer
+    assert L.fp8blk_amax_ema(A, 128, 100, 128, A, A, A, 64, S) == 2
+    assert L.fp8blk_amax_ema(A, 128, 128, 128, A, A, MISALIGNED, 64, S) == 3
+    assert L.fp8blk_quantize_tensor(A, 128, 128, 128, NULL, A, S) == 1
+    assert L.fp8blk_quantize_tensor(A, 128, 128, 128, A, MISALIGNED, S) == 3
+    assert L.fp8blk_gemm_tensor_scaled(128, 128, 96, A, A, A, A, A, 128, S) == 2
+    assert L.fp8blk_gemm_tensor_scaled(128, 128, 128, A, NULL, A, A, A, 128, S) == 1
+    assert L.fp8blk_gemm_tensor_scaled(128, 256, 128, A, A, A, A, A, 128, S) == 1   # ldd < N
