@@ -28,7 +28,7 @@ struct QuantArgs {
 cudaError_t launch_quant(int mode, const QuantArgs& a, cudaStream_t stream);
 
 // Per-tensor delayed scaling (tensor.cu).
-constexpr int kTensorRowsPerPartial = 16;   // rows reduced by one CTA of the amax reduction
+constexpr int kTensorRowsPerPartial = 8;    // rows reduced by one CTA of the amax reduction
 struct TensorArgs {
   const uint16_t* x;  // [rows][ldx] bf16
   int64_t rows, cols, ldx;

@@ -4,9 +4,10 @@
 // average (beta = 0.99) before the tensor is quantised with the single scale
 // max(amax / 448, 1e-12).
 //
-//   amax_partials_kernel  max |x| of each 16-row block of the tensor, one
+//   amax_partials_kernel  max |x| of each 8-row block of the tensor, one
 //                         partial per CTA into a workspace (HBM bound: 2 B
-//                         read per element, 16-byte loads);
+//                         read per element, 16-byte loads, 8 in flight per
+//                         thread);
 //   amax_finalize_kernel  one CTA: the maximum of the partials, the EMA in
 //                         binary32 (RN(RN(amax * b) + RN(cur * c)) with
 //                         b = RN32(0.99), c = RN32(1 - 0.99)), and the scale by
@@ -39,18 +40,25 @@ __device__ __forceinline__ uint32_t absmax_bits8(const uint4& v) {
 
 }  // namespace
 
-// CTA b: rows [16 b, 16 b + 16) x all columns; partials[b] = their max |x| as
-// bf16 magnitude bits (the order of finite bf16 magnitudes is that of their bits).
+// CTA b: rows [R b, R b + R) x all columns, R = kTensorRowsPerPartial;
+// partials[b] = their max |x| as bf16 magnitude bits (the order of finite bf16
+// magnitudes is that of their bits).  Thread t reads 16-byte chunks t, t + 256,
+// ... of all R rows, the R loads of one chunk column issued back to back so
+// that R x 16 bytes per thread are in flight (a warp covers 512 contiguous
+// bytes of each row).  Rows are a multiple of 128, so every CTA has R rows.
 __global__ void __launch_bounds__(kReduceThreads) amax_partials_kernel(const uint16_t* x, int64_t rows, int64_t cols,
                                                                        int64_t ldx, uint32_t* partials) {
+  static_assert(128 % kTensorRowsPerPartial == 0, "row blocks must tile a multiple of 128 rows");
   griddep_wait();
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kTensorRowsPerPartial;
-  const int64_t nrows = min(static_cast<int64_t>(kTensorRowsPerPartial), rows - r0);
+  const uint16_t* base = x + static_cast<int64_t>(blockIdx.x) * kTensorRowsPerPartial * ldx;
   const int64_t chunks = cols / 8;   // 16-byte chunks per row (cols is a multiple of 128)
   uint32_t m = 0;
-  for (int64_t i = threadIdx.x; i < nrows * chunks; i += kReduceThreads) {
-    const int64_t r = r0 + i / chunks, c = (i % chunks) * 8;
-    m = max(m, absmax_bits8(ld_nc_v4(x + r * ldx + c)));
+  for (int64_t c = threadIdx.x; c < chunks; c += kReduceThreads) {
+    uint4 v[kTensorRowsPerPartial];
+#pragma unroll
+    for (int r = 0; r < kTensorRowsPerPartial; ++r) v[r] = ld_nc_v4(base + r * ldx + c * 8);
+#pragma unroll
+    for (int r = 0; r < kTensorRowsPerPartial; ++r) m = max(m, absmax_bits8(v[r]));
   }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));

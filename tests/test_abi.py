@@ -133,8 +133,8 @@ def test_valid_call_without_a_gpu_reports_a_cuda_error():
 def test_delayed_scaling_argument_errors():
     L = _lib.lib
     A = ALIGNED
-    assert L.fp8blk_amax_ema_workspace_bytes(128) == 32 and L.fp8blk_amax_ema_workspace_bytes(0) == 0
-    assert L.fp8blk_amax_ema(A, 128, 128, 128, A, A, A, 31, S) == 1          # workspace too small
+    assert L.fp8blk_amax_ema_workspace_bytes(128) == 64 and L.fp8blk_amax_ema_workspace_bytes(0) == 0
+    assert L.fp8blk_amax_ema(A, 128, 128, 128, A, A, A, 63, S) == 1          # workspace too small
     assert L.fp8blk_amax_ema(A, 128, 128, 128, NULL, A, A, 64, S) == 1       # no amax buffer
     assert L.fp8blk_amax_ema(A, 128, 100, 128, A, A, A, 64, S) == 2
     assert L.fp8blk_amax_ema(A, 128, 128, 128, A, A, MISALIGNED, 64, S) == 3
