@@ -32,6 +32,7 @@ from ._lib import (A_E5M2, B_E5M2, BOTH, COLWISE_T, DGRAD, E5M2, FWD, ROWWISE, W
 __all__ = [
     "fp8blk_quantize_act_1x128", "fp8blk_quantize_weight_128x128", "fp8blk_quantize_weight_128x128_t",
     "fp8blk_quantize_weight_128x128_both", "fp8blk_amax_ema", "fp8blk_amax_ema_workspace_bytes",
+    "fp8blk_amax_ema_static", "AMAX_EMA_STATIC_MAX_ROWS",
     "fp8blk_quantize_tensor", "fp8blk_gemm_tensor_scaled", "fp8_linear_delayed_forward",
     "fp8blk_gemm", "fp8blk_get_device_error", "fp8blk_version", "linear_forward", "linear_backward",
     "ROWWISE", "COLWISE_T", "BOTH", "E5M2", "FWD", "DGRAD", "WGRAD", "A_E5M2", "B_E5M2", "Fp8BlkError",
@@ -175,6 +176,26 @@ def fp8blk_amax_ema(x, amax, scale=None, workspace=None, stream=None):
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
     check(lib.fp8blk_amax_ema(_ptr(x), rows, cols, x.stride(0), _ptr(amax), _ptr(scale), _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream_handle(stream)))
+    return amax, scale
+
+
+AMAX_EMA_STATIC_MAX_ROWS = 65536   # FP8BLK_AMAX_EMA_STATIC_MAX_ROWS
+
+
+def fp8blk_amax_ema_static(x, amax, scale, stream=None):
+    """fp8blk_amax_ema with the library's own fixed scratch: allocates nothing (scale is required,
+    float32 [1] on the device).  Calls on one device must be ordered; the first call on a device
+    must come before graph capture.  Returns (amax, scale)."""
+    x = _bf16_2d(x)
+    if scale is None:
+        raise ValueError("scale is required: this entry point allocates nothing")
+    _need_cuda(x, amax, scale)
+    rows, cols = x.shape
+    for t, name in ((amax, "amax"), (scale, "scale")):
+        if t.dtype != torch.float32 or t.numel() != 1:
+            raise ValueError(f"{name} must be a float32 tensor with one element")
+    check(lib.fp8blk_amax_ema_static(_ptr(x), rows, cols, x.stride(0), _ptr(amax), _ptr(scale),
+                                     _stream_handle(stream)))
     return amax, scale
 
 

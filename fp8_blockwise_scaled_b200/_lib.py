@@ -42,6 +42,7 @@ def _load() -> ctypes.CDLL:
         "fp8blk_quantize_weight_128x128_both": [P, I64, I64, I64, P, P, P, P, P],
         "fp8blk_amax_ema": [P, I64, I64, I64, P, P, P, I64, P],
         "fp8blk_amax_ema_workspace_bytes": [I64],
+        "fp8blk_amax_ema_static": [P, I64, I64, I64, P, P, P],
         "fp8blk_quantize_tensor": [P, I64, I64, I64, P, P, P],
         "fp8blk_gemm_tensor_scaled": [I64, I64, I64, P, P, P, P, P, I64, P],
         "fp8blk_gemm": [I, I64, I64, I64, P, P, P, P, P, I64, P],

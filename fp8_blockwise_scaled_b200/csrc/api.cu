@@ -228,6 +228,21 @@ fp8blk_status fp8blk_amax_ema(const void* x, int64_t rows, int64_t cols, int64_t
   return launch_status(fp8blk::launch_amax_ema(t, static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream)));
 }
 
+fp8blk_status fp8blk_amax_ema_static(const void* x, int64_t rows, int64_t cols, int64_t ldx, float* amax,
+                                     float* scale, void* stream) {
+  static_assert(FP8BLK_AMAX_EMA_STATIC_MAX_ROWS == fp8blk::kStaticAmaxMaxRows, "header and library disagree");
+  fp8blk_status st = check_quant_common(x, rows, cols, ldx);
+  if (st != FP8BLK_OK) return st;
+  if (rows > FP8BLK_AMAX_EMA_STATIC_MAX_ROWS) return FP8BLK_ERR_SHAPE;
+  if (!amax || !scale) return FP8BLK_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(amax) & 3u) || (reinterpret_cast<uintptr_t>(scale) & 3u)) return FP8BLK_ERR_ALIGN;
+  if ((st = check_device()) != FP8BLK_OK) return st;
+  uint32_t* partials = nullptr;
+  if (fp8blk::static_amax_partials(&partials) != cudaSuccess) return FP8BLK_ERR_CUDA;
+  fp8blk::TensorArgs t{static_cast<const uint16_t*>(x), rows, cols, ldx, amax, scale, pdl_enabled()};
+  return launch_status(fp8blk::launch_amax_ema(t, partials, static_cast<cudaStream_t>(stream)));
+}
+
 fp8blk_status fp8blk_quantize_tensor(const void* x, int64_t rows, int64_t cols, int64_t ldx, const float* scale,
                                      uint8_t* q, void* stream) {
   fp8blk_status st = check_quant_common(x, rows, cols, ldx);

@@ -38,6 +38,13 @@ struct TensorArgs {
 };
 // partials: ceil(rows / kTensorRowsPerPartial) words of scratch, fully rewritten.
 cudaError_t launch_amax_ema(const TensorArgs& t, uint32_t* partials, cudaStream_t stream);
+// The allocation-free variant keeps its partials in a fixed device array of
+// this library: tensors of at most kStaticAmaxMaxRows rows.
+constexpr int64_t kStaticAmaxMaxRows = 65536;
+constexpr int kStaticAmaxPartials = static_cast<int>(kStaticAmaxMaxRows / kTensorRowsPerPartial);   // 32 KiB
+// Device address of that array on the current device; cudaGetSymbolAddress
+// runs once per device (the first call), later calls return the cached address.
+cudaError_t static_amax_partials(uint32_t** out);
 cudaError_t launch_quant_tensor(const TensorArgs& t, uint8_t* q, cudaStream_t stream);
 
 struct GemmArgs {

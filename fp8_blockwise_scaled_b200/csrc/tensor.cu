@@ -19,7 +19,9 @@
 //                         above 448; inputs beyond 1024 s are first clamped to
 //                         +-1024 s (same saturated code, no overflow to
 //                         infinity in the quotient).
+#include <atomic>
 #include <cfloat>
+#include <mutex>
 
 #include "device.cuh"
 #include "kernels.h"
@@ -37,6 +39,11 @@ __device__ __forceinline__ uint32_t absmax_bits8(const uint4& v) {
   const uint32_t m = __vmaxu2(__vmaxu2(v.x & kAbs2, v.y & kAbs2), __vmaxu2(v.z & kAbs2, v.w & kAbs2));
   return max(m & 0xFFFFu, m >> 16);
 }
+
+// Partials of fp8blk_amax_ema_static: every call rewrites the words it reads
+// (one per 8-row block of its tensor) before the finalize kernel reads them,
+// so nothing here needs to start at zero.
+static __device__ __align__(256) uint32_t g_static_amax_partials[kStaticAmaxPartials];
 
 }  // namespace
 
@@ -128,6 +135,30 @@ cudaError_t launch_amax_ema(const TensorArgs& t, uint32_t* partials, cudaStream_
                          t.scale, static_cast<float>(beta), static_cast<float>(1.0 - beta));
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+cudaError_t static_amax_partials(uint32_t** out) {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<uint32_t*> cached[kMaxDevices];   // static storage: starts null
+  static std::mutex lookup;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  uint32_t* p = cached[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> hold(lookup);
+    p = cached[dev].load(std::memory_order_relaxed);
+    if (p == nullptr) {
+      void* addr = nullptr;
+      e = cudaGetSymbolAddress(&addr, g_static_amax_partials);
+      if (e != cudaSuccess) return e;
+      p = static_cast<uint32_t*>(addr);
+      cached[dev].store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
+  return cudaSuccess;
 }
 
 cudaError_t launch_quant_tensor(const TensorArgs& t, uint8_t* q, cudaStream_t stream) {

@@ -178,6 +178,28 @@ fp8blk_status fp8blk_amax_ema(const void* x, int64_t rows, int64_t cols, int64_t
 int64_t fp8blk_amax_ema_workspace_bytes(int64_t rows);
 
 /*
+ * fp8blk_amax_ema without a caller workspace and without allocating: the same
+ * two kernels and the same result bits, the partial maxima kept in a fixed
+ * 32 KiB device array inside this library.  The pages have no counterpart of
+ * this entry point; it serves callers that must not allocate (an allocator
+ * being set up, a captured graph built without a memory pool).
+ *   Rows above FP8BLK_AMAX_EMA_STATIC_MAX_ROWS: FP8BLK_ERR_SHAPE; other
+ *   argument errors as for fp8blk_amax_ema.
+ *   Nothing needs to start at zero: each call rewrites every partial it reads.
+ *   The array is one per device and per process: calls on one device must be
+ *   ordered (one stream, or events); two in flight at once on different
+ *   streams race on it and may return a wrong amax.
+ *   The first call on a device looks up the array's address
+ *   (cudaGetSymbolAddress; a failure returns FP8BLK_ERR_CUDA) and caches it:
+ *   make that call before capturing a CUDA graph that contains this entry
+ *   point.  Later calls look nothing up and allocate nothing: the device
+ *   check and the two kernel launches.
+ */
+#define FP8BLK_AMAX_EMA_STATIC_MAX_ROWS 65536
+fp8blk_status fp8blk_amax_ema_static(const void* x, int64_t rows, int64_t cols, int64_t ldx, float* amax,
+                                     float* scale, void* stream);
+
+/*
  * Quantise a whole tensor with the one scale *scale (device float, e.g. from
  * fp8blk_amax_ema): q = E4M3(RN(clamp(x / scale, -448, 448))).  A stale amax
  * may put |x / scale| far above 448: those values saturate to +-448.

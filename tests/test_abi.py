@@ -138,8 +138,17 @@ def test_delayed_scaling_argument_errors():
     assert L.fp8blk_amax_ema(A, 128, 128, 128, NULL, A, A, 64, S) == 1       # no amax buffer
     assert L.fp8blk_amax_ema(A, 128, 100, 128, A, A, A, 64, S) == 2
     assert L.fp8blk_amax_ema(A, 128, 128, 128, A, A, MISALIGNED, 64, S) == 3
+    assert L.fp8blk_amax_ema_static(A, 65536 + 128, 128, 128, A, A, S) == 2   # above the static array
+    assert L.fp8blk_amax_ema_static(A, 128, 128, 128, NULL, A, S) == 1
+    assert L.fp8blk_amax_ema_static(A, 128, 128, 128, A, P(0x10002), S) == 3   # scale not 4-byte aligned
     assert L.fp8blk_quantize_tensor(A, 128, 128, 128, NULL, A, S) == 1
     assert L.fp8blk_quantize_tensor(A, 128, 128, 128, A, MISALIGNED, S) == 3
     assert L.fp8blk_gemm_tensor_scaled(128, 128, 96, A, A, A, A, A, 128, S) == 2
     assert L.fp8blk_gemm_tensor_scaled(128, 128, 128, A, NULL, A, A, A, 128, S) == 1
     assert L.fp8blk_gemm_tensor_scaled(128, 256, 128, A, A, A, A, A, 128, S) == 1   # ldd < N
+
+
+def test_static_amax_row_limit_matches_the_header():
+    text = open(HEADER).read()
+    assert int(re.search(r"#define FP8BLK_AMAX_EMA_STATIC_MAX_ROWS (\d+)", text).group(1)) == \
+        fb.AMAX_EMA_STATIC_MAX_ROWS
