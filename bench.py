@@ -530,7 +530,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "per_op_median": per_op,
         "e2e": {"value": flops_all * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": nops * args.steps,
+        # one kernel per op, two for an amax EMA (partial maxima, then the EMA)
+        "gpu_launches": sum(2 if ".amax_" in label else 1 for label, _, _, _ in prog.ops) * args.steps,
         "clocks": clocks,
         "device_error": prog.fb.status_string(err),
     }
