@@ -31,7 +31,8 @@
 //               registers with packed f32x2 FMAs,
 //                   FWD/DGRAD: acc += P * (sa[m] * sb[n-block])
 //                   WGRAD    : acc += (P * sb[n]) * sa[m]
-//               then hand the TMEM buffer and the scale slot back; after the
+//               handing the TMEM buffer back as soon as its last load has
+//               landed (before those FMAs) and the scale slot after them; after the
 //               last K-block they round the tile to bf16 and store it with
 //               32-byte vector stores.
 // The MMA of K-block kb+1 runs while the promotion of kb is in flight
@@ -521,6 +522,15 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
         const float f = kWgrad ? 0.0f : sa * ss.sb[BN == 256 ? wg : 0];
         const float* sbc = ss.sb + col0;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * BN + col0;
+        // The accumulator buffer goes back to the MMA issuer as soon as this
+        // warp's last TMEM load has landed in registers, before the FMAs that
+        // consume it: the next K-block's MMAs into this buffer wait only for
+        // the reads, not for the arithmetic.
+        auto release_tmem = [&]() {
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctrl->tempty[abuf]);
+        };
         if constexpr (C::kHalf == 64) {
           // 64 columns per thread: all four loads in flight, one wait.
           uint32_t r0[16], r1[16], r2[16], r3[16];
@@ -532,6 +542,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
           tmem_wait_ld16(r1);
           tmem_wait_ld16(r2);
           tmem_wait_ld16(r3);
+          release_tmem();
           promote16<kWgrad>(acc, r0, f, sbc, sa);
           promote16<kWgrad>(acc + 8, r1, f, sbc + 16, sa);
           promote16<kWgrad>(acc + 16, r2, f, sbc + 32, sa);
@@ -543,6 +554,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
             uint32_t r[64];
             tmem_ld_32x32b_x64(taddr + c, r);
             tmem_wait_ld64(r);
+            if (c + 64 == C::kHalf) release_tmem();
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               promote16<kWgrad>(acc + c / 2 + 8 * q, *reinterpret_cast<const uint32_t(*)[16]>(r + 16 * q), f,
@@ -558,6 +570,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
             tmem_ld_32x32b_x16(taddr + c + 16, rb);
             promote16<kWgrad>(acc + c / 2, ra, f, sbc + c, sa);
             tmem_wait_ld16(rb);
+            if (c + 32 == C::kHalf) release_tmem();
             if (c + 32 < C::kHalf) tmem_ld_32x32b_x16(taddr + c + 32, ra);
             promote16<kWgrad>(acc + c / 2 + 8, rb, f, sbc + c + 16, sa);
             if (c + 32 < C::kHalf) tmem_wait_ld16(ra);
@@ -568,15 +581,12 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
             uint32_t r[16];
             tmem_ld_32x32b_x16(taddr + c, r);
             tmem_wait_ld16(r);
+            if (c + 16 == C::kHalf) release_tmem();
             promote16<kWgrad>(acc + c / 2, r, f, sbc + c, sa);
           }
         }
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&ctrl->tempty[abuf]);
-          mbar_arrive(&ctrl->sempty[slot]);
-        }
+        __syncwarp();   // every lane has read its scales from the slot
+        if (lane == 0) mbar_arrive(&ctrl->sempty[slot]);
         if (++abuf == C::kAccBufs) {
           abuf = 0;
           aphase ^= 1u;
