@@ -97,23 +97,49 @@ __global__ void __launch_bounds__(kFinalizeThreads) amax_finalize_kernel(const u
   }
 }
 
-// Every element with the single scale *scale; 8 elements per thread per step.
+// Every element with the single scale *scale.  Thread t starts at 16-byte
+// chunk t of the flattened [rows][cols / 8] chunk grid and strides by the
+// grid's thread count, split on the host into whole rows (step_r) and extra
+// chunks (step_c) so that no division sits in the loop; four chunks per
+// iteration are loaded before any is converted (four loads in flight).
 __global__ void __launch_bounds__(kQuantThreads) quant_tensor_kernel(const uint16_t* x, int64_t rows, int64_t cols,
-                                                                     int64_t ldx, const float* scale, uint8_t* q) {
+                                                                     int64_t ldx, const float* scale, uint8_t* q,
+                                                                     int64_t step_r, int64_t step_c) {
   griddep_wait();
   const float s = *scale;
   const QScale qs{s, -__frcp_rn(s)};
   const float lim = fminf(1024.0f * s, FLT_MAX);   // 1024 s saturates like anything larger
   const int64_t chunks = cols / 8;
-  const int64_t total = rows * chunks;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * kQuantThreads) {
-    const int64_t r = i / chunks, c = (i % chunks) * 8;
-    float f[8];
-    unpack8(ld_nc_v4(x + r * ldx + c), f);
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
+  int64_t r = first / chunks, c = first % chunks;
+  constexpr int kUnroll = 4;
+  while (r < rows) {
+    int64_t pr[kUnroll], pc[kUnroll];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) f[j] = fminf(fmaxf(f[j], -lim), lim);
-    *reinterpret_cast<uint2*>(q + r * cols + c) = quant8<false>(f, qs);
+    for (int u = 0; u < kUnroll; ++u) {
+      pr[u] = r;
+      pc[u] = c;
+      r += step_r;
+      c += step_c;
+      if (c >= chunks) {
+        c -= chunks;
+        ++r;
+      }
+    }
+    uint4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      if (pr[u] < rows) v[u] = ld_nc_v4(x + pr[u] * ldx + pc[u] * 8);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (pr[u] < rows) {
+        float f[8];
+        unpack8(v[u], f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] = fminf(fmaxf(f[j], -lim), lim);
+        *reinterpret_cast<uint2*>(q + pr[u] * cols + pc[u] * 8) = quant8<false>(f, qs);
+      }
+    }
   }
 }
 
@@ -180,8 +206,10 @@ cudaError_t launch_quant_tensor(const TensorArgs& t, uint8_t* q, cudaStream_t st
   cudaLaunchAttribute attr[1];
   cfg.numAttrs = set_pdl_attr(attr, t.pdl);
   cfg.attrs = attr;
+  const int64_t chunks = t.cols / 8;
+  const int64_t step = static_cast<int64_t>(cfg.gridDim.x) * kQuantThreads;
   cudaError_t e = cudaLaunchKernelEx(&cfg, quant_tensor_kernel, t.x, t.rows, t.cols, t.ldx,
-                                     static_cast<const float*>(t.scale), q);
+                                     static_cast<const float*>(t.scale), q, step / chunks, step % chunks);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
