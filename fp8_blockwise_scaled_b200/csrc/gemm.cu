@@ -403,59 +403,72 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
                            abort, lane);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_e4m3_f32(BM, BN) | p.fmt_bits;
-      int stage = 0;
-      uint32_t phase = 0, abuf = 0, aphase = 0;
-      bool ok = true;
-      if (p.inject_stall) ok = mbar_wait_bounded(&ctrl->never, 0, abort, p.timeout_ns, p.err);
-      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-        if constexpr (kTensor) {   // one accumulator buffer per tile
-          if (!mbar_wait_bounded(&ctrl->tempty[abuf], aphase ^ 1u, abort, p.timeout_ns, p.err)) {
-            ok = false;
-            break;
-          }
+    // The whole warp runs the loop and waits, so the stage addresses,
+    // descriptors and counters are warp-uniform and reach tcgen05.mma from
+    // uniform registers; one elected lane issues the MMAs and the commits.
+    // (Run by a single lane, every MMA and commit paid a move of its operands
+    // into uniform registers: 70-100 cycles each, measured on B200, which
+    // put ~500 cycles of issue latency into every K-block.)
+    const bool leader = elect_one();
+    const uint32_t idesc = idesc_e4m3_f32(BM, BN) | p.fmt_bits;
+    int stage = 0;
+    uint32_t phase = 0, abuf = 0, aphase = 0;
+    bool ok = true;
+    if (p.inject_stall) ok = mbar_wait_bounded(&ctrl->never, 0, abort, p.timeout_ns, p.err);
+    ok = __all_sync(0xFFFFFFFFu, ok);
+    for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+      if constexpr (kTensor) {   // one accumulator buffer per tile
+        if (!__all_sync(0xFFFFFFFFu,
+                        mbar_wait_bounded(&ctrl->tempty[abuf], aphase ^ 1u, abort, p.timeout_ns, p.err))) {
+          ok = false;
+          break;
         }
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded(&ctrl->full[stage], phase, abort, p.timeout_ns, p.err) ||
-              (!kTensor && !mbar_wait_bounded(&ctrl->tempty[abuf], aphase ^ 1u, abort, p.timeout_ns, p.err))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
-          const uint32_t a_addr = smem_addr(smem + stage * C::kStageBytes);
-          const uint64_t adesc = smem_desc_kmajor_sw128(a_addr);
-          const uint64_t bdesc = smem_desc_kmajor_sw128(a_addr + C::kABytes);
-          const uint32_t d_tmem = tmem_base + abuf * BN;
+      }
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const bool got = mbar_wait_bounded(&ctrl->full[stage], phase, abort, p.timeout_ns, p.err) &&
+                         (kTensor || mbar_wait_bounded(&ctrl->tempty[abuf], aphase ^ 1u, abort, p.timeout_ns, p.err));
+        if (!__all_sync(0xFFFFFFFFu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t a_addr = smem_addr(smem + stage * C::kStageBytes);
+        const uint64_t adesc = smem_desc_kmajor_sw128(a_addr);
+        const uint64_t bdesc = smem_desc_kmajor_sw128(a_addr + C::kABytes);
+        const uint32_t d_tmem = tmem_base + abuf * BN;
+        if (leader) {
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k)  // 32 E4M3 values = 32 bytes = 2 x 16 B per step
             umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (k > 0 || (kTensor && kb > 0)) ? 1u : 0u);
           umma_commit(&ctrl->empty[stage]);
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-          if constexpr (!kTensor) {
-            umma_commit(&ctrl->tfull[abuf]);
-            if (++abuf == C::kAccBufs) {
-              abuf = 0;
-              aphase ^= 1u;
-            }
-          }
+          if constexpr (!kTensor) umma_commit(&ctrl->tfull[abuf]);
         }
-        if constexpr (kTensor) {
-          if (!ok) break;
-          umma_commit(&ctrl->tfull[abuf]);   // the tile's whole K loop is in this buffer
+        __syncwarp();
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        if constexpr (!kTensor) {
           if (++abuf == C::kAccBufs) {
             abuf = 0;
             aphase ^= 1u;
           }
         }
       }
-      // Every MMA issued so far has finished once this arrives.
-      umma_commit(&ctrl->mma_done);
-      mbar_wait_bounded(&ctrl->mma_done, 0, nullptr, p.timeout_ns, p.err);
+      if constexpr (kTensor) {
+        if (!ok) break;
+        if (leader) umma_commit(&ctrl->tfull[abuf]);   // the tile's whole K loop is in this buffer
+        __syncwarp();
+        if (++abuf == C::kAccBufs) {
+          abuf = 0;
+          aphase ^= 1u;
+        }
+      }
     }
+    // Every MMA issued so far has finished once this arrives.
+    if (leader) umma_commit(&ctrl->mma_done);
+    __syncwarp();
+    mbar_wait_bounded(&ctrl->mma_done, 0, nullptr, p.timeout_ns, p.err);
   }
   } else {
     if constexpr (kSplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
