@@ -10,31 +10,36 @@
 // the tensor cores produce one fp32 partial product per K-block and the
 // scales are applied to it before it joins the running sum.
 //
-// Design (one persistent CTA per SM, 384 threads, 128 x BN output tiles):
-//   warp 0      producer.  Lane 0 issues, per K-block, TMA loads of a 128x128
-//               A tile and a BNx128 B tile (E4M3, 128-byte swizzle) into a
-//               ring of shared-memory stages ("full" mbarrier counts bytes).
-//               All 32 lanes stream the K-block's scales (sa for the tile's
-//               128 rows; sb for its columns or n-blocks) into a separate
-//               8-deep shared-memory ring with cp.async, completion tracked
-//               by an mbarrier, so no global load sits on the promotion path.
-//   warp 1      TMEM owner and MMA issuer (one thread): 4 x tcgen05.mma
-//               kind::f8f6f4 (M=128, N=BN, K=32) per K-block into one of two
-//               TMEM accumulators (2 x BN fp32 columns), then tcgen05.commit
-//               to release the smem stage and to signal the accumulator.
-//   warps 2,3   idle: with warps 0 and 1 they form warpgroup 0, which hands
-//               most of its registers to the promotion warpgroups (setmaxnreg).
-//   warps 4..11 promotion + epilogue: two warpgroups, each owning BN/2
-//               columns of the tile (a warp reads the 32 TMEM lanes given by
-//               its index mod 4); per K-block they read the partial product
-//               from TMEM (double-buffered 16-column loads) and fold it into fp32
-//               registers with packed f32x2 FMAs,
+// Design (one persistent CTA per SM, 384 threads = 12 warps, 128 x BN output
+// tiles).  Warp roles, plain layout (split layout in brackets, see Layout):
+//   warp 0      A producer: lane 0 issues, per K-block, the TMA load of the
+//               128x128 A tile (E4M3, 128-byte swizzle) into a ring of
+//               shared-memory stages and arms the stage barrier with the
+//               bytes of both tiles.
+//   warp 11 [3] B producer: the BNx128 B tile of the same stage.
+//   warp 10 [2] scale producer: per K-block the tile's 128 per-row A scales
+//               (and, for WGRAD, the BN per-column B scales) by TMA bulk
+//               copies into an 8-deep scale ring; FWD/DGRAD's per-block B
+//               scales are read 32 K-blocks at a time and handed out by
+//               shuffle.  No global load sits on the promotion path.
+//   warp 1      TMEM owner and MMA issuer: the whole warp runs the loop, one
+//               elected lane issues 4 x tcgen05.mma kind::f8f6f4 (M=128,
+//               N=BN, K=32) per K-block into one of two TMEM accumulators
+//               (2 x BN fp32 columns), then tcgen05.commit to release the
+//               smem stage and to signal the accumulator.
+//   warps 2..9 [4..11]  promotion + epilogue: two warpgroups' worth of warps,
+//               each half owning BN/2 columns of the tile (a warp reads the
+//               32 TMEM lanes given by its index mod 4); per K-block they read
+//               the partial product from TMEM and fold it into fp32 registers
+//               with packed f32x2 FMAs,
 //                   FWD/DGRAD: acc += P * (sa[m] * sb[n-block])
 //                   WGRAD    : acc += (P * sb[n]) * sa[m]
 //               handing the TMEM buffer back as soon as its last load has
-//               landed (before those FMAs) and the scale slot after them; after the
-//               last K-block they round the tile to bf16 and store it with
-//               32-byte vector stores.
+//               landed (before those FMAs) and the scale slot after them;
+//               after the last K-block they round the tile to bf16 and store
+//               it with 32-byte vector stores.  In the split layout warpgroup
+//               0 (warps 0-3) hands registers to the promotion warps with
+//               setmaxnreg, which pays for 64-column TMEM loads.
 // The MMA of K-block kb+1 runs while the promotion of kb is in flight
 // (double-buffered TMEM), and TMA runs up to kStages K-blocks ahead.
 //
