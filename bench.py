@@ -51,8 +51,8 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM traffic of the 12 GEMM launches of one decoder-layer step at 16384 tokens
 # (dram__bytes_read.sum + dram__bytes_write.sum, one ncu pass over the launches of
 # one step; profiles/gemm_dram_layer_16384.md), for the GEMM kernel of commit
-# 639beb8; algorithmic minimum 2.59 GB (codes read once, bf16 outputs written once).
-GEMM_STEP_DRAM_BYTES_16384 = 2.94e9
+# f6bf0e3; algorithmic minimum 2.59 GB (codes read once, bf16 outputs written once).
+GEMM_STEP_DRAM_BYTES_16384 = 2.95e9
 
 WORKLOAD_DESC = {
     "layer": "qwen2-1.5b-shaped decoder layer linears (qkv 2048x1536, o 1536x1536, gate_up 17920x1536, "
