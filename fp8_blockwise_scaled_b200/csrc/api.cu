@@ -206,6 +206,7 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   if (const char* e = std::getenv("FP8BLK_GEMM_GROUP_M")) g.group_m = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_TMEM_DB")) g.tmem_db = std::atoi(e);
+  if (const char* e = std::getenv("FP8BLK_GEMM_QUAD")) g.quad = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) g.inject_stall = std::atoi(e) != 0;
   return launch_status(fp8blk::launch_gemm(g, static_cast<cudaStream_t>(stream)));
 }

@@ -75,15 +75,27 @@ constexpr int kSRing = 8;        // scale ring depth (K-blocks)
 // 16 KB boxes 46 B/clk per issuing thread, two issuing warps 76 B/clk), so
 // A and B tiles are issued by different warps.  The scale producer runs
 // ahead of the operand ring by up to the scale ring's depth.
+// Quad layout (kQuad, split layout only): 20 warps, warpgroup 0 as in the
+// split layout and 16 promotion warps, four per TMEM lane quadrant, each
+// owning BN/4 columns; the launch allocates 96 registers per thread, and
+// setmaxnreg gives warpgroup 0 64 and the promotion warps 104.
 constexpr int kLowRegs = 56;
 constexpr int kHighRegs = 224;
 static_assert(128 * kLowRegs + 256 * kHighRegs == 384 * 168, "register split must match the launch allocation");
-template <bool kSplit>
+constexpr int kQuadLowRegs = 64;
+constexpr int kQuadHighRegs = 104;
+static_assert(128 * kQuadLowRegs + 512 * kQuadHighRegs == 640 * 96, "quad register split must match 96 per thread");
+template <bool kSplit, bool kQuad = false>
 struct Layout {
-  static constexpr int kThreads = 384;
+  static_assert(!kQuad || kSplit, "the quad layout is a split layout");
+  static constexpr int kThreads = kQuad ? 640 : 384;
+  static constexpr int kPromoWarps = kQuad ? 16 : 8;
   static constexpr int kEpiWarp0 = kSplit ? 4 : 2;
   static constexpr int kScaleWarp = kSplit ? 2 : 10;
   static constexpr int kBWarp = kSplit ? 3 : 11;
+  static constexpr int kLow = kQuad ? kQuadLowRegs : kLowRegs;
+  static constexpr int kHigh = kQuad ? kQuadHighRegs : kHighRegs;
+  static_assert(kLow % 8 == 0 && kHigh % 8 == 0, "setmaxnreg takes multiples of 8");
 };
 
 template <int BN>
@@ -96,7 +108,6 @@ struct Cfg {
   // that the MMA can run three K-blocks ahead of the promotion.
   static constexpr int kAccBufs = (BN == 256) ? 2 : 4;
   static constexpr int kTmemCols = kAccBufs * BN;
-  static constexpr int kHalf = BN / 2;  // columns per epilogue warpgroup
 };
 
 // One K-block's scales for one tile.
@@ -301,14 +312,19 @@ __device__ __forceinline__ void tile_coords(int tile, int num_mb, int num_nb, in
 // kTensor: one scale per operand (per-tensor scaling).  No per-K-block
 // promotion: the MMAs accumulate the whole K loop of a tile in TMEM and the
 // promotion warps only apply sa * sb, round to bf16 and store, once per tile.
-template <int BN, bool kWgrad, bool kSplit, bool kTensor = false>
-__global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
+template <int BN, bool kWgrad, bool kSplit, bool kTensor = false, bool kQuad = false>
+__global__ void __launch_bounds__(Layout<kSplit, kQuad>::kThreads, 1)
     gemm_blockwise_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const GemmParams p) {
   using C = Cfg<BN>;
-  constexpr int kEpiWarp0 = Layout<kSplit>::kEpiWarp0;
-  constexpr bool kTmemDB = kSplit;
-  constexpr bool kWide = kSplit;  // the split layout has the registers for 64-column TMEM reads
+  using L = Layout<kSplit, kQuad>;
+  constexpr int kEpiWarp0 = L::kEpiWarp0;
+  constexpr int kPromo = L::kPromoWarps;
+  constexpr int kCols = BN / (kPromo / 4);   // columns per promotion warp
+  // The split layout has the registers for 64-column TMEM reads; the quad
+  // layout's promotion warps read their columns 16 at a time.
+  constexpr bool kTmemDB = kSplit && !kQuad;
+  constexpr bool kWide = kSplit && !kQuad;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + C::kStages * C::kStageBytes);
@@ -327,11 +343,11 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     }
     for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&ctrl->tfull[b], 1);
-      mbar_init(&ctrl->tempty[b], kEpiWarps);
+      mbar_init(&ctrl->tempty[b], kPromo);
     }
     for (int s = 0; s < kSRing; ++s) {
       mbar_init(&ctrl->sfull[s], 1);    // the scale producer's arrive + the bytes of its copies
-      mbar_init(&ctrl->sempty[s], kEpiWarps);
+      mbar_init(&ctrl->sempty[s], kPromo);
     }
     mbar_init(&ctrl->mma_done, 1);
     mbar_init(&ctrl->never, 1);
@@ -352,9 +368,9 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
   const uint32_t tmem_base = ctrl->tmem_base;
   volatile int* abort = &ctrl->abort;
 
-  if (warp < kEpiWarp0 || warp >= kEpiWarp0 + kEpiWarps) {
-  if constexpr (kSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
-  if (warp == 0 || warp == Layout<kSplit>::kBWarp) {
+  if (warp < kEpiWarp0 || warp >= kEpiWarp0 + kPromo) {
+  if constexpr (kSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(L::kLow));
+  if (warp == 0 || warp == L::kBWarp) {
     // ------------------------------------------------------------ operand producers (A: warp 0, B: kBWarp)
     // Both wait for the same free stage; the A producer arms the stage's full
     // barrier with the bytes of both tiles (the B bytes may land first: the
@@ -395,7 +411,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
         mbar_wait_bounded(&ctrl->full[j % C::kStages], static_cast<uint32_t>((j / C::kStages) & 1), nullptr,
                           p.timeout_ns, p.err);
     }
-  } else if (warp == Layout<kSplit>::kScaleWarp) {
+  } else if (warp == L::kScaleWarp) {
     // ------------------------------------------------------------ scale producer (whole warp)
     if constexpr (!kTensor)
       scale_feed<BN, kWgrad>(ctrl, p, blockIdx.x, gridDim.x, tiles, kblocks,
@@ -476,13 +492,13 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     mbar_wait_bounded(&ctrl->mma_done, 0, nullptr, p.timeout_ns, p.err);
   }
   } else {
-    if constexpr (kSplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
+    if constexpr (kSplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(L::kHigh));
     // ------------------------------------------------------------ promotion + epilogue
-    const int ew = warp - kEpiWarp0;  // 0..7
-    const int wg = ew >> 2;           // which half of the tile's columns
+    const int ew = warp - kEpiWarp0;  // 0 .. kPromo - 1
+    const int wg = ew >> 2;           // which slice of the tile's columns
     const int quarter = warp & 3;     // TMEM lanes this warp may read
     const int row = quarter * 32 + lane;
-    const int col0 = wg * C::kHalf;
+    const int col0 = wg * kCols;
     uint32_t abuf = 0, aphase = 0, sphase = 0;
     int slot = 0;
     bool ok = true;
@@ -498,7 +514,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * BN + col0;
         uint16_t* drow = p.d + (static_cast<int64_t>(mb) * BM + row) * p.ldd + static_cast<int64_t>(nb) * BN + col0;
 #pragma unroll
-        for (int c = 0; c < C::kHalf; c += 16) {
+        for (int c = 0; c < kCols; c += 16) {
           uint32_t r[16];
           tmem_ld_32x32b_x16(taddr + c, r);
           tmem_wait_ld16(r);
@@ -518,14 +534,14 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
       }
       ok = false;   // skip the blockwise loop below
     }
-    float2 acc[C::kHalf / 2];
+    float2 acc[kCols / 2];
     for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
       int mb, nb;
       tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
       const int64_t m = static_cast<int64_t>(mb) * BM + row;
       const int64_t ncol0 = static_cast<int64_t>(nb) * BN + col0;
 #pragma unroll
-      for (int j = 0; j < C::kHalf / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
+      for (int j = 0; j < kCols / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
 
       for (int kb = 0; kb < kblocks; ++kb) {
         const bool got = mbar_wait_bounded(&ctrl->sfull[slot], sphase, abort, p.timeout_ns, p.err) &&
@@ -537,7 +553,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
         tc_fence_after_sync();
         const ScaleSlot& ss = ctrl->slots[slot];
         const float sa = ss.sa[row];
-        const float f = kWgrad ? 0.0f : sa * ss.sb[BN == 256 ? wg : 0];
+        const float f = kWgrad ? 0.0f : sa * ss.sb[col0 / 128];   // the column slice's n-block
         const float* sbc = ss.sb + col0;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * BN + col0;
         // The accumulator buffer goes back to the MMA issuer as soon as this
@@ -549,7 +565,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctrl->tempty[abuf]);
         };
-        if constexpr (C::kHalf == 64) {
+        if constexpr (kCols == 64 && !kQuad) {
           // 64 columns per thread: all four loads in flight, one wait.
           uint32_t r0[16], r1[16], r2[16], r3[16];
           tmem_ld_32x32b_x16(taddr, r0);
@@ -568,11 +584,11 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
         } else if constexpr (kTmemDB && kWide) {
           // 64-column loads: two TMEM round trips per K-block for 128 columns.
 #pragma unroll
-          for (int c = 0; c < C::kHalf; c += 64) {
+          for (int c = 0; c < kCols; c += 64) {
             uint32_t r[64];
             tmem_ld_32x32b_x64(taddr + c, r);
             tmem_wait_ld64(r);
-            if (c + 64 == C::kHalf) release_tmem();
+            if (c + 64 == kCols) release_tmem();
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               promote16<kWgrad>(acc + c / 2 + 8 * q, *reinterpret_cast<const uint32_t(*)[16]>(r + 16 * q), f,
@@ -584,22 +600,22 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
           tmem_ld_32x32b_x16(taddr, ra);
           tmem_wait_ld16(ra);
 #pragma unroll
-          for (int c = 0; c < C::kHalf; c += 32) {
+          for (int c = 0; c < kCols; c += 32) {
             tmem_ld_32x32b_x16(taddr + c + 16, rb);
             promote16<kWgrad>(acc + c / 2, ra, f, sbc + c, sa);
             tmem_wait_ld16(rb);
-            if (c + 32 == C::kHalf) release_tmem();
-            if (c + 32 < C::kHalf) tmem_ld_32x32b_x16(taddr + c + 32, ra);
+            if (c + 32 == kCols) release_tmem();
+            if (c + 32 < kCols) tmem_ld_32x32b_x16(taddr + c + 32, ra);
             promote16<kWgrad>(acc + c / 2 + 8, rb, f, sbc + c + 16, sa);
-            if (c + 32 < C::kHalf) tmem_wait_ld16(ra);
+            if (c + 32 < kCols) tmem_wait_ld16(ra);
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < C::kHalf; c += 16) {
+          for (int c = 0; c < kCols; c += 16) {
             uint32_t r[16];
             tmem_ld_32x32b_x16(taddr + c, r);
             tmem_wait_ld16(r);
-            if (c + 16 == C::kHalf) release_tmem();
+            if (c + 16 == kCols) release_tmem();
             promote16<kWgrad>(acc + c / 2, r, f, sbc + c, sa);
           }
         }
@@ -617,7 +633,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
       if (!ok) break;
       uint16_t* drow = p.d + m * p.ldd + ncol0;
 #pragma unroll
-      for (int j = 0; j < C::kHalf; j += 16) {
+      for (int j = 0; j < kCols; j += 16) {
         uint32_t v[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) v[q] = pack_bf16x2(acc[j / 2 + q].x, acc[j / 2 + q].y);
@@ -938,12 +954,12 @@ int num_sms() {
   return sms;
 }
 
-template <int BN, bool kWgrad, bool kSplit, bool kTensor = false>
+template <int BN, bool kWgrad, bool kSplit, bool kTensor = false, bool kQuad = false>
 cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   static bool attr_set = false;
   constexpr int kSmem = smem_bytes<BN>();
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_blockwise_kernel<BN, kWgrad, kSplit, kTensor>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_blockwise_kernel<BN, kWgrad, kSplit, kTensor, kQuad>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -959,13 +975,13 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(Layout<kSplit>::kThreads, 1, 1);
+  cfg.blockDim = dim3(Layout<kSplit, kQuad>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   cfg.numAttrs = set_pdl_attr(attr, g.pdl);
   cfg.attrs = attr;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<BN, kWgrad, kSplit, kTensor>, ta, tb, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<BN, kWgrad, kSplit, kTensor, kQuad>, ta, tb, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1039,6 +1055,14 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   // The register split with double-buffered TMEM reads pays off where the
   // promotion does more work per column (WGRAD); measured on B200, the plain
   // layout is faster for the forward/data-gradient promotion.
+  // Sixteen promotion warps (quad layout): opt-in.
+  if (g.quad > 0) {
+    if (bn == 256)
+      return wgrad ? launch_variant<256, true, true, false, true>(g, stream)
+                   : launch_variant<256, false, true, false, true>(g, stream);
+    return wgrad ? launch_variant<128, true, true, false, true>(g, stream)
+                 : launch_variant<128, false, true, false, true>(g, stream);
+  }
   const bool db = g.tmem_db < 0 ? wgrad : g.tmem_db != 0;
   if (bn == 256) {
     if (wgrad) return db ? launch_variant<256, true, true>(g, stream) : launch_variant<256, true, false>(g, stream);
