@@ -5,6 +5,7 @@
 #include <cstring>
 
 #include "../../include/fp8blk.h"
+#include "context.h"
 #include "device.cuh"
 #include "kernels.h"
 
@@ -15,19 +16,17 @@ __device__ unsigned int g_error_word = 0;
 
 namespace {
 
-// Device address of g_error_word on the current device (looked up once per device).
+// Device address of g_error_word in the current context (looked up once per context).
 unsigned int* error_word() {
-  static thread_local int dev_cached = -1;
-  static thread_local unsigned int* ptr = nullptr;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev != dev_cached) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, fp8blk::g_error_word) != cudaSuccess) return nullptr;
-    ptr = static_cast<unsigned int*>(p);
-    dev_cached = dev;
-  }
-  return ptr;
+  static fp8blk::PerContext<unsigned int*> cached;
+  unsigned int* p = nullptr;
+  const cudaError_t e = cached.get(&p, [](unsigned int** out) {
+    void* addr = nullptr;
+    const cudaError_t r = cudaGetSymbolAddress(&addr, fp8blk::g_error_word);
+    *out = static_cast<unsigned int*>(addr);
+    return r;
+  });
+  return e == cudaSuccess ? p : nullptr;
 }
 
 using fp8blk::QuantArgs;
@@ -196,7 +195,6 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   g.block_n = 0;
   g.err = error_word();
   if (!g.err) return FP8BLK_ERR_CUDA;
-  g.tmem_db = -1;
   g.pair = 0;   // pair tiles measured slower (cross-SM hand-offs per K-block); opt in with FP8BLK_GEMM_PAIR=1
   g.group_m = 0;
   g.pdl = pdl_enabled();
@@ -205,8 +203,6 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   if (const char* e = std::getenv("FP8BLK_GEMM_PAIR")) g.pair = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_GROUP_M")) g.group_m = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);
-  if (const char* e = std::getenv("FP8BLK_GEMM_TMEM_DB")) g.tmem_db = std::atoi(e);
-  if (const char* e = std::getenv("FP8BLK_GEMM_QUAD")) g.quad = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) g.inject_stall = std::atoi(e) != 0;
   return launch_status(fp8blk::launch_gemm(g, static_cast<cudaStream_t>(stream)));
 }
@@ -280,7 +276,6 @@ fp8blk_status fp8blk_gemm_tensor_scaled(int64_t M, int64_t N, int64_t K, const u
   g.timeout_ns = wait_timeout_ns();
   g.err = error_word();
   if (!g.err) return FP8BLK_ERR_CUDA;
-  g.tmem_db = -1;
   g.pdl = pdl_enabled();
   g.tensor_sa = sa;
   g.tensor_sb = sb;
@@ -290,10 +285,21 @@ fp8blk_status fp8blk_gemm_tensor_scaled(int64_t M, int64_t N, int64_t K, const u
 }
 
 fp8blk_status fp8blk_get_device_error(void* stream) {
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP8BLK_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FP8BLK_ERR_CUDA;
+  // The word read is the one of the device the stream belongs to (the legacy
+  // and per-thread default streams belong to the current device).
+  int cur = 0, dev = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return FP8BLK_ERR_CUDA;
+  dev = cur;
+  if (s != nullptr && s != cudaStreamLegacy && s != cudaStreamPerThread && cudaStreamGetDevice(s, &dev) != cudaSuccess)
+    return FP8BLK_ERR_CUDA;
+  if (dev != cur && cudaSetDevice(dev) != cudaSuccess) return FP8BLK_ERR_CUDA;
   unsigned int word = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&word, fp8blk::g_error_word, sizeof word) != cudaSuccess) return FP8BLK_ERR_CUDA;
-  if (word && cudaMemcpyToSymbol(fp8blk::g_error_word, &zero, sizeof zero) != cudaSuccess) return FP8BLK_ERR_CUDA;
+  bool ok = cudaMemcpyFromSymbol(&word, fp8blk::g_error_word, sizeof word) == cudaSuccess;
+  if (ok && word) ok = cudaMemcpyToSymbol(fp8blk::g_error_word, &zero, sizeof zero) == cudaSuccess;
+  if (dev != cur && cudaSetDevice(cur) != cudaSuccess) ok = false;
+  if (!ok) return FP8BLK_ERR_CUDA;
   return (word & fp8blk::kErrTimeoutBit) ? FP8BLK_ERR_TIMEOUT : FP8BLK_OK;
 }
 

@@ -58,17 +58,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
+// The same poll without the hint: a completed phase is seen in ~14 cycles
+// instead of ~47 (measured on B200), for the waits on the critical path of a
+// pipeline (the MMA issuer and the promotion warps of the GEMM).
+__device__ __forceinline__ bool mbar_try_wait_nohint(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 // Waits for the phase of `bar` with the given parity to complete.  Gives up
 // (returns false) when *abort becomes non-zero (abort may be null: then only
 // the time limit applies) or after timeout_ns of waiting; on a timeout it
 // raises *abort and the device error word so that every other role of the
-// CTA stops too.  Never traps.
+// CTA stops too.  Never traps.  kHint: poll with the suspend-time hint (roles
+// off the critical path) or without it (kHint = false).
+template <bool kHint = true>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                   uint64_t timeout_ns, unsigned int* err) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto poll = [&]() { return kHint ? mbar_try_wait(bar, parity) : mbar_try_wait_nohint(bar, parity); };
+  if (poll()) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (poll()) return true;
     if ((it & 63u) == 0) {
       if (abort && *abort) return false;
       if (global_timer_ns() - t0 > timeout_ns) {
@@ -218,9 +236,10 @@ __device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uin
 
 // mbar_wait_bounded for barriers that the other CTA of a pair arrives on.  On a
 // timeout it also raises the peer's abort flag (peer_abort: cluster address).
+template <bool kHint = true>
 __device__ __forceinline__ bool mbar_wait_bounded_pair(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                        uint32_t peer_abort, uint64_t timeout_ns, unsigned int* err) {
-  auto poll = [&]() { return mbar_try_wait(bar, parity); };
+  auto poll = [&]() { return kHint ? mbar_try_wait(bar, parity) : mbar_try_wait_nohint(bar, parity); };
   if (poll()) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {

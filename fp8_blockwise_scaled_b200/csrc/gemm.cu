@@ -10,42 +10,45 @@
 // the tensor cores produce one fp32 partial product per K-block and the
 // scales are applied to it before it joins the running sum.
 //
-// Design (one persistent CTA per SM, 384 threads = 12 warps, 128 x BN output
-// tiles).  Warp roles, plain layout (split layout in brackets, see Layout):
+// Two kernels share one thread layout (384 threads = 12 warps):
 //   warp 0      A producer: lane 0 issues, per K-block, the TMA load of the
-//               128x128 A tile (E4M3, 128-byte swizzle) into a ring of
-//               shared-memory stages and arms the stage barrier with the
-//               bytes of both tiles.
-//   warp 11 [3] B producer: the BNx128 B tile of the same stage.
-//   warp 10 [2] scale producer: per K-block the tile's 128 per-row A scales
-//               (and, for WGRAD, the BN per-column B scales) by TMA bulk
-//               copies into an 8-deep scale ring; FWD/DGRAD's per-block B
-//               scales are read 32 K-blocks at a time and handed out by
-//               shuffle.  No global load sits on the promotion path.
+//               A tile (E4M3, 128-byte swizzle) into a ring of shared-memory
+//               stages and arms the stage barrier with the bytes of both tiles.
 //   warp 1      TMEM owner and MMA issuer: the whole warp runs the loop, one
-//               elected lane issues 4 x tcgen05.mma kind::f8f6f4 (M=128,
-//               N=BN, K=32) per K-block into one of two TMEM accumulators
-//               (2 x BN fp32 columns), then tcgen05.commit to release the
-//               smem stage and to signal the accumulator.
-//   warps 2..9 [4..11]  promotion + epilogue: two warpgroups' worth of warps,
-//               each half owning BN/2 columns of the tile (a warp reads the
-//               32 TMEM lanes given by its index mod 4); per K-block they read
-//               the partial product from TMEM and fold it into fp32 registers
-//               with packed f32x2 FMAs,
+//               elected lane issues 4 x tcgen05.mma kind::f8f6f4 (K = 32) per
+//               K-block into one of the TMEM accumulators, then tcgen05.commit
+//               to release the smem stage and to signal the accumulator.
+//   warp 2      scale producer: per K-block the tile's 128 per-row A scales
+//               (and, for WGRAD, the per-column B scales) by TMA bulk copies
+//               into an 8-deep scale ring; FWD/DGRAD's per-block B scales are
+//               read 32 K-blocks at a time and handed out by shuffle.
+//   warp 3      B producer: the B tile of the same stage.
+//   warps 4-11  promotion + epilogue, two warpgroups each owning half of the
+//               tile's columns (a warp reads the 32 TMEM lanes its index mod 4
+//               allows).  Warpgroup 0 hands registers to them (setmaxnreg
+//               80 / 208), which pays for 64-column TMEM loads next to the
+//               128 fp32 running sums of a thread.  Per K-block a warp takes
+//               its scales from the ring, waits for the accumulator, reads it
+//               from TMEM in two 64-column loads, hands the buffer back to the
+//               MMA issuer as soon as the last load has landed, and folds the
+//               partial product into its registers with packed f32x2 FMAs:
 //                   FWD/DGRAD: acc += P * (sa[m] * sb[n-block])
 //                   WGRAD    : acc += (P * sb[n]) * sa[m]
-//               handing the TMEM buffer back as soon as its last load has
-//               landed (before those FMAs) and the scale slot after them;
-//               after the last K-block they round the tile to bf16 and store
-//               it with 32-byte vector stores.  In the split layout warpgroup
-//               0 (warps 0-3) hands registers to the promotion warps with
-//               setmaxnreg, which pays for 64-column TMEM loads.
-// The MMA of K-block kb+1 runs while the promotion of kb is in flight
-// (double-buffered TMEM), and TMA runs up to kStages K-blocks ahead.
+//               after the last K-block it rounds the tile to bf16 and stores
+//               it with 32-byte vector stores.
+// Waits on the critical path (MMA issuer, promotion) poll without a
+// suspend-time hint; the producers, which run ahead, sleep in theirs.
+//
+// gemm_blockwise_kernel: one CTA per SM, 128 x BN tiles (BN = 256 or 128),
+// double-buffered TMEM (2 x 256 or 4 x 128 columns).
+// gemm_pair_kernel: a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256): each CTA loads its own 128 A rows and
+// half of the 256 B rows, so a K-block moves 32 KB into each SM instead of
+// 48 KB, and the MMAs of both SMs are issued by the leader CTA alone.
 //
 // Every mbarrier wait is bounded (see mbar_wait_bounded): on a timeout the
-// CTA raises its abort flag, each role leaves its loop, the producer waits
-// for its TMA loads in flight, the issuer waits for its MMAs, and the TMEM
+// CTA raises its abort flag, each role leaves its loop, the producers wait
+// for their TMA loads in flight, the issuer waits for its MMAs, and the TMEM
 // is freed before the CTA exits.  Decisions that a whole warp must take
 // together (tcgen05.ld is warp-collective) are made warp-uniform.
 #include <cuda_bf16.h>
@@ -53,6 +56,7 @@
 
 #include <cstddef>
 
+#include "context.h"
 #include "device.cuh"
 #include "kernels.h"
 
@@ -62,41 +66,20 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 128;
-constexpr int kEpiWarps = 8;
+constexpr int kThreads = 384;
+constexpr int kPromoWarps = 8;
+constexpr int kPromoWarp0 = 4;
+constexpr int kScaleWarp = 2;
+constexpr int kBWarp = 3;
 constexpr int kSRing = 8;        // scale ring depth (K-blocks)
-// Two thread layouts, 384 threads each.  Plain: A-operand producer, MMA
-// issuer, 8 promotion warps, scale producer, B-operand producer.  Split:
-// warpgroup 0 (A producer, MMA issuer, scale producer, B producer) hands
-// registers to the two promotion warpgroups with setmaxnreg, which pays for
-// double-buffered TMEM reads.  The launch allocates 168 per thread (ptxas
-// pins it when setmaxnreg is used).
-// Two operand producers: one thread's stream of TMA box loads completes
-// about one box per ~350 cycles whatever the box size (measured on B200:
-// 16 KB boxes 46 B/clk per issuing thread, two issuing warps 76 B/clk), so
-// A and B tiles are issued by different warps.  The scale producer runs
-// ahead of the operand ring by up to the scale ring's depth.
-// Quad layout (kQuad, split layout only): 20 warps, warpgroup 0 as in the
-// split layout and 16 promotion warps, four per TMEM lane quadrant, each
-// owning BN/4 columns; the launch allocates 96 registers per thread, and
-// setmaxnreg gives warpgroup 0 64 and the promotion warps 104.
-constexpr int kLowRegs = 56;
-constexpr int kHighRegs = 224;
-static_assert(128 * kLowRegs + 256 * kHighRegs == 384 * 168, "register split must match the launch allocation");
-constexpr int kQuadLowRegs = 64;
-constexpr int kQuadHighRegs = 104;
-static_assert(128 * kQuadLowRegs + 512 * kQuadHighRegs == 640 * 96, "quad register split must match 96 per thread");
-template <bool kSplit, bool kQuad = false>
-struct Layout {
-  static_assert(!kQuad || kSplit, "the quad layout is a split layout");
-  static constexpr int kThreads = kQuad ? 640 : 384;
-  static constexpr int kPromoWarps = kQuad ? 16 : 8;
-  static constexpr int kEpiWarp0 = kSplit ? 4 : 2;
-  static constexpr int kScaleWarp = kSplit ? 2 : 10;
-  static constexpr int kBWarp = kSplit ? 3 : 11;
-  static constexpr int kLow = kQuad ? kQuadLowRegs : kLowRegs;
-  static constexpr int kHigh = kQuad ? kQuadHighRegs : kHighRegs;
-  static_assert(kLow % 8 == 0 && kHigh % 8 == 0, "setmaxnreg takes multiples of 8");
-};
+// Register split: warpgroup 0 (producers, MMA issuer) drops to kLowRegs and
+// the two promotion warpgroups rise to kHighRegs; the launch allocates 168
+// per thread (ptxas pins it when setmaxnreg is used), and the split must not
+// exceed what the launch holds.
+constexpr int kLowRegs = 80;
+constexpr int kHighRegs = 208;
+static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * 168, "register split exceeds the launch allocation");
+static_assert(kLowRegs % 8 == 0 && kHighRegs % 8 == 0, "setmaxnreg takes multiples of 8");
 
 template <int BN>
 struct Cfg {
@@ -104,8 +87,7 @@ struct Cfg {
   static constexpr int kABytes = BM * BK;
   static constexpr int kBBytes = BN * BK;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  // TMEM accumulators: 2 x 256 columns for BN=256; 4 x 128 for BN=128, so
-  // that the MMA can run three K-blocks ahead of the promotion.
+  // TMEM accumulators: 2 x 256 columns for BN=256; 4 x 128 for BN=128.
   static constexpr int kAccBufs = (BN == 256) ? 2 : 4;
   static constexpr int kTmemCols = kAccBufs * BN;
 };
@@ -213,7 +195,7 @@ __device__ __forceinline__ void tmem_wait_ld64(uint32_t (&r)[64]) {
 //   FWD/DGRAD: acc += P * f           (f = sa[m] * sb[n-block])
 //   WGRAD    : acc += (P * sb[n]) * sa[m]
 template <bool kWgrad>
-__device__ __forceinline__ void promote16(float2* acc, const uint32_t (&r)[16], float f, const float* sbc, float sa) {
+__device__ __forceinline__ void promote16(float2* acc, const uint32_t* r, float f, const float* sbc, float sa) {
   const float2 f2 = make_float2(f, f), sa2 = make_float2(sa, sa);
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -231,6 +213,83 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&v)[8]) {
                : "memory");
 }
 
+// Rounds kCols fp32 sums of one row to bf16 and stores them (32-byte stores).
+template <int kCols>
+__device__ __forceinline__ void store_row_bf16(uint16_t* drow, const float2* acc) {
+#pragma unroll
+  for (int j = 0; j < kCols; j += 16) {
+    uint32_t v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v[q] = pack_bf16x2(acc[j / 2 + q].x, acc[j / 2 + q].y);
+    st_global_v8(drow + j, v);
+  }
+}
+
+// Ring position: an index into a ring of N slots and the parity of its use.
+template <int N>
+struct Ring {
+  int idx = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void next() {
+    if (++idx == N) {
+      idx = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+// One promotion warp's K loop over one output tile: its 32 TMEM lanes (rows)
+// times kCols = BN/2 columns starting at col0.  `release(buf)` hands TMEM
+// buffer buf back to the MMA issuer.  Returns false when a wait gave up.
+template <int BN, bool kWgrad, typename Release>
+__device__ __forceinline__ bool promote_tile(Ctrl* ctrl, const GemmParams& p, float2 (&acc)[BN / 4], int kblocks,
+                                             uint32_t tmem_lanes, int row, int col0, Ring<Cfg<BN>::kAccBufs>& tbuf,
+                                             Ring<kSRing>& sring, volatile int* abort, int lane, Release release) {
+  constexpr int kCols = BN / 2;
+#pragma unroll
+  for (int j = 0; j < kCols / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
+  for (int kb = 0; kb < kblocks; ++kb) {
+    // The scale producer runs up to kSRing K-blocks ahead: this wait normally
+    // finds the slot filled, and the scales are in registers before the
+    // accumulator arrives.
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded<false>(&ctrl->sfull[sring.idx], sring.phase, abort,
+                                                          p.timeout_ns, p.err)))
+      return false;
+    const ScaleSlot& ss = ctrl->slots[sring.idx];
+    const float sa = ss.sa[row];
+    float f = 0.0f;
+    if constexpr (!kWgrad) {
+      f = sa * ss.sb[col0 / 128];          // the column slice's n-block
+      __syncwarp();                        // every lane has its scales: the slot can be refilled
+      if (lane == 0) mbar_arrive(&ctrl->sempty[sring.idx]);
+    }
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded<false>(&ctrl->tfull[tbuf.idx], tbuf.phase, abort, p.timeout_ns,
+                                                          p.err)))
+      return false;
+    tc_fence_after_sync();
+    const uint32_t taddr = tmem_lanes + tbuf.idx * BN;
+    const float* sbc = ss.sb + col0;
+#pragma unroll
+    for (int c = 0; c < kCols; c += 64) {
+      uint32_t r[64];
+      tmem_ld_32x32b_x64(taddr + c, r);
+      tmem_wait_ld64(r);
+      // The buffer goes back to the MMA issuer as soon as this warp's last
+      // TMEM load has landed, before the FMAs that consume it.
+      if (c + 64 == kCols) release(tbuf.idx);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) promote16<kWgrad>(acc + c / 2 + 8 * q, r + 16 * q, f, sbc + c + 16 * q, sa);
+    }
+    if constexpr (kWgrad) {
+      __syncwarp();                        // the column scales were read during the FMAs
+      if (lane == 0) mbar_arrive(&ctrl->sempty[sring.idx]);
+    }
+    tbuf.next();
+    sring.next();
+  }
+  return true;
+}
+
 }  // namespace
 
 // Scale producer (one warp): fills the scale ring, up to kSRing K-blocks ahead
@@ -242,8 +301,7 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&v)[8]) {
 template <int BN, bool kWgrad, typename Coords>
 __device__ __forceinline__ void scale_feed(Ctrl* ctrl, const GemmParams& p, int first_tile, int tile_step, int tiles,
                                            int kblocks, Coords coords, volatile int* abort, int lane) {
-  int slot = 0;
-  uint32_t sphase = 0;
+  Ring<kSRing> ring;
   int64_t issued = 0;
   bool ok = true;
   [[maybe_unused]] float sb0 = 0.0f, sb1 = 0.0f;   // FWD/DGRAD: B scales of K-blocks (kb & ~31) + lane
@@ -259,11 +317,12 @@ __device__ __forceinline__ void scale_feed(Ctrl* ctrl, const GemmParams& p, int 
           if constexpr (BN == 256) sb1 = k < kblocks ? __ldg(row + kblocks + k) : 0.0f;
         }
       }
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&ctrl->sempty[slot], sphase ^ 1u, abort, p.timeout_ns, p.err))) {
+      if (!__all_sync(0xFFFFFFFFu,
+                      mbar_wait_bounded(&ctrl->sempty[ring.idx], ring.phase ^ 1u, abort, p.timeout_ns, p.err))) {
         ok = false;
         break;
       }
-      ScaleSlot& ss = ctrl->slots[slot];
+      ScaleSlot& ss = ctrl->slots[ring.idx];
       if constexpr (!kWgrad) {
         const float v0 = __shfl_sync(0xFFFFFFFFu, sb0, kb & 31);
         const float v1 = __shfl_sync(0xFFFFFFFFu, sb1, kb & 31);
@@ -277,15 +336,13 @@ __device__ __forceinline__ void scale_feed(Ctrl* ctrl, const GemmParams& p, int 
         // bulk copies below write it through the async proxy: order them.
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         constexpr uint32_t kBytes = BM * 4 + (kWgrad ? BN * 4 : 0);
-        mbar_arrive_expect_tx(&ctrl->sfull[slot], kBytes);   // releases the sb stores above
-        bulk_load(ss.sa, p.sa + static_cast<int64_t>(kb) * p.M + m0, BM * 4, &ctrl->sfull[slot]);
-        if constexpr (kWgrad) bulk_load(ss.sb, p.sb + static_cast<int64_t>(kb) * p.N + n0, BN * 4, &ctrl->sfull[slot]);
+        mbar_arrive_expect_tx(&ctrl->sfull[ring.idx], kBytes);   // releases the sb stores above
+        bulk_load(ss.sa, p.sa + static_cast<int64_t>(kb) * p.M + m0, BM * 4, &ctrl->sfull[ring.idx]);
+        if constexpr (kWgrad)
+          bulk_load(ss.sb, p.sb + static_cast<int64_t>(kb) * p.N + n0, BN * 4, &ctrl->sfull[ring.idx]);
       }
       ++issued;
-      if (++slot == kSRing) {
-        slot = 0;
-        sphase ^= 1u;
-      }
+      ring.next();
     }
   }
   // Let the copies still in flight land before the CTA's smem goes away (on
@@ -312,19 +369,12 @@ __device__ __forceinline__ void tile_coords(int tile, int num_mb, int num_nb, in
 // kTensor: one scale per operand (per-tensor scaling).  No per-K-block
 // promotion: the MMAs accumulate the whole K loop of a tile in TMEM and the
 // promotion warps only apply sa * sb, round to bf16 and store, once per tile.
-template <int BN, bool kWgrad, bool kSplit, bool kTensor = false, bool kQuad = false>
-__global__ void __launch_bounds__(Layout<kSplit, kQuad>::kThreads, 1)
+template <int BN, bool kWgrad, bool kTensor = false>
+__global__ void __launch_bounds__(kThreads, 1)
     gemm_blockwise_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const GemmParams p) {
   using C = Cfg<BN>;
-  using L = Layout<kSplit, kQuad>;
-  constexpr int kEpiWarp0 = L::kEpiWarp0;
-  constexpr int kPromo = L::kPromoWarps;
-  constexpr int kCols = BN / (kPromo / 4);   // columns per promotion warp
-  // The split layout has the registers for 64-column TMEM reads; the quad
-  // layout's promotion warps read their columns 16 at a time.
-  constexpr bool kTmemDB = kSplit && !kQuad;
-  constexpr bool kWide = kSplit && !kQuad;
+  constexpr int kCols = BN / 2;   // columns per promotion warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + C::kStages * C::kStageBytes);
@@ -343,11 +393,11 @@ __global__ void __launch_bounds__(Layout<kSplit, kQuad>::kThreads, 1)
     }
     for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&ctrl->tfull[b], 1);
-      mbar_init(&ctrl->tempty[b], kPromo);
+      mbar_init(&ctrl->tempty[b], kPromoWarps);
     }
     for (int s = 0; s < kSRing; ++s) {
       mbar_init(&ctrl->sfull[s], 1);    // the scale producer's arrive + the bytes of its copies
-      mbar_init(&ctrl->sempty[s], kPromo);
+      mbar_init(&ctrl->sempty[s], kPromoWarps);
     }
     mbar_init(&ctrl->mma_done, 1);
     mbar_init(&ctrl->never, 1);
@@ -368,150 +418,135 @@ __global__ void __launch_bounds__(Layout<kSplit, kQuad>::kThreads, 1)
   const uint32_t tmem_base = ctrl->tmem_base;
   volatile int* abort = &ctrl->abort;
 
-  if (warp < kEpiWarp0 || warp >= kEpiWarp0 + kPromo) {
-  if constexpr (kSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(L::kLow));
-  if (warp == 0 || warp == L::kBWarp) {
-    // ------------------------------------------------------------ operand producers (A: warp 0, B: kBWarp)
-    // Both wait for the same free stage; the A producer arms the stage's full
-    // barrier with the bytes of both tiles (the B bytes may land first: the
-    // transaction count may go negative until the arrival).
-    const bool is_a = warp == 0;
-    if (lane == 0) {
-      tma_prefetch_map(is_a ? &tm_a : &tm_b);
-      int stage = 0;
-      uint32_t phase = 0;
-      int64_t issued = 0;
+  if (warp < kPromoWarp0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
+    if (warp == 0 || warp == kBWarp) {
+      // ---------------------------------------------------------- operand producers (A: warp 0, B: warp 3)
+      // Both wait for the same free stage; the A producer arms the stage's full
+      // barrier with the bytes of both tiles (the B bytes may land first: the
+      // transaction count may go negative until the arrival).
+      const bool is_a = warp == 0;
+      if (lane == 0) {
+        tma_prefetch_map(is_a ? &tm_a : &tm_b);
+        Ring<C::kStages> st;
+        int64_t issued = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+          int mb, nb;
+          tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
+          for (int kb = 0; kb < kblocks; ++kb) {
+            if (!mbar_wait_bounded(&ctrl->empty[st.idx], st.phase ^ 1u, abort, p.timeout_ns, p.err)) {
+              ok = false;
+              break;
+            }
+            uint8_t* stage = smem + st.idx * C::kStageBytes;
+            if (is_a) {
+              mbar_arrive_expect_tx(&ctrl->full[st.idx], C::kStageBytes);
+              tma_load_2d(stage, &tm_a, &ctrl->full[st.idx], kb * BK, mb * BM);
+            } else {
+              tma_load_2d(stage + C::kABytes, &tm_b, &ctrl->full[st.idx], kb * BK, nb * BN);
+            }
+            ++issued;
+            st.next();
+          }
+        }
+        // Let the copies still in flight land before the CTA's smem goes away
+        // (on the normal path they have all been consumed: no wait).
+        const int64_t first = issued > C::kStages ? issued - C::kStages : 0;
+        for (int64_t j = first; j < issued; ++j)
+          mbar_wait_bounded(&ctrl->full[j % C::kStages], static_cast<uint32_t>((j / C::kStages) & 1), nullptr,
+                            p.timeout_ns, p.err);
+      }
+    } else if (warp == kScaleWarp) {
+      // ---------------------------------------------------------- scale producer (whole warp)
+      if constexpr (!kTensor)
+        scale_feed<BN, kWgrad>(ctrl, p, blockIdx.x, gridDim.x, tiles, kblocks,
+                               [&](int tile, int64_t& m0, int64_t& n0) {
+                                 int mb, nb;
+                                 tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
+                                 m0 = static_cast<int64_t>(mb) * BM;
+                                 n0 = static_cast<int64_t>(nb) * BN;
+                               },
+                               abort, lane);
+    } else {
+      // ---------------------------------------------------------- MMA issuer (warp 1)
+      // The whole warp runs the loop and waits, so the stage addresses,
+      // descriptors and counters are warp-uniform and reach tcgen05.mma from
+      // uniform registers; one elected lane issues the MMAs and the commits.
+      const bool leader = elect_one();
+      const uint32_t idesc = idesc_e4m3_f32(BM, BN) | p.fmt_bits;
+      const uint32_t smem0 = smem_addr(smem);
+      Ring<C::kStages> st;
+      Ring<C::kAccBufs> acc;
       bool ok = true;
+      if (p.inject_stall) ok = mbar_wait_bounded(&ctrl->never, 0, abort, p.timeout_ns, p.err);
+      ok = __all_sync(0xFFFFFFFFu, ok);
       for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-        int mb, nb;
-        tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded(&ctrl->empty[stage], phase ^ 1u, abort, p.timeout_ns, p.err)) {
+        if constexpr (kTensor) {   // one accumulator buffer per tile
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded<false>(&ctrl->tempty[acc.idx], acc.phase ^ 1u, abort,
+                                                                p.timeout_ns, p.err))) {
             ok = false;
             break;
           }
-          uint8_t* st = smem + stage * C::kStageBytes;
-          if (is_a) {
-            mbar_arrive_expect_tx(&ctrl->full[stage], C::kStageBytes);
-            tma_load_2d(st, &tm_a, &ctrl->full[stage], kb * BK, mb * BM);
-          } else {
-            tma_load_2d(st + C::kABytes, &tm_b, &ctrl->full[stage], kb * BK, nb * BN);
+        }
+        for (int kb = 0; kb < kblocks; ++kb) {
+          const bool got =
+              mbar_wait_bounded<false>(&ctrl->full[st.idx], st.phase, abort, p.timeout_ns, p.err) &&
+              (kTensor || mbar_wait_bounded<false>(&ctrl->tempty[acc.idx], acc.phase ^ 1u, abort, p.timeout_ns, p.err));
+          if (!__all_sync(0xFFFFFFFFu, got)) {
+            ok = false;
+            break;
           }
-          ++issued;
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      // Let the copies still in flight land before the CTA's smem goes away
-      // (on the normal path they have all been consumed: no wait).
-      const int64_t first = issued > C::kStages ? issued - C::kStages : 0;
-      for (int64_t j = first; j < issued; ++j)
-        mbar_wait_bounded(&ctrl->full[j % C::kStages], static_cast<uint32_t>((j / C::kStages) & 1), nullptr,
-                          p.timeout_ns, p.err);
-    }
-  } else if (warp == L::kScaleWarp) {
-    // ------------------------------------------------------------ scale producer (whole warp)
-    if constexpr (!kTensor)
-      scale_feed<BN, kWgrad>(ctrl, p, blockIdx.x, gridDim.x, tiles, kblocks,
-                           [&](int tile, int64_t& m0, int64_t& n0) {
-                             int mb, nb;
-                             tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
-                             m0 = static_cast<int64_t>(mb) * BM;
-                             n0 = static_cast<int64_t>(nb) * BN;
-                           },
-                           abort, lane);
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // The whole warp runs the loop and waits, so the stage addresses,
-    // descriptors and counters are warp-uniform and reach tcgen05.mma from
-    // uniform registers; one elected lane issues the MMAs and the commits.
-    // (Run by a single lane, every MMA and commit paid a move of its operands
-    // into uniform registers: 70-100 cycles each, measured on B200, which
-    // put ~500 cycles of issue latency into every K-block.)
-    const bool leader = elect_one();
-    const uint32_t idesc = idesc_e4m3_f32(BM, BN) | p.fmt_bits;
-    int stage = 0;
-    uint32_t phase = 0, abuf = 0, aphase = 0;
-    bool ok = true;
-    if (p.inject_stall) ok = mbar_wait_bounded(&ctrl->never, 0, abort, p.timeout_ns, p.err);
-    ok = __all_sync(0xFFFFFFFFu, ok);
-    for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-      if constexpr (kTensor) {   // one accumulator buffer per tile
-        if (!__all_sync(0xFFFFFFFFu,
-                        mbar_wait_bounded(&ctrl->tempty[abuf], aphase ^ 1u, abort, p.timeout_ns, p.err))) {
-          ok = false;
-          break;
-        }
-      }
-      for (int kb = 0; kb < kblocks; ++kb) {
-        const bool got = mbar_wait_bounded(&ctrl->full[stage], phase, abort, p.timeout_ns, p.err) &&
-                         (kTensor || mbar_wait_bounded(&ctrl->tempty[abuf], aphase ^ 1u, abort, p.timeout_ns, p.err));
-        if (!__all_sync(0xFFFFFFFFu, got)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-        const uint32_t a_addr = smem_addr(smem + stage * C::kStageBytes);
-        const uint64_t adesc = smem_desc_kmajor_sw128(a_addr);
-        const uint64_t bdesc = smem_desc_kmajor_sw128(a_addr + C::kABytes);
-        const uint32_t d_tmem = tmem_base + abuf * BN;
-        if (leader) {
+          tc_fence_after_sync();
+          const uint32_t a_addr = smem0 + st.idx * C::kStageBytes;
+          const uint64_t adesc = smem_desc_kmajor_sw128(a_addr);
+          const uint64_t bdesc = smem_desc_kmajor_sw128(a_addr + C::kABytes);
+          const uint32_t d_tmem = tmem_base + acc.idx * BN;
+          if (leader) {
+            umma_e4m3(d_tmem, adesc, bdesc, idesc, (kTensor && kb > 0) ? 1u : 0u);
 #pragma unroll
-          for (int k = 0; k < BK / 32; ++k)  // 32 E4M3 values = 32 bytes = 2 x 16 B per step
-            umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (k > 0 || (kTensor && kb > 0)) ? 1u : 0u);
-          umma_commit(&ctrl->empty[stage]);
-          if constexpr (!kTensor) umma_commit(&ctrl->tfull[abuf]);
-        }
-        __syncwarp();
-        if (++stage == C::kStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
-        if constexpr (!kTensor) {
-          if (++abuf == C::kAccBufs) {
-            abuf = 0;
-            aphase ^= 1u;
+            for (int k = 1; k < BK / 32; ++k)  // 32 E4M3 values = 32 bytes = 2 x 16 B per step
+              umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, 1u);
+            umma_commit(&ctrl->empty[st.idx]);
+            if constexpr (!kTensor) umma_commit(&ctrl->tfull[acc.idx]);
           }
+          __syncwarp();
+          st.next();
+          if constexpr (!kTensor) acc.next();
+        }
+        if constexpr (kTensor) {
+          if (!ok) break;
+          if (leader) umma_commit(&ctrl->tfull[acc.idx]);   // the tile's whole K loop is in this buffer
+          __syncwarp();
+          acc.next();
         }
       }
-      if constexpr (kTensor) {
-        if (!ok) break;
-        if (leader) umma_commit(&ctrl->tfull[abuf]);   // the tile's whole K loop is in this buffer
-        __syncwarp();
-        if (++abuf == C::kAccBufs) {
-          abuf = 0;
-          aphase ^= 1u;
-        }
-      }
+      // Every MMA issued so far has finished once this arrives.
+      if (leader) umma_commit(&ctrl->mma_done);
+      __syncwarp();
+      mbar_wait_bounded(&ctrl->mma_done, 0, nullptr, p.timeout_ns, p.err);
     }
-    // Every MMA issued so far has finished once this arrives.
-    if (leader) umma_commit(&ctrl->mma_done);
-    __syncwarp();
-    mbar_wait_bounded(&ctrl->mma_done, 0, nullptr, p.timeout_ns, p.err);
-  }
   } else {
-    if constexpr (kSplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(L::kHigh));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
     // ------------------------------------------------------------ promotion + epilogue
-    const int ew = warp - kEpiWarp0;  // 0 .. kPromo - 1
-    const int wg = ew >> 2;           // which slice of the tile's columns
-    const int quarter = warp & 3;     // TMEM lanes this warp may read
+    const int ew = warp - kPromoWarp0;  // 0 .. 7
+    const int wg = ew >> 2;             // which half of the tile's columns
+    const int quarter = warp & 3;       // TMEM lanes this warp may read
     const int row = quarter * 32 + lane;
     const int col0 = wg * kCols;
-    uint32_t abuf = 0, aphase = 0, sphase = 0;
-    int slot = 0;
-    bool ok = true;
+    const uint32_t tmem_lanes = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + col0;
+    Ring<C::kAccBufs> tbuf;
     if constexpr (kTensor) {
       // ---------------------------------------------------------- per-tensor epilogue
       const float f = *p.tsa * *p.tsb;
       for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
         int mb, nb;
         tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&ctrl->tfull[abuf], aphase, abort, p.timeout_ns, p.err)))
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded<false>(&ctrl->tfull[tbuf.idx], tbuf.phase, abort,
+                                                              p.timeout_ns, p.err)))
           break;
         tc_fence_after_sync();
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * BN + col0;
+        const uint32_t taddr = tmem_lanes + tbuf.idx * BN;
         uint16_t* drow = p.d + (static_cast<int64_t>(mb) * BM + row) * p.ldd + static_cast<int64_t>(nb) * BN + col0;
 #pragma unroll
         for (int c = 0; c < kCols; c += 16) {
@@ -526,118 +561,25 @@ __global__ void __launch_bounds__(Layout<kSplit, kQuad>::kThreads, 1)
         }
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ctrl->tempty[abuf]);
-        if (++abuf == C::kAccBufs) {
-          abuf = 0;
-          aphase ^= 1u;
-        }
+        if (lane == 0) mbar_arrive(&ctrl->tempty[tbuf.idx]);
+        tbuf.next();
       }
-      ok = false;   // skip the blockwise loop below
-    }
-    float2 acc[kCols / 2];
-    for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-      int mb, nb;
-      tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
-      const int64_t m = static_cast<int64_t>(mb) * BM + row;
-      const int64_t ncol0 = static_cast<int64_t>(nb) * BN + col0;
-#pragma unroll
-      for (int j = 0; j < kCols / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
-
-      for (int kb = 0; kb < kblocks; ++kb) {
-        const bool got = mbar_wait_bounded(&ctrl->sfull[slot], sphase, abort, p.timeout_ns, p.err) &&
-                         mbar_wait_bounded(&ctrl->tfull[abuf], aphase, abort, p.timeout_ns, p.err);
-        if (!__all_sync(0xFFFFFFFFu, got)) {
-          ok = false;
+    } else {
+      Ring<kSRing> sring;
+      float2 acc[BN / 4];
+      auto release = [&](int b) {
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->tempty[b]);
+      };
+      for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
+        if (!promote_tile<BN, kWgrad>(ctrl, p, acc, kblocks, tmem_lanes, row, col0, tbuf, sring, abort, lane,
+                                      release))
           break;
-        }
-        tc_fence_after_sync();
-        const ScaleSlot& ss = ctrl->slots[slot];
-        const float sa = ss.sa[row];
-        const float f = kWgrad ? 0.0f : sa * ss.sb[col0 / 128];   // the column slice's n-block
-        const float* sbc = ss.sb + col0;
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * BN + col0;
-        // The accumulator buffer goes back to the MMA issuer as soon as this
-        // warp's last TMEM load has landed in registers, before the FMAs that
-        // consume it: the next K-block's MMAs into this buffer wait only for
-        // the reads, not for the arithmetic.
-        auto release_tmem = [&]() {
-          tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ctrl->tempty[abuf]);
-        };
-        if constexpr (kCols == 64 && !kQuad) {
-          // 64 columns per thread: all four loads in flight, one wait.
-          uint32_t r0[16], r1[16], r2[16], r3[16];
-          tmem_ld_32x32b_x16(taddr, r0);
-          tmem_ld_32x32b_x16(taddr + 16, r1);
-          tmem_ld_32x32b_x16(taddr + 32, r2);
-          tmem_ld_32x32b_x16(taddr + 48, r3);
-          tmem_wait_ld16(r0);
-          tmem_wait_ld16(r1);
-          tmem_wait_ld16(r2);
-          tmem_wait_ld16(r3);
-          release_tmem();
-          promote16<kWgrad>(acc, r0, f, sbc, sa);
-          promote16<kWgrad>(acc + 8, r1, f, sbc + 16, sa);
-          promote16<kWgrad>(acc + 16, r2, f, sbc + 32, sa);
-          promote16<kWgrad>(acc + 24, r3, f, sbc + 48, sa);
-        } else if constexpr (kTmemDB && kWide) {
-          // 64-column loads: two TMEM round trips per K-block for 128 columns.
-#pragma unroll
-          for (int c = 0; c < kCols; c += 64) {
-            uint32_t r[64];
-            tmem_ld_32x32b_x64(taddr + c, r);
-            tmem_wait_ld64(r);
-            if (c + 64 == kCols) release_tmem();
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              promote16<kWgrad>(acc + c / 2 + 8 * q, *reinterpret_cast<const uint32_t(*)[16]>(r + 16 * q), f,
-                                sbc + c + 16 * q, sa);
-          }
-        } else if constexpr (kTmemDB) {
-          // Two 16-column buffers: the load of the next chunk overlaps the FMAs of this one.
-          uint32_t ra[16], rb[16];
-          tmem_ld_32x32b_x16(taddr, ra);
-          tmem_wait_ld16(ra);
-#pragma unroll
-          for (int c = 0; c < kCols; c += 32) {
-            tmem_ld_32x32b_x16(taddr + c + 16, rb);
-            promote16<kWgrad>(acc + c / 2, ra, f, sbc + c, sa);
-            tmem_wait_ld16(rb);
-            if (c + 32 == kCols) release_tmem();
-            if (c + 32 < kCols) tmem_ld_32x32b_x16(taddr + c + 32, ra);
-            promote16<kWgrad>(acc + c / 2 + 8, rb, f, sbc + c + 16, sa);
-            if (c + 32 < kCols) tmem_wait_ld16(ra);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < kCols; c += 16) {
-            uint32_t r[16];
-            tmem_ld_32x32b_x16(taddr + c, r);
-            tmem_wait_ld16(r);
-            if (c + 16 == kCols) release_tmem();
-            promote16<kWgrad>(acc + c / 2, r, f, sbc + c, sa);
-          }
-        }
-        __syncwarp();   // every lane has read its scales from the slot
-        if (lane == 0) mbar_arrive(&ctrl->sempty[slot]);
-        if (++abuf == C::kAccBufs) {
-          abuf = 0;
-          aphase ^= 1u;
-        }
-        if (++slot == kSRing) {
-          slot = 0;
-          sphase ^= 1u;
-        }
-      }
-      if (!ok) break;
-      uint16_t* drow = p.d + m * p.ldd + ncol0;
-#pragma unroll
-      for (int j = 0; j < kCols; j += 16) {
-        uint32_t v[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = pack_bf16x2(acc[j / 2 + q].x, acc[j / 2 + q].y);
-        st_global_v8(drow + j, v);
+        const int64_t m = static_cast<int64_t>(mb) * BM + row;
+        store_row_bf16<kCols>(p.d + m * p.ldd + static_cast<int64_t>(nb) * BN + col0, acc);
       }
     }
   }
@@ -652,34 +594,32 @@ __global__ void __launch_bounds__(Layout<kSplit, kQuad>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Pair-tile variant: a cluster of two CTAs computes a 256 x 256 tile with
-// tcgen05.mma.cta_group::2 (M = 256).  Each CTA keeps the same roles as above
-// and owns 128 rows of the tile in its own TMEM; it TMA-loads its own 128 A
-// rows and its half of the tile's 256 B rows, so a K-block moves 32 KB into
-// each SM instead of 48 KB (operand traffic was the limit of the 128 x 256
-// tile).  The loads complete on the leader's "full" barrier; the leader alone
-// issues the MMAs and commits them to the stage and accumulator barriers of
-// both CTAs; both CTAs' promotion warps hand each accumulator buffer back to
-// the leader.  Scale rings stay local.  A timeout raises the abort flag of
-// both CTAs; the TMEM is freed after a cluster barrier, once every MMA of the
-// pair has completed.
+// Pair-tile kernel: a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256).  Each CTA keeps the roles above and owns
+// 128 rows of the tile in its own TMEM; it TMA-loads its own 128 A rows and
+// its half of the tile's 256 B rows.  The loads complete on the leader's
+// "full" barrier; the leader alone issues the MMAs and commits them to the
+// stage and accumulator barriers of both CTAs; both CTAs' promotion warps
+// hand each accumulator buffer back to the leader.  Scale rings stay local.
+// A timeout raises the abort flag of both CTAs; the TMEM is freed after a
+// cluster barrier, once every MMA of the pair has completed.
 namespace {
 constexpr int kPairStages = 6;
 constexpr int kPairHalfBytes = 128 * BK;              // own A rows, or own half of B
 constexpr int kPairStageBytes = 2 * kPairHalfBytes;
 constexpr int kPairBN = 256;
+constexpr int kPairAccBufs = 2;
 constexpr int pair_smem_bytes() { return 1024 + kPairStages * kPairStageBytes + static_cast<int>(sizeof(Ctrl)); }
 static_assert(kPairStages <= 8, "Ctrl holds 8 stage barriers");
+static_assert(Cfg<kPairBN>::kAccBufs == kPairAccBufs, "the pair promotes through Cfg<256>'s TMEM ring");
 }  // namespace
 
-template <bool kWgrad, bool kSplit>
-__global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
+template <bool kWgrad>
+__global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const GemmParams p) {
   constexpr int BN = kPairBN;
-  constexpr int kHalf = BN / 2;
-  constexpr int kEpiWarp0 = Layout<kSplit>::kEpiWarp0;
-  constexpr int kAccBufs = 2;
+  constexpr int kCols = BN / 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + kPairStages * kPairStageBytes);
@@ -699,13 +639,13 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
       mbar_init(&ctrl->full[s], 1);     // the leader's arrive + the bytes of both CTAs
       mbar_init(&ctrl->empty[s], 1);    // the leader's MMA commit
     }
-    for (int b = 0; b < kAccBufs; ++b) {
+    for (int b = 0; b < kPairAccBufs; ++b) {
       mbar_init(&ctrl->tfull[b], 1);
-      mbar_init(&ctrl->tempty[b], 2 * kEpiWarps);   // promotion warps of both CTAs
+      mbar_init(&ctrl->tempty[b], 2 * kPromoWarps);   // promotion warps of both CTAs
     }
     for (int s = 0; s < kSRing; ++s) {
       mbar_init(&ctrl->sfull[s], 1);
-      mbar_init(&ctrl->sempty[s], kEpiWarps);
+      mbar_init(&ctrl->sempty[s], kPromoWarps);
     }
     mbar_init(&ctrl->mma_done, 1);
     mbar_init(&ctrl->never, 1);
@@ -713,7 +653,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc_pair(&ctrl->tmem_base, kAccBufs * BN);
+    tmem_alloc_pair(&ctrl->tmem_base, kPairAccBufs * BN);
     tmem_relinquish_pair();
   }
   tc_fence_before_sync();
@@ -726,178 +666,128 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
   volatile int* abort = &ctrl->abort;
   const uint32_t peer_abort = mapa_shared(smem_addr(&ctrl->abort), rank ^ 1u);
 
-  if (warp < kEpiWarp0 || warp >= kEpiWarp0 + kEpiWarps) {
-  if constexpr (kSplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
-  if (warp == 0 || warp == Layout<kSplit>::kBWarp) {
-    // ------------------------------------------------------------ operand producers (A: warp 0, B half: kBWarp)
-    const bool is_a = warp == 0;
-    if (lane == 0) {
-      tma_prefetch_map(is_a ? &tm_a : &tm_b);
-      int stage = 0;
-      uint32_t phase = 0;
-      int64_t issued = 0;
-      bool ok = true;
-      for (int tile = pair; ok && tile < tiles; tile += npairs) {
-        const int mp = tile % num_mp, nb = tile / num_mp;
-        const int64_t m0 = static_cast<int64_t>(mp) * 2 * BM + rank * BM, n0 = static_cast<int64_t>(nb) * BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded_pair(&ctrl->empty[stage], phase ^ 1u, abort, peer_abort, p.timeout_ns, p.err)) {
-            ok = false;
-            break;
-          }
-          uint8_t* st = smem + stage * kPairStageBytes;
-          const uint32_t full_leader = mapa_shared(smem_addr(&ctrl->full[stage]), 0);
-          if (is_a) {
-            if (leader) mbar_arrive_expect_tx(&ctrl->full[stage], 2 * kPairStageBytes);
-            tma_load_2d_pair(st, &tm_a, full_leader, kb * BK, static_cast<int>(m0));
-          } else {
-            tma_load_2d_pair(st + kPairHalfBytes, &tm_b, full_leader, kb * BK, static_cast<int>(n0 + rank * BM));
-          }
-          ++issued;
-          if (++stage == kPairStages) {
-            stage = 0;
-            phase ^= 1u;
+  if (warp < kPromoWarp0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
+    if (warp == 0 || warp == kBWarp) {
+      // ---------------------------------------------------------- operand producers (A: warp 0, B half: warp 3)
+      const bool is_a = warp == 0;
+      if (lane == 0) {
+        tma_prefetch_map(is_a ? &tm_a : &tm_b);
+        Ring<kPairStages> st;
+        int64_t issued = 0;
+        bool ok = true;
+        for (int tile = pair; ok && tile < tiles; tile += npairs) {
+          const int mp = tile % num_mp, nb = tile / num_mp;
+          const int64_t m0 = static_cast<int64_t>(mp) * 2 * BM + rank * BM, n0 = static_cast<int64_t>(nb) * BN;
+          for (int kb = 0; kb < kblocks; ++kb) {
+            if (!mbar_wait_bounded_pair(&ctrl->empty[st.idx], st.phase ^ 1u, abort, peer_abort, p.timeout_ns, p.err)) {
+              ok = false;
+              break;
+            }
+            uint8_t* stage = smem + st.idx * kPairStageBytes;
+            const uint32_t full_leader = mapa_shared(smem_addr(&ctrl->full[st.idx]), 0);
+            if (is_a) {
+              if (leader) mbar_arrive_expect_tx(&ctrl->full[st.idx], 2 * kPairStageBytes);
+              tma_load_2d_pair(stage, &tm_a, full_leader, kb * BK, static_cast<int>(m0));
+            } else {
+              tma_load_2d_pair(stage + kPairHalfBytes, &tm_b, full_leader, kb * BK, static_cast<int>(n0 + rank * BM));
+            }
+            ++issued;
+            st.next();
           }
         }
+        if (leader) {
+          // The leader's full barriers count the bytes of both CTAs: once the last
+          // stages it armed are complete, no load of the pair is in flight.
+          const int64_t first = issued > kPairStages ? issued - kPairStages : 0;
+          for (int64_t j = first; j < issued; ++j)
+            mbar_wait_bounded(&ctrl->full[j % kPairStages], static_cast<uint32_t>((j / kPairStages) & 1), nullptr,
+                              p.timeout_ns, p.err);
+        }
       }
-      if (leader) {
-        // The leader's full barriers count the bytes of both CTAs: once the last
-        // stages it armed are complete, no load of the pair is in flight.
-        const int64_t first = issued > kPairStages ? issued - kPairStages : 0;
-        for (int64_t j = first; j < issued; ++j)
-          mbar_wait_bounded(&ctrl->full[j % kPairStages], static_cast<uint32_t>((j / kPairStages) & 1), nullptr,
-                            p.timeout_ns, p.err);
-      }
-    }
-  } else if (warp == Layout<kSplit>::kScaleWarp) {
-    // ------------------------------------------------------------ scale producer (whole warp)
-    scale_feed<BN, kWgrad>(ctrl, p, pair, npairs, tiles, kblocks,
-                           [&](int tile, int64_t& m0, int64_t& n0) {
-                             const int mp = tile % num_mp, nb = tile / num_mp;
-                             m0 = static_cast<int64_t>(mp) * 2 * BM + rank * BM;
-                             n0 = static_cast<int64_t>(nb) * BN;
-                           },
-                           abort, lane);
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (leader CTA only)
-    if (leader && lane == 0) {
+    } else if (warp == kScaleWarp) {
+      // ---------------------------------------------------------- scale producer (whole warp)
+      scale_feed<BN, kWgrad>(ctrl, p, pair, npairs, tiles, kblocks,
+                             [&](int tile, int64_t& m0, int64_t& n0) {
+                               const int mp = tile % num_mp, nb = tile / num_mp;
+                               m0 = static_cast<int64_t>(mp) * 2 * BM + rank * BM;
+                               n0 = static_cast<int64_t>(nb) * BN;
+                             },
+                             abort, lane);
+    } else if (leader) {
+      // ---------------------------------------------------------- MMA issuer (warp 1 of the leader CTA)
+      const bool issuer = elect_one();
       const uint32_t idesc = idesc_e4m3_f32(2 * BM, BN) | p.fmt_bits;
-      int stage = 0;
-      uint32_t phase = 0, abuf = 0, aphase = 0;
+      const uint32_t smem0 = smem_addr(smem);
+      Ring<kPairStages> st;
+      Ring<kPairAccBufs> acc;
       bool ok = true;
-      if (p.inject_stall)
-        ok = mbar_wait_bounded_pair(&ctrl->never, 0, abort, peer_abort, p.timeout_ns, p.err);
+      if (p.inject_stall) ok = mbar_wait_bounded_pair(&ctrl->never, 0, abort, peer_abort, p.timeout_ns, p.err);
+      ok = __all_sync(0xFFFFFFFFu, ok);
       for (int tile = pair; ok && tile < tiles; tile += npairs) {
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded_pair(&ctrl->full[stage], phase, abort, peer_abort, p.timeout_ns, p.err) ||
-              !mbar_wait_bounded_pair(&ctrl->tempty[abuf], aphase ^ 1u, abort, peer_abort, p.timeout_ns, p.err)) {
+          const bool got =
+              mbar_wait_bounded_pair<false>(&ctrl->full[st.idx], st.phase, abort, peer_abort, p.timeout_ns, p.err) &&
+              mbar_wait_bounded_pair<false>(&ctrl->tempty[acc.idx], acc.phase ^ 1u, abort, peer_abort, p.timeout_ns,
+                                            p.err);
+          if (!__all_sync(0xFFFFFFFFu, got)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t a_addr = smem_addr(smem + stage * kPairStageBytes);
+          const uint32_t a_addr = smem0 + st.idx * kPairStageBytes;
           const uint64_t adesc = smem_desc_kmajor_sw128(a_addr);
           const uint64_t bdesc = smem_desc_kmajor_sw128(a_addr + kPairHalfBytes);
-          const uint32_t d_tmem = tmem_base + abuf * BN;
+          const uint32_t d_tmem = tmem_base + acc.idx * BN;
+          if (issuer) {
+            umma_e4m3_pair(d_tmem, adesc, bdesc, idesc, 0u);
 #pragma unroll
-          for (int k = 0; k < BK / 32; ++k)
-            umma_e4m3_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
-          umma_commit_pair(&ctrl->empty[stage], 0x3);
-          umma_commit_pair(&ctrl->tfull[abuf], 0x3);
-          if (++stage == kPairStages) {
-            stage = 0;
-            phase ^= 1u;
+            for (int k = 1; k < BK / 32; ++k) umma_e4m3_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, 1u);
+            umma_commit_pair(&ctrl->empty[st.idx], 0x3);
+            umma_commit_pair(&ctrl->tfull[acc.idx], 0x3);
           }
-          if (++abuf == kAccBufs) {
-            abuf = 0;
-            aphase ^= 1u;
-          }
+          __syncwarp();
+          st.next();
+          acc.next();
         }
       }
-      umma_commit_pair(&ctrl->mma_done, 0x1);
+      if (issuer) umma_commit_pair(&ctrl->mma_done, 0x1);
+      __syncwarp();
       mbar_wait_bounded(&ctrl->mma_done, 0, nullptr, p.timeout_ns, p.err);
     }
-  }
   } else {
-    if constexpr (kSplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
     // ------------------------------------------------------------ promotion + epilogue
-    const int ew = warp - kEpiWarp0;  // 0..7
-    const int wg = ew >> 2;           // which half of the tile's columns
-    const int quarter = warp & 3;     // TMEM lanes this warp may read
+    const int ew = warp - kPromoWarp0;  // 0..7
+    const int wg = ew >> 2;             // which half of the tile's columns
+    const int quarter = warp & 3;       // TMEM lanes this warp may read
     const int row = quarter * 32 + lane;
-    const int col0 = wg * kHalf;
-    uint32_t abuf = 0, aphase = 0, sphase = 0;
-    int slot = 0;
-    float2 acc[kHalf / 2];
-    bool ok = true;
-    for (int tile = pair; ok && tile < tiles; tile += npairs) {
+    const int col0 = wg * kCols;
+    const uint32_t tmem_lanes = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + col0;
+    Ring<kPairAccBufs> tbuf;
+    Ring<kSRing> sring;
+    float2 acc[BN / 4];
+    // The accumulator hand-back goes to the leader, which issues the MMAs.  A
+    // CTA-scope release suffices for the peer's remote arrival: it publishes
+    // no data (the buffer's reads are ordered by tcgen05.wait::ld and
+    // tcgen05.fence::before_thread_sync), and a cluster-scope release would
+    // first wait for all of this thread's outstanding memory traffic.
+    auto release = [&](int b) {
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(&ctrl->tempty[b]);
+        else
+          mbar_arrive_remote(mapa_shared(smem_addr(&ctrl->tempty[b]), 0));
+      }
+    };
+    for (int tile = pair; tile < tiles; tile += npairs) {
       const int mp = tile % num_mp, nb = tile / num_mp;
+      if (!promote_tile<BN, kWgrad>(ctrl, p, acc, kblocks, tmem_lanes, row, col0, tbuf, sring, abort, lane, release))
+        break;
       const int64_t m = static_cast<int64_t>(mp) * 2 * BM + rank * BM + row;
-      const int64_t ncol0 = static_cast<int64_t>(nb) * BN + col0;
-#pragma unroll
-      for (int j = 0; j < kHalf / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
-
-      for (int kb = 0; kb < kblocks; ++kb) {
-        const bool got =
-            mbar_wait_bounded_pair(&ctrl->sfull[slot], sphase, abort, peer_abort, p.timeout_ns, p.err) &&
-            mbar_wait_bounded_pair(&ctrl->tfull[abuf], aphase, abort, peer_abort, p.timeout_ns, p.err);
-        if (!__all_sync(0xFFFFFFFFu, got)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-        const ScaleSlot& ss = ctrl->slots[slot];
-        const float sa = ss.sa[row];
-        const float f = kWgrad ? 0.0f : sa * ss.sb[wg];
-        const float* sbc = ss.sb + col0;
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + abuf * BN + col0;
-        if constexpr (kSplit) {
-#pragma unroll
-          for (int c = 0; c < kHalf; c += 64) {
-            uint32_t r[64];
-            tmem_ld_32x32b_x64(taddr + c, r);
-            tmem_wait_ld64(r);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              promote16<kWgrad>(acc + c / 2 + 8 * q, *reinterpret_cast<const uint32_t(*)[16]>(r + 16 * q), f,
-                                sbc + c + 16 * q, sa);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < kHalf; c += 16) {
-            uint32_t r[16];
-            tmem_ld_32x32b_x16(taddr + c, r);
-            tmem_wait_ld16(r);
-            promote16<kWgrad>(acc + c / 2, r, f, sbc + c, sa);
-          }
-        }
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) {
-          if (leader)
-            mbar_arrive(&ctrl->tempty[abuf]);
-          else
-            mbar_arrive_remote(mapa_shared(smem_addr(&ctrl->tempty[abuf]), 0));
-          mbar_arrive(&ctrl->sempty[slot]);
-        }
-        if (++abuf == kAccBufs) {
-          abuf = 0;
-          aphase ^= 1u;
-        }
-        if (++slot == kSRing) {
-          slot = 0;
-          sphase ^= 1u;
-        }
-      }
-      if (!ok) break;
-      uint16_t* drow = p.d + m * p.ldd + ncol0;
-#pragma unroll
-      for (int j = 0; j < kHalf; j += 16) {
-        uint32_t v[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = pack_bf16x2(acc[j / 2 + q].x, acc[j / 2 + q].y);
-        st_global_v8(drow + j, v);
-      }
+      store_row_bf16<kCols>(p.d + m * p.ldd + static_cast<int64_t>(nb) * BN + col0, acc);
     }
   }
 
@@ -907,7 +797,7 @@ __global__ void __launch_bounds__(Layout<kSplit>::kThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
-    tmem_dealloc_pair(tmem_base, kAccBufs * BN);
+    tmem_dealloc_pair(tmem_base, kPairAccBufs * BN);
   }
 }
 
@@ -943,27 +833,35 @@ uint32_t fmt_bits(const GemmArgs& g) {
   return (static_cast<uint32_t>(g.a_e5m2 != 0) << 7) | (static_cast<uint32_t>(g.b_e5m2 != 0) << 10);
 }
 
+// SM count of the current device (cached per context).
 int num_sms() {
-  static int sms = 0;
-  if (!sms) {
+  static PerContext<int> cache;
+  int sms = 0;
+  const cudaError_t e = cache.get(&sms, [](int* v) {
     int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 1;
-  }
-  return sms;
+    cudaError_t r = cudaGetDevice(&dev);
+    if (r == cudaSuccess) r = cudaDeviceGetAttribute(v, cudaDevAttrMultiProcessorCount, dev);
+    return r;
+  });
+  return (e == cudaSuccess && sms > 0) ? sms : 1;
 }
 
-template <int BN, bool kWgrad, bool kSplit, bool kTensor = false, bool kQuad = false>
+// Opts a kernel into `bytes` of dynamic shared memory, once per context.
+template <typename Kernel>
+cudaError_t set_smem_once(PerContext<int>& cache, Kernel kernel, int bytes) {
+  int done = 0;
+  return cache.get(&done, [&](int* v) {
+    *v = 1;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  });
+}
+
+template <int BN, bool kWgrad, bool kTensor = false>
 cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
-  static bool attr_set = false;
+  static PerContext<int> smem_set;
   constexpr int kSmem = smem_bytes<BN>();
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_blockwise_kernel<BN, kWgrad, kSplit, kTensor, kQuad>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  if (cudaError_t e = set_smem_once(smem_set, gemm_blockwise_kernel<BN, kWgrad, kTensor>, kSmem); e != cudaSuccess)
+    return e;
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BN)) return cudaErrorInvalidValue;
   const int num_mb = static_cast<int>(g.M / BM);
@@ -975,27 +873,22 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(Layout<kSplit, kQuad>::kThreads, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   cfg.numAttrs = set_pdl_attr(attr, g.pdl);
   cfg.attrs = attr;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<BN, kWgrad, kSplit, kTensor, kQuad>, ta, tb, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<BN, kWgrad, kTensor>, ta, tb, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-template <bool kWgrad, bool kSplit>
+template <bool kWgrad>
 cudaError_t launch_pair(const GemmArgs& g, cudaStream_t stream) {
-  static bool attr_set = false;
+  static PerContext<int> smem_set;
   constexpr int kSmem = pair_smem_bytes();
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<kWgrad, kSplit>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  if (cudaError_t e = set_smem_once(smem_set, gemm_pair_kernel<kWgrad>, kSmem); e != cudaSuccess) return e;
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BM)) return cudaErrorInvalidValue;
   GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, 0, fmt_bits(g), nullptr,
@@ -1005,7 +898,7 @@ cudaError_t launch_pair(const GemmArgs& g, cudaStream_t stream) {
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(Layout<kSplit>::kThreads, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -1015,7 +908,7 @@ cudaError_t launch_pair(const GemmArgs& g, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1 + set_pdl_attr(attr + 1, g.pdl);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kWgrad, kSplit>, ta, tb, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<kWgrad>, ta, tb, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1032,11 +925,8 @@ double wave_eff(int64_t tiles) {
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   const bool wgrad = g.layout == 2;
   // Pair tiles (256 x 256 over two SMs) only on request, when the shape allows them.
-  if (g.pair > 0 && g.block_n == 0 && g.M % 256 == 0 && g.N % 256 == 0) {
-    const bool split = g.tmem_db < 0 ? wgrad : g.tmem_db != 0;
-    if (wgrad) return split ? launch_pair<true, true>(g, stream) : launch_pair<true, false>(g, stream);
-    return split ? launch_pair<false, true>(g, stream) : launch_pair<false, false>(g, stream);
-  }
+  if (g.pair > 0 && g.block_n == 0 && !g.tensor_sa && g.M % 256 == 0 && g.N % 256 == 0)
+    return wgrad ? launch_pair<true>(g, stream) : launch_pair<false>(g, stream);
   int bn = g.block_n;
   if (bn == 0) {
     bn = 128;
@@ -1047,31 +937,12 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream) {
     }
   }
   if (bn == 256 && g.N % 256 != 0) return cudaErrorInvalidValue;
-  if (g.tensor_sa) {   // per-tensor scales: plain layout, no per-K-block promotion
+  if (g.tensor_sa) {   // per-tensor scales: no per-K-block promotion
     if (g.layout != 0) return cudaErrorInvalidValue;
-    return bn == 256 ? launch_variant<256, false, false, true>(g, stream)
-                     : launch_variant<128, false, false, true>(g, stream);
+    return bn == 256 ? launch_variant<256, false, true>(g, stream) : launch_variant<128, false, true>(g, stream);
   }
-  // The register split with double-buffered TMEM reads pays off where the
-  // promotion does more work per column (WGRAD); measured on B200, the plain
-  // layout is faster for the forward/data-gradient promotion.
-  // Sixteen promotion warps (quad layout): opt-in.
-  if (g.quad > 0) {
-    if (bn == 256)
-      return wgrad ? launch_variant<256, true, true, false, true>(g, stream)
-                   : launch_variant<256, false, true, false, true>(g, stream);
-    return wgrad ? launch_variant<128, true, true, false, true>(g, stream)
-                 : launch_variant<128, false, true, false, true>(g, stream);
-  }
-  const bool db = g.tmem_db < 0 ? wgrad : g.tmem_db != 0;
-  if (bn == 256) {
-    if (wgrad) return db ? launch_variant<256, true, true>(g, stream) : launch_variant<256, true, false>(g, stream);
-    return db ? launch_variant<256, false, true>(g, stream) : launch_variant<256, false, false>(g, stream);
-  }
-  if (bn == 128) {
-    if (wgrad) return db ? launch_variant<128, true, true>(g, stream) : launch_variant<128, true, false>(g, stream);
-    return db ? launch_variant<128, false, true>(g, stream) : launch_variant<128, false, false>(g, stream);
-  }
+  if (bn == 256) return wgrad ? launch_variant<256, true>(g, stream) : launch_variant<256, false>(g, stream);
+  if (bn == 128) return wgrad ? launch_variant<128, true>(g, stream) : launch_variant<128, false>(g, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -59,8 +59,6 @@ struct GemmArgs {
   uint64_t timeout_ns;        // bound on every device-side wait
   int inject_stall;           // test hook: the MMA issuer waits on a barrier nothing completes
   int block_n;                // 0 = choose, else 128 or 256
-  int tmem_db;                // -1 = choose, 0/1 = single/double-buffered TMEM reads
-  int quad;                   // 1 = sixteen promotion warps (quad layout), 0 = eight
   int pair;                   // 1 = use 256 x 256 pair tiles when the shape allows, 0 = never
   int group_m;                // tile order: M-blocks per group (0 = default)
   int pdl;                    // 1 = launch with programmatic stream serialization

@@ -41,6 +41,7 @@
 // 448 rounds or saturates to 448.
 #include <cuda_fp8.h>
 
+#include "context.h"
 #include "device.cuh"
 #include "kernels.h"
 #include "qmath.cuh"
@@ -365,18 +366,19 @@ bool make_input_map(CUtensorMap* map, const QuantArgs& a) {
 
 template <int MODE>
 cudaError_t launch_mode(const QuantArgs& a, cudaStream_t stream) {
-  static int grid_cap = 0;  // resident CTAs on this device (set on first use)
+  static PerContext<int> resident;   // resident CTAs on the device, after the shared-memory opt-in
   constexpr int kSmem = smem_bytes_for<MODE>();
-  if (grid_cap == 0) {
-    cudaError_t e = cudaFuncSetAttribute(quant_tile_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
+  int grid_cap = 0;
+  cudaError_t e = resident.get(&grid_cap, [](int* cap) {
+    cudaError_t r = cudaFuncSetAttribute(quant_tile_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     int dev = 0, sms = 0, per_sm = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_tile_kernel<MODE>, kThreads, kSmem);
-    if (e != cudaSuccess) return e;
-    grid_cap = sms * (per_sm > 0 ? per_sm : 1);
-  }
+    if (r == cudaSuccess) r = cudaGetDevice(&dev);
+    if (r == cudaSuccess) r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (r == cudaSuccess) r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_tile_kernel<MODE>, kThreads, kSmem);
+    *cap = sms * (per_sm > 0 ? per_sm : 1);
+    return r;
+  });
+  if (e != cudaSuccess) return e;
   CUtensorMap map;
   if (!make_input_map(&map, a)) return cudaErrorInvalidValue;
   const int64_t tiles = a.tiles_r * a.tiles_c;
@@ -389,7 +391,7 @@ cudaError_t launch_mode(const QuantArgs& a, cudaStream_t stream) {
   cudaLaunchAttribute attr[1];
   cfg.numAttrs = set_pdl_attr(attr, a.pdl);
   cfg.attrs = attr;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, quant_tile_kernel<MODE>, map, a);
+  e = cudaLaunchKernelEx(&cfg, quant_tile_kernel<MODE>, map, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -19,10 +19,9 @@
 //                         above 448; inputs beyond 1024 s are first clamped to
 //                         +-1024 s (same saturated code, no overflow to
 //                         infinity in the quotient).
-#include <atomic>
 #include <cfloat>
-#include <mutex>
 
+#include "context.h"
 #include "device.cuh"
 #include "kernels.h"
 #include "qmath.cuh"
@@ -164,39 +163,29 @@ cudaError_t launch_amax_ema(const TensorArgs& t, uint32_t* partials, cudaStream_
 }
 
 cudaError_t static_amax_partials(uint32_t** out) {
-  constexpr int kMaxDevices = 64;
-  static std::atomic<uint32_t*> cached[kMaxDevices];   // static storage: starts null
-  static std::mutex lookup;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  uint32_t* p = cached[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    std::lock_guard<std::mutex> hold(lookup);
-    p = cached[dev].load(std::memory_order_relaxed);
-    if (p == nullptr) {
-      void* addr = nullptr;
-      e = cudaGetSymbolAddress(&addr, g_static_amax_partials);
-      if (e != cudaSuccess) return e;
-      p = static_cast<uint32_t*>(addr);
-      cached[dev].store(p, std::memory_order_release);
-    }
-  }
-  *out = p;
-  return cudaSuccess;
+  // The array's address belongs to the context: a process driving several
+  // devices, or a context re-created after cudaDeviceReset, looks it up again.
+  static PerContext<uint32_t*> cached;
+  return cached.get(out, [](uint32_t** p) {
+    void* addr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&addr, g_static_amax_partials);
+    *p = static_cast<uint32_t*>(addr);
+    return e;
+  });
 }
 
 cudaError_t launch_quant_tensor(const TensorArgs& t, uint8_t* q, cudaStream_t stream) {
-  static int grid_cap = 0;
-  if (grid_cap == 0) {
+  static PerContext<int> resident;   // resident CTAs on the device
+  int grid_cap = 0;
+  cudaError_t e = resident.get(&grid_cap, [](int* cap) {
     int dev = 0, sms = 0, per_sm = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_tensor_kernel, kQuantThreads, 0);
-    if (e != cudaSuccess) return e;
-    grid_cap = sms * (per_sm > 0 ? per_sm : 1);
-  }
+    cudaError_t r = cudaGetDevice(&dev);
+    if (r == cudaSuccess) r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (r == cudaSuccess) r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_tensor_kernel, kQuantThreads, 0);
+    *cap = sms * (per_sm > 0 ? per_sm : 1);
+    return r;
+  });
+  if (e != cudaSuccess) return e;
   const int64_t work = t.rows * (t.cols / 8);
   const int64_t blocks = (work + kQuantThreads - 1) / kQuantThreads;
   cudaLaunchConfig_t cfg = {};
@@ -208,7 +197,7 @@ cudaError_t launch_quant_tensor(const TensorArgs& t, uint8_t* q, cudaStream_t st
   cfg.attrs = attr;
   const int64_t chunks = t.cols / 8;
   const int64_t step = static_cast<int64_t>(cfg.gridDim.x) * kQuantThreads;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, quant_tensor_kernel, t.x, t.rows, t.cols, t.ldx,
+  e = cudaLaunchKernelEx(&cfg, quant_tensor_kernel, t.x, t.rows, t.cols, t.ldx,
                                      static_cast<const float*>(t.scale), q, step / chunks, step % chunks);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

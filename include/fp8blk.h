@@ -42,10 +42,8 @@
  *      FP8BLK_WAIT_TIMEOUT_MS     bound of each device-side wait (default 4000)
  *      FP8BLK_PDL=1               launch with programmatic dependent launch
  *      FP8BLK_GEMM_BLOCK_N        128 or 256: force the GEMM tile width
- *      FP8BLK_GEMM_TMEM_DB        0 or 1: force the plain or register-split
- *                                 GEMM thread layout
- *      FP8BLK_GEMM_QUAD=1         sixteen promotion warps (640 threads)
- *      FP8BLK_GEMM_PAIR=1         256x256 tiles on CTA pairs where possible
+ *      FP8BLK_GEMM_PAIR           1: 256x256 tiles on CTA pairs wherever M and
+ *                                 N are multiples of 256; 0: never (default)
  *      FP8BLK_GEMM_GROUP_M        M-blocks per group of the GEMM tile order
  *      FP8BLK_TEST_INJECT_STALL=1 tests only: one wait of the next launch
  *                                 never completes, so that the bounded-wait
