@@ -50,9 +50,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_FLUSH_BYTES = 256 << 20
 # DRAM traffic of the 12 GEMM launches of one decoder-layer step at 16384 tokens
 # (dram__bytes_read.sum + dram__bytes_write.sum, one ncu pass over the launches of
-# one step; profiles/gemm_dram_layer_16384.md), for the GEMM kernel of commit
-# f6bf0e3; algorithmic minimum 2.59 GB (codes read once, bf16 outputs written once).
-GEMM_STEP_DRAM_BYTES_16384 = 2.95e9
+# one step; profiles/gemm_dram_layer_16384.md); algorithmic minimum 2.59 GB (codes
+# read once, bf16 outputs written once).  It describes the GEMM source whose
+# SHA-256 prefix is given; for any other source the bench reports no traffic.
+GEMM_STEP_DRAM = {"bytes": 2.95e9, "gemm_cu_sha256": "0000000000000000"}
+GEMM_SOURCE = os.path.join(ROOT, "fp8_blockwise_scaled_b200", "csrc", "gemm.cu")
 
 WORKLOAD_DESC = {
     "layer": "qwen2-1.5b-shaped decoder layer linears (qkv 2048x1536, o 1536x1536, gate_up 17920x1536, "
@@ -69,6 +71,20 @@ def load_peaks() -> tuple[dict, str]:
         with open(path) as f:
             return json.load(f), "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_source_sha() -> str:
+    import hashlib
+    with open(GEMM_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def fp8_peaks(peaks: dict) -> dict:
+    """Dense FP8 denominators: the measured bf16 GEMM rate times the nominal FP8/BF16 ratio,
+    burst (for kernels timed on their own) and sustained, and NVIDIA's dense FP8 figure."""
+    return {"burst": peaks["bf16_tflops"] * FP8_PER_BF16,
+            "sustained": peaks["bf16_tflops_sustained"] * FP8_PER_BF16,
+            "spec": SPEC_FP8_TFLOPS}
 
 
 # --------------------------------------------------------------------------- workload programs
@@ -101,6 +117,7 @@ class Program:
         self.inputs = []       # (device tensor, host array) copied in by the end-to-end run
         self.outputs = []      # device tensors read back by the end-to-end run
         self.grads = []        # weight gradients all-reduced across ranks
+        self.named = {}        # "<linear>.<buffer>" -> device tensor (the parity tests read them)
         self.gemm_flops = 0
         E4 = torch.float8_e4m3fn
         if recipe == "delayed":
@@ -121,6 +138,8 @@ class Program:
             qxT = f(K, T) if need_colt_x else None
             sxT = f(T // 128, K, dt=torch.float32) if need_colt_x else None
             mode = (fb.ROWWISE if need_row_x else 0) | (fb.COLWISE_T if need_colt_x else 0)
+            self.named.update({f"{g}.X": x, f"{g}.W": w, f"{g}.qx": qx, f"{g}.sx": sx, f"{g}.qxT": qxT,
+                               f"{g}.sxT": sxT})
             qbytes = T * K * (2 + (1 + 4 / 128) * (int(need_row_x) + int(need_colt_x)))
             self._op(f"{g}.quant_x", "quant", qbytes,
                      lambda x=x, m=mode, a=qx, b=sx, c=qxT, d=sxT: fb.fp8blk_quantize_act_1x128(x, m, a, b, c, d))
@@ -137,8 +156,12 @@ class Program:
             elif "dgrad" in passes:
                 self._op(f"{g}.quant_wt", "quant", N * K * (3 + 4 / 16384),
                          lambda w=w, q=qwT, s=swT: fb.fp8blk_quantize_weight_128x128_t(w, q, s))
+            self.named.update({f"{g}.qw": qw if "fwd" in passes else None, f"{g}.sw": sw if "fwd" in passes else None,
+                               f"{g}.qwT": qwT if "dgrad" in passes else None,
+                               f"{g}.swT": swT if "dgrad" in passes else None})
             if "fwd" in passes:
                 y = torch.empty(T, N, dtype=torch.bfloat16, device=device)
+                self.named[f"{g}.Y"] = y
                 self._op(f"{g}.gemm_fwd", "gemm", 2 * T * N * K,
                          lambda a=qx, sa=sx, b=qw, sb=sw, d=y: fb.fp8blk_gemm(fb.FWD, a, sa, b, sb, d))
                 self.outputs.append(y)
@@ -151,6 +174,7 @@ class Program:
                 sd = f(N // 128, T, dt=torch.float32) if need_row_d else None
                 qdT = f(N, T, dt=gdt) if need_colt_d else None
                 sdT = f(T // 128, N, dt=torch.float32) if need_colt_d else None
+                self.named.update({f"{g}.dY": dy, f"{g}.qd": qd, f"{g}.sd": sd, f"{g}.qdT": qdT, f"{g}.sdT": sdT})
                 mode_d = ((fb.ROWWISE if need_row_d else 0) | (fb.COLWISE_T if need_colt_d else 0)
                           | (fb.E5M2 if grad_e5m2 else 0))
                 self._op(f"{g}.quant_dy", "quant", T * N * (2 + (1 + 4 / 128) * (int(need_row_d) + int(need_colt_d))),
@@ -158,15 +182,20 @@ class Program:
                          fb.fp8blk_quantize_act_1x128(x, m, a, b, c, d))
                 if need_row_d:
                     dx = torch.empty(T, K, dtype=torch.bfloat16, device=device)
+                    self.named[f"{g}.dX"] = dx
                     self._op(f"{g}.gemm_dgrad", "gemm", 2 * T * N * K,
                              lambda a=qd, sa=sd, b=qwT, sb=swT, d=dx: fb.fp8blk_gemm(fb.DGRAD, a, sa, b, sb, d))
                     self.outputs.append(dx)
                 if need_colt_d:
                     dw = torch.empty(N, K, dtype=torch.bfloat16, device=device)
+                    self.named[f"{g}.dW"] = dw
+                    # Data parallel: this rank's partial dW in fp32, summed across ranks, rounded once.
+                    part = torch.empty(N, K, dtype=torch.float32, device=device) if world > 1 else dw
                     self._op(f"{g}.gemm_wgrad", "gemm", 2 * T * N * K,
-                             lambda a=qdT, sa=sdT, b=qxT, sb=sxT, d=dw: fb.fp8blk_gemm(fb.WGRAD, a, sa, b, sb, d))
+                             lambda a=qdT, sa=sdT, b=qxT, sb=sxT, d=part: fb.fp8blk_gemm(fb.WGRAD, a, sa, b, sb, d))
                     self.outputs.append(dw)
-                    self.grads.append(dw)
+                    if world > 1:
+                        self.grads.append((part, dw))
         self.gemm_flops = sum(u for _, k, u, _ in self.ops if k == "gemm")
         self.quant_bytes = sum(u for _, k, u, _ in self.ops if k == "quant")
 
@@ -344,6 +373,108 @@ def cpu_baseline(specs) -> dict:
             "sample": desc, "seconds": round(dt, 3)}
 
 
+# --------------------------------------------------------------------------- extra measurements
+def time_program(prog, flush, steps: int, warmup: int) -> dict:
+    """Median per-op event times of eager launches, and the median device time of the
+    whole step replayed as one CUDA graph (L2 flushed before every step)."""
+    import torch
+    for _ in range(warmup):
+        flush.zero_()
+        prog.run(reduce=False)
+    torch.cuda.synchronize()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in prog.ops]
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        prog.run(ev[i], reduce=False)
+    torch.cuda.synchronize()
+    op_ms = [statistics.median(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(steps))
+             for j in range(len(prog.ops))]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        prog.run(reduce=False)
+    graph.replay()
+    torch.cuda.synchronize()
+    st = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        st[i][0].record()
+        graph.replay()
+        st[i][1].record()
+    torch.cuda.synchronize()
+    step_ms = statistics.median(a.elapsed_time(b) for a, b in st)
+    del graph
+    gemm_ms = sum(ms for ms, (_, kind, _, _) in zip(op_ms, prog.ops) if kind == "gemm")
+    quant_ms = sum(ms for ms, (_, kind, _, _) in zip(op_ms, prog.ops) if kind == "quant")
+    return {"op_ms": op_ms, "step_ms": step_ms, "gemm_ms": gemm_ms, "quant_ms": quant_ms}
+
+
+def time_configs_8192(dev, flush, fp8: dict, steps: int) -> dict:
+    """The 8192-token configs (QKV forward, MLP forward, MLP down backward), each one step of its
+    quantisers and GEMMs: the GEMM kernel alone and the sequential step including quantisation."""
+    import torch
+    out = {}
+    for name in ("qkv_fwd", "mlp_fwd", "down_bwd"):
+        prog = Program(workload_tensors(name, 8192), dev, 1)
+        t = time_program(prog, flush, steps, 3)
+        gemm = prog.gemm_flops / (t["gemm_ms"] * 1e-3) / 1e12
+        incl = prog.gemm_flops / (t["step_ms"] * 1e-3) / 1e12
+        out[name] = {"gemm_tflops": round(gemm, 1), "gemm_frac": round(gemm / fp8["burst"], 3),
+                     "gemm_frac_of_spec": round(gemm / fp8["spec"], 3),
+                     "incl_quant_tflops": round(incl, 1), "incl_quant_frac": round(incl / fp8["burst"], 3),
+                     "incl_quant_frac_of_spec": round(incl / fp8["spec"], 3),
+                     "quant_gbs": round(prog.quant_bytes / (t["quant_ms"] * 1e-3) / 1e9, 1),
+                     "step_ms": round(t["step_ms"], 4)}
+        del prog
+        torch.cuda.empty_cache()
+    return out
+
+
+def time_sweep(dev, flush, fp8: dict, steps: int) -> dict:
+    """Token sweep of the decoder layer (all 12 GEMMs and their quantisers) at every count in
+    workloads.TOKEN_SWEEP: the step including quantisation (one graph) and the GEMMs alone."""
+    import torch
+    rows = []
+    for m in workloads.TOKEN_SWEEP:
+        prog = Program(workload_tensors("layer", m), dev, 1)
+        t = time_program(prog, flush, steps, 3)
+        incl = prog.gemm_flops / (t["step_ms"] * 1e-3) / 1e12
+        gemm = prog.gemm_flops / (t["gemm_ms"] * 1e-3) / 1e12
+        rows.append({"tokens": m, "incl_quant_tflops": round(incl, 1), "gemm_tflops": round(gemm, 1),
+                     "incl_quant_frac_of_spec": round(incl / fp8["spec"], 3)})
+        del prog
+        torch.cuda.empty_cache()
+    best = max(r["incl_quant_tflops"] for r in rows)
+    knee = next(r["tokens"] for r in rows if r["incl_quant_tflops"] >= 0.95 * best)
+    return {"points": rows, "knee_tokens": knee,
+            "knee_rule": "smallest token count within 5% of the best step rate including quantisation"}
+
+
+def time_fp8_proxy(dev) -> dict:
+    """Context only: the library's per-tensor-scaled FP8 GEMM (torch._scaled_mm, cuBLASLt) at
+    8192^3, best of 10 launches.  No 1x128 / 128x128 blockwise library kernel exists on sm_100
+    to compare against; this is the plain FP8 tensor-core rate on this GPU."""
+    import torch
+    try:
+        a = torch.randn(8192, 8192, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(8192, 8192, device=dev).to(torch.float8_e4m3fn)
+        one = torch.ones((), device=dev)
+        for _ in range(3):
+            torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        return {"kernel": "torch._scaled_mm per-tensor FP8 8192^3", "tflops": round(2 * 8192**3 / (best * 1e-3) / 1e12, 1)}
+    except Exception as e:     # context only: never fails the bench
+        return {"kernel": "torch._scaled_mm per-tensor FP8 8192^3", "unavailable": str(e)[:200]}
+
+
 # --------------------------------------------------------------------------- arms
 def run_reference(args, rank: int, world: int):
     """The oracle, as it stands, on the host cores: each step a bounded sample of the workload."""
@@ -490,7 +621,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     err = prog.fb.fp8blk_get_device_error()
 
     peaks, peak_src = load_peaks()
-    fp8_peak = peaks["bf16_tflops_sustained"] * FP8_PER_BF16
+    fp8 = fp8_peaks(peaks)
+    fp8_peak = fp8["burst"]
     flops_all = prog.gemm_flops * world
     value = flops_all * args.steps / (total_ms * 1e-3) / 1e12
     gemm_tflops = prog.gemm_flops * args.steps / (gemm_ms * 1e-3) / 1e12
@@ -499,7 +631,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     for j, (label, kind, units, _) in enumerate(prog.ops):
         ms = statistics.median(per_op_ms[i][j] for i in range(args.steps))
         rate = units / (ms * 1e-3) / (1e12 if kind == "gemm" else 1e9)
-        per_op[label] = {"us": round(ms * 1e3, 1), ("tflops" if kind == "gemm" else "gbs"): round(rate, 1)}
+        per_op[label] = {"us": round(ms * 1e3, 1), ("tflops" if kind == "gemm" else "gbs"): round(rate, 1),
+                         "frac": round(rate / (fp8_peak if kind == "gemm" else peaks["hbm_gbs"]), 3)}
+    traffic_ok = args.workload == "layer" and tokens == 16384 and gemm_source_sha() == GEMM_STEP_DRAM["gemm_cu_sha256"]
+    extra = {}
+    if rank == 0 and world == 1 and args.workload == "layer" and not args.no_extra:
+        extra["configs_8192"] = time_configs_8192(dev, flush, fp8, max(3, min(args.steps, 10)))
+        extra["token_sweep"] = time_sweep(dev, flush, fp8, 5)
+        extra["fp8_library_proxy"] = time_fp8_proxy(dev)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -517,9 +656,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "frac_of_spec_fp8_peak": value / SPEC_FP8_TFLOPS,
         "roofline": {"bound": "tensor", "kernel": "gemm_blockwise_kernel", "achieved": gemm_tflops,
                      "peak": fp8_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
-                     "traffic": GEMM_STEP_DRAM_BYTES_16384 if (args.workload == "layer" and tokens == 16384) else None,
+                     "traffic": GEMM_STEP_DRAM["bytes"] if traffic_ok else None,
                      "traffic_scope": "bytes per step, the 12 GEMM launches together (achieved is over the same launches)",
-                     "peak_source": f"{peak_src} bf16 sustained x {FP8_PER_BF16:g} (nominal fp8/bf16 ratio)",
+                     "traffic_note": "ncu capture of this GEMM source" if traffic_ok else
+                                     "no capture of this GEMM source (or another workload): not reported",
+                     "peak_source": f"{peak_src} bf16 burst x {FP8_PER_BF16:g} (nominal fp8/bf16 ratio); each GEMM "
+                                    "is timed on its own by CUDA events, so the burst figure applies",
+                     "frac_of_sustained_derived_peak": gemm_tflops / fp8["sustained"],
                      "frac_of_spec_fp8": gemm_tflops / SPEC_FP8_TFLOPS},
         "quant": {"kernel": "quant_tile_kernel", "achieved_gbs": quant_gbs, "peak_gbs": peaks["hbm_gbs"],
                   "frac": quant_gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm copy"},
@@ -530,10 +673,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "per_op_median": per_op,
         "e2e": {"value": flops_all * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        # one kernel per op, two for an amax EMA (partial maxima, then the EMA)
-        "gpu_launches": sum(2 if ".amax_" in label else 1 for label, _, _, _ in prog.ops) * args.steps,
+        # one kernel per op, two for an amax EMA (partial maxima, then the EMA), and with
+        # data parallelism one rounding kernel per weight gradient after its all-reduce
+        "gpu_launches": (sum(2 if ".amax_" in label else 1 for label, _, _, _ in prog.ops)
+                         + len(prog.grads)) * args.steps,
         "clocks": clocks,
         "device_error": prog.fb.status_string(err),
+        **extra,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(workload_tensors(args.workload, 256) if tokens != 256 else specs)
@@ -587,6 +733,8 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=0, help="tokens per GPU (default 16384 for layer, else 8192)")
     ap.add_argument("--sweep", action="store_true", help="token sweep of the layer GEMMs (one JSON line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the 8192-token configs, the token sweep and the library FP8 proxy")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of the step's CUDA graph")
     ap.add_argument("--recipe", choices=["blockwise", "delayed"], default="blockwise",
                     help="blockwise 1x128 / 128x128 scaling (fwd+dgrad+wgrad), or the per-tensor delayed-scaling "

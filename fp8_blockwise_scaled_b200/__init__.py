@@ -26,16 +26,17 @@ import ctypes
 
 import torch
 
-from ._lib import (A_E5M2, B_E5M2, BOTH, COLWISE_T, DGRAD, E5M2, FWD, ROWWISE, WGRAD, Fp8BlkError, LIB_PATH,
-                   check, lib, status_string)
+from ._lib import (A_E5M2, B_E5M2, BOTH, COLWISE_T, DGRAD, E5M2, FWD, OUT_F32, ROWWISE, WGRAD, Fp8BlkError,
+                   LIB_PATH, check, lib, status_string)
 
 __all__ = [
     "fp8blk_quantize_act_1x128", "fp8blk_quantize_weight_128x128", "fp8blk_quantize_weight_128x128_t",
     "fp8blk_quantize_weight_128x128_both", "fp8blk_amax_ema", "fp8blk_amax_ema_workspace_bytes",
     "fp8blk_amax_ema_static", "AMAX_EMA_STATIC_MAX_ROWS",
     "fp8blk_quantize_tensor", "fp8blk_gemm_tensor_scaled", "fp8_linear_delayed_forward",
-    "fp8blk_gemm", "fp8blk_get_device_error", "fp8blk_version", "linear_forward", "linear_backward",
-    "ROWWISE", "COLWISE_T", "BOTH", "E5M2", "FWD", "DGRAD", "WGRAD", "A_E5M2", "B_E5M2", "Fp8BlkError",
+    "fp8blk_gemm", "fp8blk_round_f32_to_bf16", "fp8blk_get_device_error", "fp8blk_version", "linear_forward",
+    "linear_backward", "ROWWISE", "COLWISE_T", "BOTH", "E5M2", "FWD", "DGRAD", "WGRAD", "A_E5M2", "B_E5M2",
+    "OUT_F32", "Fp8BlkError",
     "LIB_PATH", "status_string",
 ]
 
@@ -134,8 +135,9 @@ def fp8blk_quantize_weight_128x128_both(w, q=None, s=None, qT=None, sT=None, str
     return q, s, qT, sT
 
 
-def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None):
-    """Blockwise-scaled E4M3 GEMM, D[M,N] = dequant(A) . dequant(B)^T in bf16."""
+def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None, out_dtype=torch.bfloat16):
+    """Blockwise-scaled E4M3 GEMM, D[M,N] = dequant(A) . dequant(B)^T in bf16 (or, with
+    out_dtype=torch.float32 or an fp32 d, the unrounded fp32 sums)."""
     _need_cuda(a, sa, b, sb, d)
     m, k = a.shape
     n = b.shape[0]
@@ -149,13 +151,26 @@ def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None):
     if not (a.is_contiguous() and b.is_contiguous() and sa.is_contiguous() and sb.is_contiguous()):
         raise ValueError("operands and scales must be contiguous")
     if d is None:
-        d = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
-    elif d.dtype != torch.bfloat16 or d.dim() != 2 or d.stride(1) != 1 or tuple(d.shape) != (m, n):
-        raise ValueError("d must be a bfloat16 [M,N] tensor with unit column stride")
+        if out_dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
+        d = torch.empty((m, n), dtype=out_dtype, device=a.device)
+    elif d.dtype not in (torch.bfloat16, torch.float32) or d.dim() != 2 or d.stride(1) != 1 or tuple(d.shape) != (m, n):
+        raise ValueError("d must be a bfloat16 or float32 [M,N] tensor with unit column stride")
     flags = (A_E5M2 if a.dtype == E5M2_DTYPE else 0) | (B_E5M2 if b.dtype == E5M2_DTYPE else 0)
+    flags |= OUT_F32 if d.dtype == torch.float32 else 0
     check(lib.fp8blk_gemm(int(layout) | flags, m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d), d.stride(0),
                           _stream_handle(stream)))
     return d
+
+
+def fp8blk_round_f32_to_bf16(x, y=None, stream=None):
+    """y = bf16(x) (round to nearest even), elementwise; x a contiguous float32 CUDA tensor."""
+    _need_cuda(x, y)
+    if x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 tensor")
+    y = _out(y, tuple(x.shape), torch.bfloat16, x.device)
+    check(lib.fp8blk_round_f32_to_bf16(_ptr(x), x.numel(), _ptr(y), _stream_handle(stream)))
+    return y
 
 
 def fp8blk_amax_ema_workspace_bytes(rows: int) -> int:

@@ -13,6 +13,7 @@ LIB_PATH = _build.LIB
 ROWWISE, COLWISE_T, BOTH = 1, 2, 3
 E5M2 = 4                       # OR into an activation mode: E5M2 codes
 A_E5M2, B_E5M2 = 8, 16         # OR into a GEMM layout: that operand holds E5M2 codes
+OUT_F32 = 32                   # OR into a GEMM layout: fp32 output (unrounded sums)
 FWD, DGRAD, WGRAD = 0, 1, 2
 
 STATUS_NAMES = {
@@ -46,6 +47,7 @@ def _load() -> ctypes.CDLL:
         "fp8blk_quantize_tensor": [P, I64, I64, I64, P, P, P],
         "fp8blk_gemm_tensor_scaled": [I64, I64, I64, P, P, P, P, P, I64, P],
         "fp8blk_gemm": [I, I64, I64, I64, P, P, P, P, P, I64, P],
+        "fp8blk_round_f32_to_bf16": [P, I64, P, P],
         "fp8blk_get_device_error": [P],
         "fp8blk_status_string": [I],
         "fp8blk_version": [],

@@ -166,7 +166,8 @@ fp8blk_status fp8blk_quantize_weight_128x128_both(const void* w, int64_t n, int6
 fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uint8_t* a, const float* sa,
                           const uint8_t* b, const float* sb, void* d, int64_t ldd, void* stream) {
   const int formats = layout & (FP8BLK_A_E5M2 | FP8BLK_B_E5M2);
-  layout &= ~(FP8BLK_A_E5M2 | FP8BLK_B_E5M2);
+  const bool out_f32 = (layout & FP8BLK_OUT_F32) != 0;
+  layout &= ~(FP8BLK_A_E5M2 | FP8BLK_B_E5M2 | FP8BLK_OUT_F32);
   if (layout != FP8BLK_FWD && layout != FP8BLK_DGRAD && layout != FP8BLK_WGRAD) return FP8BLK_ERR_INVALID_ARG;
   if (!a || !sa || !b || !sb || !d) return FP8BLK_ERR_INVALID_ARG;
   if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K)) return FP8BLK_ERR_SHAPE;
@@ -174,13 +175,14 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return FP8BLK_ERR_SHAPE;
   if (ldd < N) return FP8BLK_ERR_INVALID_ARG;
   // The epilogue writes 32-byte vectors: d and every output row start on a 32-byte boundary.
-  if (!aligned16(a) || !aligned16(b) || (reinterpret_cast<uintptr_t>(d) & 31u) || ldd % 16 != 0)
+  if (!aligned16(a) || !aligned16(b) || (reinterpret_cast<uintptr_t>(d) & 31u) || ldd % (out_f32 ? 8 : 16) != 0)
     return FP8BLK_ERR_ALIGN;
   if (!aligned16(sa) || !aligned16(sb)) return FP8BLK_ERR_ALIGN;
   fp8blk_status st = check_device();
   if (st != FP8BLK_OK) return st;
   fp8blk::GemmArgs g{};
   g.layout = layout;
+  g.out_f32 = out_f32;
   g.M = M;
   g.N = N;
   g.K = K;
@@ -188,7 +190,7 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   g.sa = sa;
   g.b = b;
   g.sb = sb;
-  g.d = static_cast<uint16_t*>(d);
+  g.d = d;
   g.ldd = ldd;
   g.timeout_ns = wait_timeout_ns();
   g.inject_stall = 0;
@@ -271,7 +273,7 @@ fp8blk_status fp8blk_gemm_tensor_scaled(int64_t M, int64_t N, int64_t K, const u
   g.K = K;
   g.a = a;
   g.b = b;
-  g.d = static_cast<uint16_t*>(d);
+  g.d = d;
   g.ldd = ldd;
   g.timeout_ns = wait_timeout_ns();
   g.err = error_word();
@@ -282,6 +284,16 @@ fp8blk_status fp8blk_gemm_tensor_scaled(int64_t M, int64_t N, int64_t K, const u
   if (const char* e = std::getenv("FP8BLK_GEMM_GROUP_M")) g.group_m = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) g.inject_stall = std::atoi(e) != 0;
   return launch_status(fp8blk::launch_gemm(g, static_cast<cudaStream_t>(stream)));
+}
+
+fp8blk_status fp8blk_round_f32_to_bf16(const float* x, int64_t n, void* y, void* stream) {
+  if (!x || !y) return FP8BLK_ERR_INVALID_ARG;
+  if (n <= 0) return FP8BLK_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(y)) return FP8BLK_ERR_ALIGN;
+  fp8blk_status st = check_device();
+  if (st != FP8BLK_OK) return st;
+  return launch_status(
+      fp8blk::launch_round_bf16(x, n, static_cast<uint16_t*>(y), pdl_enabled(), static_cast<cudaStream_t>(stream)));
 }
 
 fp8blk_status fp8blk_get_device_error(void* stream) {

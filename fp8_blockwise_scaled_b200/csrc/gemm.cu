@@ -122,8 +122,9 @@ struct GemmParams {
   int64_t M, N, K;
   const float* sa;
   const float* sb;
-  uint16_t* d;
-  int64_t ldd;
+  void* d;                // bf16 [M][ldd], or fp32 [M][ldd] when out_f32
+  int64_t ldd;            // in elements of the output type
+  int out_f32;
   uint64_t timeout_ns;
   unsigned int* err;
   int inject_stall;
@@ -223,6 +224,31 @@ __device__ __forceinline__ void store_row_bf16(uint16_t* drow, const float2* acc
     for (int q = 0; q < 8; ++q) v[q] = pack_bf16x2(acc[j / 2 + q].x, acc[j / 2 + q].y);
     st_global_v8(drow + j, v);
   }
+}
+
+// Stores kCols fp32 sums of one row unrounded (32-byte stores): the output of a
+// partial product that is summed further (the data-parallel weight gradient).
+template <int kCols>
+__device__ __forceinline__ void store_row_f32(float* drow, const float2* acc) {
+#pragma unroll
+  for (int j = 0; j < kCols; j += 8) {
+    uint32_t v[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      v[2 * q] = __float_as_uint(acc[j / 2 + q].x);
+      v[2 * q + 1] = __float_as_uint(acc[j / 2 + q].y);
+    }
+    st_global_v8(drow + j, v);
+  }
+}
+
+// The finished row of a tile: bf16 (rounded once) or fp32.
+template <int kCols>
+__device__ __forceinline__ void store_row(const GemmParams& p, int64_t m, int64_t n0, const float2* acc) {
+  if (p.out_f32)
+    store_row_f32<kCols>(static_cast<float*>(p.d) + m * p.ldd + n0, acc);
+  else
+    store_row_bf16<kCols>(static_cast<uint16_t*>(p.d) + m * p.ldd + n0, acc);
 }
 
 // Ring position: an index into a ring of N slots and the parity of its use.
@@ -547,7 +573,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         tc_fence_after_sync();
         const uint32_t taddr = tmem_lanes + tbuf.idx * BN;
-        uint16_t* drow = p.d + (static_cast<int64_t>(mb) * BM + row) * p.ldd + static_cast<int64_t>(nb) * BN + col0;
+        uint16_t* drow = static_cast<uint16_t*>(p.d) + (static_cast<int64_t>(mb) * BM + row) * p.ldd +
+                         static_cast<int64_t>(nb) * BN + col0;
 #pragma unroll
         for (int c = 0; c < kCols; c += 16) {
           uint32_t r[16];
@@ -578,8 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!promote_tile<BN, kWgrad>(ctrl, p, acc, kblocks, tmem_lanes, row, col0, tbuf, sring, abort, lane,
                                       release))
           break;
-        const int64_t m = static_cast<int64_t>(mb) * BM + row;
-        store_row_bf16<kCols>(p.d + m * p.ldd + static_cast<int64_t>(nb) * BN + col0, acc);
+        store_row<kCols>(p, static_cast<int64_t>(mb) * BM + row, static_cast<int64_t>(nb) * BN + col0, acc);
       }
     }
   }
@@ -786,8 +812,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mp = tile % num_mp, nb = tile / num_mp;
       if (!promote_tile<BN, kWgrad>(ctrl, p, acc, kblocks, tmem_lanes, row, col0, tbuf, sring, abort, lane, release))
         break;
-      const int64_t m = static_cast<int64_t>(mp) * 2 * BM + rank * BM + row;
-      store_row_bf16<kCols>(p.d + m * p.ldd + static_cast<int64_t>(nb) * BN + col0, acc);
+      store_row<kCols>(p, static_cast<int64_t>(mp) * 2 * BM + rank * BM + row, static_cast<int64_t>(nb) * BN + col0,
+                       acc);
     }
   }
 
@@ -867,8 +893,8 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   const int num_mb = static_cast<int>(g.M / BM);
   int group_m = g.group_m > 0 ? g.group_m : 8;
   if (group_m > num_mb) group_m = num_mb;
-  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, group_m, fmt_bits(g),
-               g.tensor_sa, g.tensor_sb};
+  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.out_f32, g.timeout_ns, g.err, g.inject_stall, group_m,
+               fmt_bits(g), g.tensor_sa, g.tensor_sb};
   const int64_t tiles = (g.M / BM) * (g.N / BN);
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
   cudaLaunchConfig_t cfg = {};
@@ -891,8 +917,8 @@ cudaError_t launch_pair(const GemmArgs& g, cudaStream_t stream) {
   if (cudaError_t e = set_smem_once(smem_set, gemm_pair_kernel<kWgrad>, kSmem); e != cudaSuccess) return e;
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BM)) return cudaErrorInvalidValue;
-  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.timeout_ns, g.err, g.inject_stall, 0, fmt_bits(g), nullptr,
-               nullptr};
+  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.out_f32, g.timeout_ns, g.err, g.inject_stall, 0, fmt_bits(g),
+               nullptr, nullptr};
   const int64_t tiles = (g.M / (2 * BM)) * (g.N / kPairBN);
   const int64_t max_pairs = num_sms() / 2;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
@@ -937,8 +963,8 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream) {
     }
   }
   if (bn == 256 && g.N % 256 != 0) return cudaErrorInvalidValue;
-  if (g.tensor_sa) {   // per-tensor scales: no per-K-block promotion
-    if (g.layout != 0) return cudaErrorInvalidValue;
+  if (g.tensor_sa) {   // per-tensor scales: no per-K-block promotion, bf16 output
+    if (g.layout != 0 || g.out_f32) return cudaErrorInvalidValue;
     return bn == 256 ? launch_variant<256, false, true>(g, stream) : launch_variant<128, false, true>(g, stream);
   }
   if (bn == 256) return wgrad ? launch_variant<256, true>(g, stream) : launch_variant<256, false>(g, stream);

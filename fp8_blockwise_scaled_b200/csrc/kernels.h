@@ -54,8 +54,9 @@ struct GemmArgs {
   const float* sa;            // [K/128][M]
   const uint8_t* b;           // [N][K]
   const float* sb;            // FWD/DGRAD [N/128][K/128];  WGRAD [K/128][N]
-  uint16_t* d;                // [M][ldd] bf16
-  int64_t ldd;
+  void* d;                    // [M][ldd] bf16, or fp32 when out_f32
+  int64_t ldd;                // in elements of the output type
+  int out_f32;                // 1 = fp32 output (unrounded partial sums)
   uint64_t timeout_ns;        // bound on every device-side wait
   int inject_stall;           // test hook: the MMA issuer waits on a barrier nothing completes
   int block_n;                // 0 = choose, else 128 or 256
@@ -69,6 +70,9 @@ struct GemmArgs {
 };
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream);
+
+// y[i] = bf16_round_nearest_even(x[i]) for i < n (x, y 16-byte aligned).
+cudaError_t launch_round_bf16(const float* x, int64_t n, uint16_t* y, int pdl, cudaStream_t stream);
 
 // Fills attr[0] with programmatic stream serialization when `enable` (the
 // kernel may start its prologue while the previous kernel of the stream

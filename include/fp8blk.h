@@ -82,10 +82,14 @@ typedef enum {
   FP8BLK_WGRAD = 2  /* B scales per row and K-block: sb[K/128][N] */
 } fp8blk_layout;
 
-/* OR-ed into a layout: operand A (or B) holds E5M2 codes instead of E4M3. */
+/* OR-ed into a layout: operand A (or B) holds E5M2 codes instead of E4M3;
+ * FP8BLK_OUT_F32: d receives the fp32 sums unrounded (for a partial result
+ * that is summed further, such as one rank's share of a data-parallel weight
+ * gradient; see fp8blk_round_f32_to_bf16). */
 typedef enum {
   FP8BLK_A_E5M2 = 8,
-  FP8BLK_B_E5M2 = 16
+  FP8BLK_B_E5M2 = 16,
+  FP8BLK_OUT_F32 = 32
 } fp8blk_operand_format;
 
 /*
@@ -155,7 +159,9 @@ fp8blk_status fp8blk_quantize_weight_128x128_both(const void* w, int64_t n, int6
  *   operand holds E5M2 codes (E5M2 gradients: DGRAD and WGRAD take dY as A).
  *   sb  FWD / DGRAD: [N/128][K/128] fp32 (per 128x128 block)
  *       WGRAD      : [K/128][N] fp32     (per row of b, per K-block)
- *   d   [M][ldd] bf16 output, ldd >= N, ldd % 16 == 0, d 32-byte aligned.
+ *   d   [M][ldd] bf16 output, ldd >= N, ldd % 16 == 0, d 32-byte aligned;
+ *       with FP8BLK_OUT_F32 in layout: fp32 output, ldd % 8 == 0 (the sums
+ *       are stored without the bf16 rounding).
  *
  * Operands per pass of a linear layer Y = X . W^T (X [T][in], W [out][in]):
  *   FWD   : a = X rowwise,      b = W (128x128),           d = Y  [T][out]
@@ -230,8 +236,21 @@ fp8blk_status fp8blk_gemm_tensor_scaled(int64_t M, int64_t N, int64_t K, const u
                                         const uint8_t* b, const float* sb, void* d, int64_t ldd, void* stream);
 
 /*
+ * y[i] = bf16(x[i]), round to nearest even, for 0 <= i < n: the single
+ * rounding of a sum of fp32 partial results.  Used for the data-parallel
+ * weight gradient: the pages' training run sums gradients across GPUs with
+ * an all-reduce ("小团队也能预训练！普罗2B" (66bd.net), the paragraph on the
+ * 24-GPU AllReduce over GPUDirect RDMA); each rank's WGRAD GEMM writes its
+ * partial dW in fp32 (FP8BLK_OUT_F32), the partials are summed in fp32 by the
+ * all-reduce, and this call rounds the sum to bf16 once.
+ *   x  [n] fp32 device array, y [n] bf16 device array, both 16-byte aligned;
+ *   n > 0 (else FP8BLK_ERR_SHAPE).  x and y must not overlap.
+ */
+fp8blk_status fp8blk_round_f32_to_bf16(const float* x, int64_t n, void* y, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word of the
- * current device.  Returns FP8BLK_OK, FP8BLK_ERR_TIMEOUT if a kernel's
+ * device the stream belongs to (the current device for the default streams).  Returns FP8BLK_OK, FP8BLK_ERR_TIMEOUT if a kernel's
  * bounded wait expired since the last call, or FP8BLK_ERR_CUDA if the
  * synchronisation itself failed.
  */

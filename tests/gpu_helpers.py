@@ -65,3 +65,13 @@ def assert_gemm_close(gpu: np.ndarray, ref: np.ndarray, what: str) -> dict:
     assert e["max_excess_over_rms"] <= MAX_ERR_RMS, f"{what}: {e}"
     assert e["mean_rel"] <= MEAN_REL, f"{what}: {e}"
     return e
+
+
+def stratified_rows(m: int, seed: int) -> np.ndarray:
+    """One seeded row from every (128-row M-block x 32-row TMEM lane quadrant) pair
+    of an M-row GEMM output, i.e. m/32 rows: every output tile row block and every
+    promotion warp's lanes are sampled.  Rows 0 and m-1 are always included."""
+    rng = np.random.default_rng(seed)
+    base = np.arange(0, m, 32)
+    rows = base + rng.integers(0, 32, size=base.size)
+    return np.unique(np.concatenate([rows, [0, m - 1]]))

@@ -98,7 +98,9 @@ def test_quantize_weight_both_argument_errors():
 @pytest.mark.parametrize("args,code", [
     ((3, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 1),   # bad layout
     ((3 | 8, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 1),   # bad layout, E5M2 A
-    ((1 | 32, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 1),  # unknown flag
+    ((1 | 64, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 1),  # unknown flag
+    ((0 | 32, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 132, S), 3),  # fp32 out, ldd % 8
+    ((2 | 32, 128, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, P(0x10010), 128, S), 3),  # fp32 out, d % 32
     ((2 | 8, 100, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 2),   # E5M2 A, bad shape
     ((0, 100, 128, 128, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 2),
     ((0, 128, 128, 96, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 128, S), 2),
@@ -152,3 +154,13 @@ def test_static_amax_row_limit_matches_the_header():
     text = open(HEADER).read()
     assert int(re.search(r"#define FP8BLK_AMAX_EMA_STATIC_MAX_ROWS (\d+)", text).group(1)) == \
         fb.AMAX_EMA_STATIC_MAX_ROWS
+
+
+def test_round_f32_to_bf16_argument_errors():
+    f = _lib.lib.fp8blk_round_f32_to_bf16
+    assert f(NULL, 128, ALIGNED, S) == 1
+    assert f(ALIGNED, 128, NULL, S) == 1
+    assert f(ALIGNED, 0, ALIGNED, S) == 2
+    assert f(ALIGNED, -4, ALIGNED, S) == 2
+    assert f(MISALIGNED, 128, ALIGNED, S) == 3
+    assert f(ALIGNED, 128, MISALIGNED, S) == 3

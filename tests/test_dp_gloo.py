@@ -1,7 +1,10 @@
 """Data-parallel host logic on the CPU: token sharding and the weight-gradient
 all-reduce, with two gloo ranks.  Each rank computes the weight gradient of
-its token shard with the oracle; after the all-reduce every rank must hold
-the full-token result (exactly, on inputs whose quantisation is exact)."""
+its token shard with the oracle and hands it over in the product's types: an
+fp32 partial (what the WGRAD GEMM writes with fp32 output) and a bf16 result
+buffer.  After the fp32 all-reduce and the single rounding every rank must
+hold the full-token result rounded to bf16 (exactly, on inputs whose
+quantisation and partial sums are exact)."""
 import os
 import socket
 
@@ -48,12 +51,30 @@ def _worker(rank, world, port, q):
         t0, t1 = shard_tokens(tokens, rank, world)
         qa, sa = oracle.quantize_act_colwise_t(dy[t0:t1])
         qb, sb = oracle.quantize_act_colwise_t(x[t0:t1])
-        part = torch.from_numpy(oracle.gemm(oracle.WGRAD, qa, sa, qb, sb))
-        allreduce_weight_grads([part])
+        part = torch.from_numpy(oracle.gemm(oracle.WGRAD, qa, sa, qb, sb)).to(torch.float32)
+        out = torch.empty(part.shape, dtype=torch.bfloat16)
+        allreduce_weight_grads([(part, out)], round_fn=lambda a, b: b.copy_(a.to(torch.bfloat16)))
         qa, sa = oracle.quantize_act_colwise_t(dy)
         qb, sb = oracle.quantize_act_colwise_t(x)
         full = oracle.gemm(oracle.WGRAD, qa, sa, qb, sb)
-        q.put((rank, bool(np.array_equal(part.numpy(), full)), (t0, t1)))
+        # Every rank holds the fp32 sum of both ranks' fp32 partials (the same on both ranks,
+        # within the fp32 rounding of the partials and of their sum from the exact full-token
+        # result), rounded once to bf16.
+        shares = []
+        for r in range(world):
+            s0, s1 = shard_tokens(tokens, r, world)
+            a, b = oracle.quantize_act_colwise_t(dy[s0:s1]), oracle.quantize_act_colwise_t(x[s0:s1])
+            shares.append(oracle.gemm(oracle.WGRAD, *a, *b).astype(np.float32))
+        want32 = shares[0] + shares[1]
+        ok = (bool(np.array_equal(part.numpy(), want32))
+              and torch.equal(out, torch.from_numpy(want32).to(torch.bfloat16))
+              and bool(np.all(np.abs(want32 - full) <= 2.0**-22 * (np.abs(shares[0]) + np.abs(shares[1])))))
+        wrong_type = False
+        try:
+            allreduce_weight_grads([(out.float(), out.float())], round_fn=lambda a, b: None)
+        except ValueError:
+            wrong_type = True
+        q.put((rank, ok and wrong_type, (t0, t1)))
     finally:
         dist.destroy_process_group()
 

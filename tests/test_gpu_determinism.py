@@ -38,7 +38,9 @@ def operands():
 
 
 @pytest.mark.parametrize("layout", [fb.FWD, fb.DGRAD, fb.WGRAD])
-def test_gemm_bitwise_repeatable(operands, layout):
+@pytest.mark.parametrize("pair", ["0", "1"])      # the 1-CTA kernel and the CTA-pair kernel
+def test_gemm_bitwise_repeatable(operands, layout, pair, monkeypatch):
+    monkeypatch.setenv("FP8BLK_GEMM_PAIR", pair)
     a, sa, b, sb = operands[layout]
     first = fb.fp8blk_gemm(layout, a, sa, b, sb)
     out = torch.empty_like(first)

@@ -1,7 +1,10 @@
 """GPU blockwise GEMM against the CPU oracle (fp64 over dequantised operands).
 
 The operands come from the oracle's quantisers, so the GEMM is checked on its
-own; the end-to-end tests at the bottom chain the GPU quantisers too.
+own; the tiny-config test chains the GPU quantisers too.  Small shapes, every
+output element; the full-size workloads are in test_gpu_full_size.py.  Shapes
+whose M and N are multiples of 256 run once on each kernel: the 1-CTA kernel
+(FP8BLK_GEMM_PAIR=0) and the CTA-pair kernel (FP8BLK_GEMM_PAIR=1).
 Tolerance: max |gpu - oracle| <= 1e-2 RMS beyond bf16's own rounding, and mean
 relative error <= 2e-3 over entries with |oracle| > 0.1 RMS.
 """
@@ -121,32 +124,23 @@ def test_exact_operands_give_bf16_of_the_exact_product():
     assert np.array_equal(got, want)
 
 
-def _rows(m, rng, n=48):
-    return np.unique(np.concatenate([rng.choice(m, n, replace=False), [0, 127, 128, m - 1]]))
+PAIR_SHAPES = [(256, 256, 128), (512, 512, 1024), (768, 1280, 640), (1024, 256, 384)]
 
 
-# Full-size workloads (in the bench's launch configuration), checked on sampled output rows.
-def test_full_qkv_fwd():
-    d = workloads.qkv_fwd(seed=1)
-    rng = np.random.default_rng(101)
-    ops = _operands(oracle.FWD, d["X"], d["W"])
-    got, ref = _run(oracle.FWD, *ops, rows=_rows(8192, rng))
-    assert_gemm_close(got, ref, "qkv fwd 8192x2048x1536")
-
-
-def test_full_mlp_fwd():
-    d = workloads.mlp_fwd(seed=2)
-    rng = np.random.default_rng(102)
-    got, ref = _run(oracle.FWD, *_operands(oracle.FWD, d["X_gate_up"], d["W_gate_up"]), rows=_rows(8192, rng, 16))
-    assert_gemm_close(got, ref, "gate_up fwd 8192x17920x1536")
-    got, ref = _run(oracle.FWD, *_operands(oracle.FWD, d["X_down"], d["W_down"]), rows=_rows(8192, rng, 24))
-    assert_gemm_close(got, ref, "down fwd 8192x1536x8960")
-
-
-def test_full_down_bwd():
-    d = workloads.down_bwd(seed=3)
-    rng = np.random.default_rng(103)
-    got, ref = _run(oracle.DGRAD, *_operands(oracle.DGRAD, d["dY"], d["W"]), rows=_rows(8192, rng, 24))
-    assert_gemm_close(got, ref, "down dgrad 8192x8960x1536")
-    got, ref = _run(oracle.WGRAD, *_operands(oracle.WGRAD, d["dY"], d["X"]), rows=_rows(1536, rng, 12))
-    assert_gemm_close(got, ref, "down wgrad 1536x8960x8192")
+@pytest.mark.parametrize("m,n,k", PAIR_SHAPES)
+@pytest.mark.parametrize("layout", [oracle.FWD, oracle.DGRAD, oracle.WGRAD])
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_both_kernels(m, n, k, layout, pair, monkeypatch):
+    monkeypatch.setenv("FP8BLK_GEMM_PAIR", pair)
+    rng = np.random.default_rng(m + 5 * n + 11 * k + layout)
+    if layout == oracle.WGRAD:     # dW [m x n] = dY^T [m x k-tokens] . X [k-tokens x n]
+        a_src = workloads.grad_output(rng, k, m)
+        b_src = workloads.swiglu_like(rng, k, n)
+    elif layout == oracle.DGRAD:   # dX [m x n] = dY [m x k] . W [k x n]
+        a_src = workloads.grad_output(rng, m, k)
+        b_src = workloads.weight(rng, k, n)
+    else:
+        a_src = workloads.activation_with_outliers(rng, m, k, frac=0.01)
+        b_src = workloads.weight(rng, n, k)
+    got, ref = _run(layout, *_operands(layout, a_src, b_src))
+    assert_gemm_close(got, ref, f"layout {layout} {m}x{n}x{k} pair={pair}")

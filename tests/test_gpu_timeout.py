@@ -34,9 +34,11 @@ def _operands(layout):
     return qa, sa, qb, sb
 
 
-@pytest.mark.parametrize("layout", [0, 2])   # both thread layouts of the GEMM kernel
-def test_stalled_gemm_reports_timeout_and_recovers(layout, monkeypatch):
+@pytest.mark.parametrize("layout", [0, 2])   # per-block and per-column B scales
+@pytest.mark.parametrize("pair", ["0", "1"])  # the 1-CTA kernel and the CTA-pair kernel
+def test_stalled_gemm_reports_timeout_and_recovers(layout, pair, monkeypatch):
     require_cuda()
+    monkeypatch.setenv("FP8BLK_GEMM_PAIR", pair)
     qa, sa, qb, sb = _operands(layout)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
     A, B = dev(qa).view(torch.float8_e4m3fn), dev(qb).view(torch.float8_e4m3fn)
