@@ -44,16 +44,33 @@ E4M3 = torch.float8_e4m3fn
 E5M2_DTYPE = torch.float8_e5m2
 
 
-def _stream_handle(stream) -> ctypes.c_void_p:
+def _stream_handle(stream, device=None) -> ctypes.c_void_p:
+    """The cudaStream_t to launch on: `stream`, else the current stream of `device`."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return ctypes.c_void_p(stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream))
 
 
-def _need_cuda(*tensors):
+def _need_cuda(*tensors) -> torch.device:
+    """All given tensors must be CUDA tensors of one device; returns it."""
+    dev = None
     for t in tensors:
-        if t is not None and not t.is_cuda:
+        if t is None:
+            continue
+        if not t.is_cuda:
             raise ValueError("fp8blk runs on CUDA tensors only (no CPU fallback)")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors on different devices: {dev} and {t.device}")
+    return dev
+
+
+def _run(device, fn, *args) -> None:
+    """Calls a C entry point with `device` current, so that the library's device
+    check, its per-device state and the launch all refer to the tensors' GPU."""
+    with torch.cuda.device(device):
+        check(fn(*args))
 
 
 def _out(t, shape, dtype, device):
@@ -79,7 +96,7 @@ def fp8blk_quantize_act_1x128(x, mode=ROWWISE, q_row=None, s_row=None, q_colT=No
     """Activation quantisation in 1x128 groups.  Returns (q_row, s_row, q_colT, s_colT); unused are None.
     ``mode`` may include E5M2 (codes as torch.float8_e5m2, for gradients)."""
     x = _bf16_2d(x)
-    _need_cuda(x)
+    dev = _need_cuda(x)
     rows, cols = x.shape
     dev = x.device
     code_dtype = E5M2_DTYPE if mode & E5M2 else E4M3
@@ -93,52 +110,52 @@ def fp8blk_quantize_act_1x128(x, mode=ROWWISE, q_row=None, s_row=None, q_colT=No
         s_colT = _out(s_colT, (rows // 128, cols), torch.float32, dev)
     else:
         q_colT = s_colT = None
-    check(lib.fp8blk_quantize_act_1x128(_ptr(x), rows, cols, x.stride(0), int(mode), _ptr(q_row), _ptr(s_row),
-                                        _ptr(q_colT), _ptr(s_colT), _stream_handle(stream)))
+    _run(dev, lib.fp8blk_quantize_act_1x128, _ptr(x), rows, cols, x.stride(0), int(mode), _ptr(q_row), _ptr(s_row),
+                                        _ptr(q_colT), _ptr(s_colT), _stream_handle(stream, dev))
     return q_row, s_row, q_colT, s_colT
 
 
 def fp8blk_quantize_weight_128x128(w, q=None, s=None, stream=None):
     """Weight quantisation in 128x128 blocks.  Returns (q[N,K], s[N/128,K/128])."""
     w = _bf16_2d(w)
-    _need_cuda(w)
+    dev = _need_cuda(w)
     n, k = w.shape
     q = _out(q, (n, k), E4M3, w.device)
     s = _out(s, (n // 128, k // 128), torch.float32, w.device)
-    check(lib.fp8blk_quantize_weight_128x128(_ptr(w), n, k, w.stride(0), _ptr(q), _ptr(s), _stream_handle(stream)))
+    _run(dev, lib.fp8blk_quantize_weight_128x128, _ptr(w), n, k, w.stride(0), _ptr(q), _ptr(s), _stream_handle(stream, dev))
     return q, s
 
 
 def fp8blk_quantize_weight_128x128_t(w, qT=None, sT=None, stream=None):
     """The same blocks written transposed.  Returns (qT[K,N], sT[K/128,N/128])."""
     w = _bf16_2d(w)
-    _need_cuda(w)
+    dev = _need_cuda(w)
     n, k = w.shape
     qT = _out(qT, (k, n), E4M3, w.device)
     sT = _out(sT, (k // 128, n // 128), torch.float32, w.device)
-    check(lib.fp8blk_quantize_weight_128x128_t(_ptr(w), n, k, w.stride(0), _ptr(qT), _ptr(sT),
-                                               _stream_handle(stream)))
+    _run(dev, lib.fp8blk_quantize_weight_128x128_t, _ptr(w), n, k, w.stride(0), _ptr(qT), _ptr(sT),
+                                               _stream_handle(stream, dev))
     return qT, sT
 
 
 def fp8blk_quantize_weight_128x128_both(w, q=None, s=None, qT=None, sT=None, stream=None):
     """Both block layouts from one read of w.  Returns (q[N,K], s[N/128,K/128], qT[K,N], sT[K/128,N/128])."""
     w = _bf16_2d(w)
-    _need_cuda(w)
+    dev = _need_cuda(w)
     n, k = w.shape
     q = _out(q, (n, k), E4M3, w.device)
     s = _out(s, (n // 128, k // 128), torch.float32, w.device)
     qT = _out(qT, (k, n), E4M3, w.device)
     sT = _out(sT, (k // 128, n // 128), torch.float32, w.device)
-    check(lib.fp8blk_quantize_weight_128x128_both(_ptr(w), n, k, w.stride(0), _ptr(q), _ptr(s), _ptr(qT), _ptr(sT),
-                                                  _stream_handle(stream)))
+    _run(dev, lib.fp8blk_quantize_weight_128x128_both, _ptr(w), n, k, w.stride(0), _ptr(q), _ptr(s), _ptr(qT), _ptr(sT),
+                                                  _stream_handle(stream, dev))
     return q, s, qT, sT
 
 
 def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None, out_dtype=torch.bfloat16):
     """Blockwise-scaled E4M3 GEMM, D[M,N] = dequant(A) . dequant(B)^T in bf16 (or, with
     out_dtype=torch.float32 or an fp32 d, the unrounded fp32 sums)."""
-    _need_cuda(a, sa, b, sb, d)
+    dev = _need_cuda(a, sa, b, sb, d)
     m, k = a.shape
     n = b.shape[0]
     if b.shape[1] != k:
@@ -158,18 +175,18 @@ def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None, out_dtype=torch.bfloa
         raise ValueError("d must be a bfloat16 or float32 [M,N] tensor with unit column stride")
     flags = (A_E5M2 if a.dtype == E5M2_DTYPE else 0) | (B_E5M2 if b.dtype == E5M2_DTYPE else 0)
     flags |= OUT_F32 if d.dtype == torch.float32 else 0
-    check(lib.fp8blk_gemm(int(layout) | flags, m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d), d.stride(0),
-                          _stream_handle(stream)))
+    _run(dev, lib.fp8blk_gemm, int(layout) | flags, m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d), d.stride(0),
+                          _stream_handle(stream, dev))
     return d
 
 
 def fp8blk_round_f32_to_bf16(x, y=None, stream=None):
     """y = bf16(x) (round to nearest even), elementwise; x a contiguous float32 CUDA tensor."""
-    _need_cuda(x, y)
+    dev = _need_cuda(x, y)
     if x.dtype != torch.float32 or not x.is_contiguous():
         raise ValueError("x must be a contiguous float32 tensor")
     y = _out(y, tuple(x.shape), torch.bfloat16, x.device)
-    check(lib.fp8blk_round_f32_to_bf16(_ptr(x), x.numel(), _ptr(y), _stream_handle(stream)))
+    _run(dev, lib.fp8blk_round_f32_to_bf16, _ptr(x), x.numel(), _ptr(y), _stream_handle(stream, dev))
     return y
 
 
@@ -181,7 +198,7 @@ def fp8blk_amax_ema(x, amax, scale=None, workspace=None, stream=None):
     """Per-tensor delayed scaling: update the amax buffer (float32 [1], in place) from max|x| by the
     EMA and write the tensor's scale.  Returns (amax, scale)."""
     x = _bf16_2d(x)
-    _need_cuda(x, amax)
+    dev = _need_cuda(x, amax, scale, workspace)
     rows, cols = x.shape
     if amax.dtype != torch.float32 or amax.numel() != 1:
         raise ValueError("amax must be a float32 tensor with one element")
@@ -189,8 +206,8 @@ def fp8blk_amax_ema(x, amax, scale=None, workspace=None, stream=None):
     need = fp8blk_amax_ema_workspace_bytes(rows)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
-    check(lib.fp8blk_amax_ema(_ptr(x), rows, cols, x.stride(0), _ptr(amax), _ptr(scale), _ptr(workspace),
-                              workspace.numel() * workspace.element_size(), _stream_handle(stream)))
+    _run(dev, lib.fp8blk_amax_ema, _ptr(x), rows, cols, x.stride(0), _ptr(amax), _ptr(scale), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream_handle(stream, dev))
     return amax, scale
 
 
@@ -204,37 +221,37 @@ def fp8blk_amax_ema_static(x, amax, scale, stream=None):
     x = _bf16_2d(x)
     if scale is None:
         raise ValueError("scale is required: this entry point allocates nothing")
-    _need_cuda(x, amax, scale)
+    dev = _need_cuda(x, amax, scale)
     rows, cols = x.shape
     for t, name in ((amax, "amax"), (scale, "scale")):
         if t.dtype != torch.float32 or t.numel() != 1:
             raise ValueError(f"{name} must be a float32 tensor with one element")
-    check(lib.fp8blk_amax_ema_static(_ptr(x), rows, cols, x.stride(0), _ptr(amax), _ptr(scale),
-                                     _stream_handle(stream)))
+    _run(dev, lib.fp8blk_amax_ema_static, _ptr(x), rows, cols, x.stride(0), _ptr(amax), _ptr(scale),
+                                     _stream_handle(stream, dev))
     return amax, scale
 
 
 def fp8blk_quantize_tensor(x, scale, q=None, stream=None):
     """The whole tensor with its one scale (device float32 [1]).  Returns q [rows, cols] E4M3."""
     x = _bf16_2d(x)
-    _need_cuda(x, scale)
+    dev = _need_cuda(x, scale, q)
     rows, cols = x.shape
     q = _out(q, (rows, cols), E4M3, x.device)
-    check(lib.fp8blk_quantize_tensor(_ptr(x), rows, cols, x.stride(0), _ptr(scale), _ptr(q), _stream_handle(stream)))
+    _run(dev, lib.fp8blk_quantize_tensor, _ptr(x), rows, cols, x.stride(0), _ptr(scale), _ptr(q), _stream_handle(stream, dev))
     return q
 
 
 def fp8blk_gemm_tensor_scaled(a, sa, b, sb, d=None, stream=None):
     """D[M,N] = bf16(sa * sb * A . B^T) with one scale per E4M3 operand (device float32 [1] each)."""
-    _need_cuda(a, sa, b, sb, d)
+    dev = _need_cuda(a, sa, b, sb, d)
     m, k = a.shape
     n = b.shape[0]
     if b.shape[1] != k or a.dtype != E4M3 or b.dtype != E4M3:
         raise ValueError("A [M,K] and B [N,K] must be float8_e4m3fn")
     if d is None:
         d = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
-    check(lib.fp8blk_gemm_tensor_scaled(m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d), d.stride(0),
-                                        _stream_handle(stream)))
+    _run(dev, lib.fp8blk_gemm_tensor_scaled, m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d), d.stride(0),
+                                        _stream_handle(stream, dev))
     return d
 
 

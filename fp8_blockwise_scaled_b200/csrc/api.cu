@@ -77,6 +77,11 @@ int pdl_enabled() {
   return e ? std::atoi(e) != 0 : 0;
 }
 
+int env_int(const char* name, int fallback) {
+  const char* e = std::getenv(name);
+  return e ? std::atoi(e) : fallback;
+}
+
 // Bounded device waits of a quantiser launch (and the stall test hook).
 fp8blk_status set_quant_waits(QuantArgs& a) {
   a.timeout_ns = wait_timeout_ns();
@@ -85,6 +90,7 @@ fp8blk_status set_quant_waits(QuantArgs& a) {
   a.inject_stall = 0;
   if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) a.inject_stall = std::atoi(e) != 0;
   a.pdl = pdl_enabled();
+  a.max_ctas = env_int("FP8BLK_QUANT_MAX_CTAS", 0);
   return FP8BLK_OK;
 }
 
@@ -203,6 +209,7 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   g.a_e5m2 = (formats & FP8BLK_A_E5M2) != 0;
   g.b_e5m2 = (formats & FP8BLK_B_E5M2) != 0;
   if (const char* e = std::getenv("FP8BLK_GEMM_PAIR")) g.pair = std::atoi(e);
+  g.max_ctas = env_int("FP8BLK_GEMM_MAX_CTAS", 0);
   if (const char* e = std::getenv("FP8BLK_GEMM_GROUP_M")) g.group_m = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) g.inject_stall = std::atoi(e) != 0;
@@ -281,6 +288,7 @@ fp8blk_status fp8blk_gemm_tensor_scaled(int64_t M, int64_t N, int64_t K, const u
   g.pdl = pdl_enabled();
   g.tensor_sa = sa;
   g.tensor_sb = sb;
+  g.max_ctas = env_int("FP8BLK_GEMM_MAX_CTAS", 0);
   if (const char* e = std::getenv("FP8BLK_GEMM_GROUP_M")) g.group_m = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) g.inject_stall = std::atoi(e) != 0;
   return launch_status(fp8blk::launch_gemm(g, static_cast<cudaStream_t>(stream)));

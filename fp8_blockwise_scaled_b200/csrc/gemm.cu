@@ -26,12 +26,14 @@
 //   warps 4-11  promotion + epilogue, two warpgroups each owning half of the
 //               tile's columns (a warp reads the 32 TMEM lanes its index mod 4
 //               allows).  Warpgroup 0 hands registers to them (setmaxnreg
-//               80 / 208), which pays for 64-column TMEM loads next to the
-//               128 fp32 running sums of a thread.  Per K-block a warp takes
-//               its scales from the ring, waits for the accumulator, reads it
-//               from TMEM in two 64-column loads, hands the buffer back to the
-//               MMA issuer as soon as the last load has landed, and folds the
-//               partial product into its registers with packed f32x2 FMAs:
+//               80 / 208), which pays for two 32-column TMEM loads in flight
+//               next to the 128 fp32 running sums of a thread.  Per K-block a
+//               warp takes its scales from the ring, waits for the
+//               accumulator, reads it from TMEM in 32-column loads (each in
+//               flight while the previous chunk's FMAs run), hands the buffer
+//               back to the MMA issuer as soon as the last load has landed,
+//               and folds the partial product into its registers with packed
+//               f32x2 FMAs:
 //                   FWD/DGRAD: acc += P * (sa[m] * sb[n-block])
 //                   WGRAD    : acc += (P * sb[n]) * sa[m]
 //               after the last K-block it rounds the tile to bf16 and stores
@@ -159,35 +161,25 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_ld_32x32b_x64(uint32_t taddr, uint32_t (&r)[64]) {
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
-      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
-      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
         "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
-        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
-        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
-        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
-        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
 
-// tcgen05.wait::ld tied to all 64 registers of a 64-column load.
-__device__ __forceinline__ void tmem_wait_ld64(uint32_t (&r)[64]) {
+// tcgen05.wait::ld tied to all 32 registers of a 32-column load.
+__device__ __forceinline__ void tmem_wait_ld32(uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;"
                : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
                  "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
                  "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
-                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]),
-                 "+r"(r[32]), "+r"(r[33]), "+r"(r[34]), "+r"(r[35]), "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]),
-                 "+r"(r[40]), "+r"(r[41]), "+r"(r[42]), "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]),
-                 "+r"(r[48]), "+r"(r[49]), "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]),
-                 "+r"(r[56]), "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]), "+r"(r[63])
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
                :
                : "memory");
 }
@@ -295,16 +287,25 @@ __device__ __forceinline__ bool promote_tile(Ctrl* ctrl, const GemmParams& p, fl
     tc_fence_after_sync();
     const uint32_t taddr = tmem_lanes + tbuf.idx * BN;
     const float* sbc = ss.sb + col0;
+    // 32-column TMEM loads, each in flight while the FMAs of the previous
+    // chunk run; the buffer goes back to the MMA issuer as soon as the last
+    // load has landed, before the FMAs that consume it.
+    uint32_t ra[32], rb[32];
+    tmem_ld_32x32b_x32(taddr, ra);
+    tmem_wait_ld32(ra);
 #pragma unroll
     for (int c = 0; c < kCols; c += 64) {
-      uint32_t r[64];
-      tmem_ld_32x32b_x64(taddr + c, r);
-      tmem_wait_ld64(r);
-      // The buffer goes back to the MMA issuer as soon as this warp's last
-      // TMEM load has landed, before the FMAs that consume it.
-      if (c + 64 == kCols) release(tbuf.idx);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) promote16<kWgrad>(acc + c / 2 + 8 * q, r + 16 * q, f, sbc + c + 16 * q, sa);
+      tmem_ld_32x32b_x32(taddr + c + 32, rb);
+      promote16<kWgrad>(acc + c / 2, ra, f, sbc + c, sa);
+      promote16<kWgrad>(acc + c / 2 + 8, ra + 16, f, sbc + c + 16, sa);
+      tmem_wait_ld32(rb);
+      if (c + 64 < kCols)
+        tmem_ld_32x32b_x32(taddr + c + 64, ra);
+      else
+        release(tbuf.idx);
+      promote16<kWgrad>(acc + c / 2 + 16, rb, f, sbc + c + 32, sa);
+      promote16<kWgrad>(acc + c / 2 + 24, rb + 16, f, sbc + c + 48, sa);
+      if (c + 64 < kCols) tmem_wait_ld32(ra);
     }
     if constexpr (kWgrad) {
       __syncwarp();                        // the column scales were read during the FMAs
@@ -890,13 +891,18 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
     return e;
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BN)) return cudaErrorInvalidValue;
+  // Tile order: groups of 8 M-blocks; with at most 16 M-blocks (the weight
+  // gradients of the narrow layers, M = out features) one group holds them
+  // all, so every B column block is streamed once while all M-blocks use it.
   const int num_mb = static_cast<int>(g.M / BM);
-  int group_m = g.group_m > 0 ? g.group_m : 8;
+  int group_m = g.group_m > 0 ? g.group_m : (num_mb <= 16 ? num_mb : 8);
   if (group_m > num_mb) group_m = num_mb;
   GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.out_f32, g.timeout_ns, g.err, g.inject_stall, group_m,
                fmt_bits(g), g.tensor_sa, g.tensor_sb};
   const int64_t tiles = (g.M / BM) * (g.N / BN);
-  const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
+  int64_t ctas = num_sms();
+  if (g.max_ctas > 0 && g.max_ctas < ctas) ctas = g.max_ctas;
+  const int grid = static_cast<int>(tiles < ctas ? tiles : ctas);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -920,7 +926,8 @@ cudaError_t launch_pair(const GemmArgs& g, cudaStream_t stream) {
   GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.out_f32, g.timeout_ns, g.err, g.inject_stall, 0, fmt_bits(g),
                nullptr, nullptr};
   const int64_t tiles = (g.M / (2 * BM)) * (g.N / kPairBN);
-  const int64_t max_pairs = num_sms() / 2;
+  int64_t max_pairs = num_sms() / 2;
+  if (g.max_ctas > 1 && g.max_ctas / 2 < max_pairs) max_pairs = g.max_ctas / 2;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);

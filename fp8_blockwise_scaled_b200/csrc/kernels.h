@@ -23,6 +23,7 @@ struct QuantArgs {
   int inject_stall;      // test hook: the consumers wait on a barrier nothing completes
   unsigned int* err;     // device error word
   int pdl;               // 1 = launch with programmatic stream serialization
+  int max_ctas;          // > 0: at most this many CTAs (leaves SMs to concurrent work)
 };
 
 cudaError_t launch_quant(int mode, const QuantArgs& a, cudaStream_t stream);
@@ -63,6 +64,7 @@ struct GemmArgs {
   int pair;                   // 1 = use 256 x 256 pair tiles when the shape allows, 0 = never
   int group_m;                // tile order: M-blocks per group (0 = default)
   int pdl;                    // 1 = launch with programmatic stream serialization
+  int max_ctas;               // > 0: at most this many CTAs (leaves SMs to concurrent work)
   int a_e5m2, b_e5m2;         // 1 = that operand holds E5M2 codes (else E4M3)
   const float* tensor_sa;     // non-null: one scale per operand (device scalars), no per-block scales
   const float* tensor_sb;

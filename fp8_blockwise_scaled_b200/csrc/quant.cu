@@ -382,6 +382,7 @@ cudaError_t launch_mode(const QuantArgs& a, cudaStream_t stream) {
   CUtensorMap map;
   if (!make_input_map(&map, a)) return cudaErrorInvalidValue;
   const int64_t tiles = a.tiles_r * a.tiles_c;
+  if (a.max_ctas > 0 && a.max_ctas < grid_cap) grid_cap = a.max_ctas;
   const int grid = static_cast<int>(tiles < grid_cap ? tiles : grid_cap);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);

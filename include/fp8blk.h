@@ -45,6 +45,11 @@
  *      FP8BLK_GEMM_PAIR           1: 256x256 tiles on CTA pairs wherever M and
  *                                 N are multiples of 256; 0: never (default)
  *      FP8BLK_GEMM_GROUP_M        M-blocks per group of the GEMM tile order
+ *      FP8BLK_GEMM_MAX_CTAS       at most this many GEMM CTAs (one per SM), so
+ *                                 that concurrent work on other streams finds
+ *                                 free SMs (default: one per SM)
+ *      FP8BLK_QUANT_MAX_CTAS      the same for the quantisers (default: as many
+ *                                 as fit, two per SM)
  *      FP8BLK_TEST_INJECT_STALL=1 tests only: one wait of the next launch
  *                                 never completes, so that the bounded-wait
  *                                 error path runs
