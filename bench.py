@@ -374,6 +374,26 @@ def cpu_baseline(specs) -> dict:
 
 
 # --------------------------------------------------------------------------- extra measurements
+def host_enqueue_seconds(prog) -> float:
+    """Host time to enqueue one step (every launch of the program), measured once."""
+    import torch
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    prog.run(reduce=False)
+    t = time.perf_counter() - t0
+    torch.cuda.synchronize()
+    return t
+
+
+def hold_device(host_seconds: float) -> None:
+    """Keeps the stream busy (a spin kernel) for about twice the host's enqueue time of a step,
+    so that the per-op events recorded next measure the kernels back to back on the device,
+    without the host's launch gaps.  The spin counts clock cycles; 2e9 per second is above the
+    B200's maximum SM clock, so the spin lasts at least that long."""
+    import torch
+    torch.cuda._sleep(int(2.0 * host_seconds * 2.0e9) + 100000)
+
+
 def time_program(prog, flush, steps: int, warmup: int) -> dict:
     """Median per-op event times of eager launches, and the median device time of the
     whole step replayed as one CUDA graph (L2 flushed before every step)."""
@@ -382,10 +402,12 @@ def time_program(prog, flush, steps: int, warmup: int) -> dict:
         flush.zero_()
         prog.run(reduce=False)
     torch.cuda.synchronize()
+    ahead = host_enqueue_seconds(prog)
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in prog.ops]
           for _ in range(steps)]
     for i in range(steps):
         flush.zero_()
+        hold_device(ahead)
         prog.run(ev[i], reduce=False)
     torch.cuda.synchronize()
     op_ms = [statistics.median(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(steps))
@@ -535,9 +557,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nops)]
           for _ in range(args.steps)]
     st = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    # Per-op device times: eager launches, one event pair around each op.
+    # Per-op device times: eager launches, one event pair around each op, the whole step
+    # enqueued behind a spin kernel so that the kernels run back to back on the device.
+    ahead = host_enqueue_seconds(prog)
     for i in range(args.steps):
         flush.zero_()
+        hold_device(ahead)
         prog.run(ev[i], reduce=False)
     barrier()
     per_op_ms = [[a.elapsed_time(b) for a, b in ev[i]] for i in range(args.steps)]
@@ -697,6 +722,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "note": "quantisers on a second stream; each GEMM waits for the quantisers it reads",
             "partitioned": partitioned},
         "per_op_median": per_op,
+        "per_op_timing": "CUDA events around each eager launch, the step enqueued behind a spin kernel "
+                         "(kernels back to back on the device, no host launch gaps); L2 flushed once per step",
         "e2e": {"value": flops_all * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         # one kernel per op, two for an amax EMA (partial maxima, then the EMA), and with

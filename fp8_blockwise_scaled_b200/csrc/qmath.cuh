@@ -87,6 +87,15 @@ __device__ __forceinline__ void neg_quotient2(float& w0, float& w1, float x0, fl
   w1 = w.y;
 }
 
+// The same for a pair whose elements have their own scales: w.i = -RN(x.i /
+// s.i) with nr.i = -RN(1/s.i) (two rows of a column, each with its row's
+// scale, or one scale twice).
+__device__ __forceinline__ float2 neg_quotient2(float2 x, float2 s, float2 nr) {
+  const float2 qn = __fmul2_rn(x, nr);
+  const float2 e = __ffma2_rn(qn, s, x);
+  return __ffma2_rn(e, nr, qn);
+}
+
 // Eight values -> eight codes packed little-endian (x[0] in the lowest byte).
 template <bool kE5>
 __device__ __forceinline__ uint2 quant8(const float (&x)[8], const QScale& q) {

@@ -68,7 +68,7 @@ struct QCtrl {
   int abort;
   float warpmax[2][8];                   // per-warp block maxima, double-buffered by tile parity
   alignas(16) float2 qs[kTile];          // per-column {s, -1/s}
-  alignas(16) float2 rq[8][2][8];        // per half-warp: {s, -1/s} of its 8 rows
+  alignas(16) float4 rq[8][2][4];        // per half-warp, row pair p: {s_2p, s_2p+1, -1/s_2p, -1/s_2p+1}
   alignas(16) uint32_t cpart[8 * 64];    // per-warp packed column maxima (16-byte stores)
 };
 static_assert(sizeof(QCtrl) % 16 == 0, "QCtrl keeps 16-byte alignment");
@@ -127,15 +127,28 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
 
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
-  const int64_t tiles = a.tiles_r * a.tiles_c;
-  auto load_tile = [&](int stage, int64_t tile) {
-    const int64_t tr = tile % a.tiles_r, tc = tile / a.tiles_r;
+  // Tile j covers rows 128 (j % tiles_r) .. and columns 128 (j / tiles_r) ..;
+  // a CTA's tiles are gridDim.x apart, so their coordinates advance by fixed
+  // steps (32-bit: the host rejects 2^31 tiles or more).
+  const uint32_t tiles_r = static_cast<uint32_t>(a.tiles_r);
+  const uint32_t tiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
+  const uint32_t step_r = gridDim.x % tiles_r, step_c = gridDim.x / tiles_r;
+  auto advance = [&](uint32_t& tr, uint32_t& tc) {
+    tr += step_r;
+    tc += step_c;
+    if (tr >= tiles_r) {
+      tr -= tiles_r;
+      ++tc;
+    }
+  };
+  auto load_tile = [&](int stage, uint32_t tr, uint32_t tc) {
     mbar_arrive_expect_tx(&ctrl->full[stage], kTileBytes);
     tma_load_2d(smem + stage * kTileBytes, &tm_x, &ctrl->full[stage], static_cast<int>(tc * kTile),
                 static_cast<int>(tr * kTile));
   };
 
-  int64_t issued = 0;   // loads issued (thread 0 only)
+  uint32_t issued = 0;                                            // loads issued (thread 0 only)
+  uint32_t ltr = blockIdx.x % tiles_r, ltc = blockIdx.x / tiles_r;   // the next tile to load
   if (t == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&ctrl->full[s], 1);
@@ -146,7 +159,10 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
     fence_mbar_init();
     tma_prefetch_map(&tm_x);
     griddep_wait();                              // the input may come from the previous kernel
-    for (int64_t tile = blockIdx.x; issued < S && tile < tiles; tile += gridDim.x) load_tile(issued++, tile);
+    for (uint32_t j = blockIdx.x; issued < static_cast<uint32_t>(S) && j < tiles; j += gridDim.x) {
+      load_tile(static_cast<int>(issued++), ltr, ltc);
+      advance(ltr, ltc);
+    }
   }
   __syncthreads();
   griddep_wait();                                // before any global write
@@ -163,18 +179,20 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
   const int bi = 2 * warp + (lane >> 4);
   const uint32_t cols = static_cast<uint32_t>(a.cols);
   const uint32_t rows = static_cast<uint32_t>(a.rows);
-  float2* rq = ctrl->rq[warp][lane >> 4];
+  float4* rq = ctrl->rq[warp][lane >> 4];
 
-  int64_t it = 0;
-  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+  uint32_t it = 0;
+  uint32_t tr = blockIdx.x % tiles_r, tc = blockIdx.x / tiles_r;
+  for (uint32_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it, advance(tr, tc)) {
     const int s = static_cast<int>(it % S);
-    const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-    bool ok = a.inject_stall ? mbar_wait_bounded(&ctrl->never, 0, abort, a.timeout_ns, a.err)
-                             : mbar_wait_bounded(&ctrl->full[s], ph, abort, a.timeout_ns, a.err);
+    const uint32_t ph = (it / S) & 1;
+    // Waits on the critical path: polled without the suspend hint (a
+    // completed phase is seen sooner).
+    bool ok = a.inject_stall ? mbar_wait_bounded<false>(&ctrl->never, 0, abort, a.timeout_ns, a.err)
+                             : mbar_wait_bounded<false>(&ctrl->full[s], ph, abort, a.timeout_ns, a.err);
     if (!consumers_all(ok)) break;
 
-    const int64_t tr = tile % a.tiles_r, tc = tile / a.tiles_r;
-    const int64_t row0 = tr * kTile, col0 = tc * kTile;
+    const int64_t row0 = static_cast<int64_t>(tr) * kTile, col0 = static_cast<int64_t>(tc) * kTile;
     uint4 v[8];
     {
       const uint8_t* xs = smem + s * kTileBytes + (8 * bi) * 256 + bj * 16;   // conflict-free: 2 rows per warp
@@ -184,12 +202,13 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
     __syncwarp();                                // everything else comes from registers: hand the stage back
     if (lane == 0) mbar_arrive(&ctrl->empty[s]);
     if (t == 0) {                                // and refill it with the tile S steps ahead
-      const int64_t next = tile + static_cast<int64_t>(S) * gridDim.x;
-      if (next < tiles && mbar_wait_bounded(&ctrl->empty[s], ph, abort, a.timeout_ns, a.err)) {
+      if (tile + static_cast<uint32_t>(S) * gridDim.x < tiles &&
+          mbar_wait_bounded<false>(&ctrl->empty[s], ph, abort, a.timeout_ns, a.err)) {
         // The warps read the stage through the generic proxy; the TMA load
         // rewrites it through the async proxy: order the two.
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        load_tile(s, next);
+        load_tile(s, ltr, ltc);
+        advance(ltr, ltc);
         ++issued;
       }
     }
@@ -237,8 +256,10 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
       const int rho = (lane >> 1) & 7;             // = 4 b + 2 c + d
       const QScale q = make_qscale<kE5>(__uint_as_float(d ? (k & 0xFFFF0000u) : (k << 16)));
       if ((lane & 1) == 0) {
-        rq[rho] = make_float2(q.s, q.nr);
-        a.s_row[tc * a.rows + row0 + 8 * bi + rho] = q.s;
+        float* rp = reinterpret_cast<float*>(&rq[rho >> 1]);
+        rp[rho & 1] = q.s;
+        rp[2 + (rho & 1)] = q.nr;
+        a.s_row[static_cast<int64_t>(tc) * a.rows + row0 + 8 * bi + rho] = q.s;
       }
       __syncwarp();
     }
@@ -256,8 +277,8 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
       for (int w = 1; w < kConsumers / 32; ++w) amax = fmaxf(amax, wm[w]);
       qblk = make_qscale<kE5>(amax);
       if (t == 0) {
-        if constexpr (kBlk) a.s_row[tr * a.tiles_c + tc] = qblk.s;
-        if constexpr (kBlkT) a.s_t[tc * a.tiles_r + tr] = qblk.s;
+        if constexpr (kBlk) a.s_row[static_cast<int64_t>(tr) * a.tiles_c + tc] = qblk.s;
+        if constexpr (kBlkT) a.s_t[static_cast<int64_t>(tc) * a.tiles_r + tr] = qblk.s;
       }
     }
 
@@ -273,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
         for (int w = 0; w < 8; ++w) mx = __vmaxu2(mx, ctrl->cpart[w * 64 + (t >> 1)]);
         const QScale q = make_qscale<kE5>(__uint_as_float((t & 1) ? (mx & 0xFFFF0000u) : (mx << 16)));
         ctrl->qs[t] = make_float2(q.s, q.nr);
-        a.s_t[tr * a.cols + col0 + t] = q.s;
+        a.s_t[static_cast<int64_t>(tr) * a.cols + col0 + t] = q.s;
       }
       consumers_sync();                          // the column scales are in
 #pragma unroll
@@ -284,34 +305,56 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
       }
     }
 
-    // Codes, two rows at a time.  In place: one 8-byte store per row (a warp
-    // writes two 128-byte row segments).  Transposed: column c of the tile
-    // collects the codes of rows 8 bi .. 8 bi + 7 in the 8-byte unit bi ^ bj of
-    // its 128-byte line in cs (the XOR spreads a half-warp over all 32 banks).
+    // Codes, two rows at a time.  Column c's values of rows 2p and 2p+1 form
+    // one f32 pair, divided in one packed step by the two row scales (in
+    // place) and by the column scale twice (transposed), so each value is
+    // unpacked once for both layouts.  In place: one 8-byte store per row (a
+    // warp writes two 128-byte row segments).  Transposed: column c of the
+    // tile collects the codes of rows 8 bi .. 8 bi + 7 in the 8-byte unit
+    // bi ^ bj of its 128-byte line in cs (the XOR spreads a half-warp over all
+    // 32 banks).
     [[maybe_unused]] uint8_t* qdst = kRow || kBlk ? a.q_row + (row0 + 8 * bi) * a.cols + col0 + 8 * bj : nullptr;
     [[maybe_unused]] uint32_t pend[8];             // transposed: codes of the previous row pair, per column
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      float f0[8], f1[8];
-      unpack8(v[2 * p], f0);
-      unpack8(v[2 * p + 1], f1);
+      float2 x[8];
+      {
+        const uint4 a0 = v[2 * p], a1 = v[2 * p + 1];
+        x[0] = make_float2(bf16lo(a0.x), bf16lo(a1.x));
+        x[1] = make_float2(bf16hi(a0.x), bf16hi(a1.x));
+        x[2] = make_float2(bf16lo(a0.y), bf16lo(a1.y));
+        x[3] = make_float2(bf16hi(a0.y), bf16hi(a1.y));
+        x[4] = make_float2(bf16lo(a0.z), bf16lo(a1.z));
+        x[5] = make_float2(bf16hi(a0.z), bf16hi(a1.z));
+        x[6] = make_float2(bf16lo(a0.w), bf16lo(a1.w));
+        x[7] = make_float2(bf16hi(a0.w), bf16hi(a1.w));
+      }
       if constexpr (kRow || kBlk) {
-        QScale q0 = qblk, q1 = qblk;
+        float2 s2, nr2;
         if constexpr (kRow) {
-          const float4 f = *reinterpret_cast<const float4*>(&rq[2 * p]);
-          q0 = QScale{f.x, f.y};
-          q1 = QScale{f.z, f.w};
+          const float4 f = rq[p];
+          s2 = make_float2(f.x, f.y);
+          nr2 = make_float2(f.z, f.w);
+        } else {
+          s2 = make_float2(qblk.s, qblk.s);
+          nr2 = make_float2(qblk.nr, qblk.nr);
         }
-        *reinterpret_cast<uint2*>(qdst + (2 * p) * cols) = quant8<kE5>(f0, q0);
-        *reinterpret_cast<uint2*>(qdst + (2 * p + 1) * cols) = quant8<kE5>(f1, q1);
+        float2 w[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) w[c] = neg_quotient2(x[c], s2, nr2);
+        *reinterpret_cast<uint2*>(qdst + (2 * p) * cols) =
+            make_uint2(cvt4<kE5>(w[0].x, w[1].x, w[2].x, w[3].x) ^ 0x80808080u,
+                       cvt4<kE5>(w[4].x, w[5].x, w[6].x, w[7].x) ^ 0x80808080u);
+        *reinterpret_cast<uint2*>(qdst + (2 * p + 1) * cols) =
+            make_uint2(cvt4<kE5>(w[0].y, w[1].y, w[2].y, w[3].y) ^ 0x80808080u,
+                       cvt4<kE5>(w[4].y, w[5].y, w[6].y, w[7].y) ^ 0x80808080u);
       }
       if constexpr (kTileSmem) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const QScale q = kColT ? cq[c] : qblk;
-          float w0, w1;
-          neg_quotient2(w0, w1, f0[c], f1[c], q.s, q.nr);
-          const uint32_t h = cvt2<kE5>(w0, w1);
+          const float2 w = neg_quotient2(x[c], make_float2(q.s, q.s), make_float2(q.nr, q.nr));
+          const uint32_t h = cvt2<kE5>(w.x, w.y);   // rows 2p (low byte) and 2p+1
           if (p & 1) {
             const uint32_t word = __byte_perm(pend[c], h, 0x5410) ^ 0x80808080u;
             *reinterpret_cast<uint32_t*>(cs + (8 * bj + c) * 128 + ((bi ^ bj) * 8) + (p >> 1) * 4) = word;
@@ -343,8 +386,8 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
   // Thread 0 lets its copies still in flight land before the CTA's shared
   // memory goes away (on the normal path every load has been consumed).
   if (t == 0) {
-    for (int64_t j = it; j < issued; ++j)
-      mbar_wait_bounded(&ctrl->full[j % S], static_cast<uint32_t>((j / S) & 1), nullptr, a.timeout_ns, a.err);
+    for (uint32_t j = it; j < issued; ++j)
+      mbar_wait_bounded(&ctrl->full[j % S], (j / S) & 1, nullptr, a.timeout_ns, a.err);
   }
 }
 
@@ -382,6 +425,7 @@ cudaError_t launch_mode(const QuantArgs& a, cudaStream_t stream) {
   CUtensorMap map;
   if (!make_input_map(&map, a)) return cudaErrorInvalidValue;
   const int64_t tiles = a.tiles_r * a.tiles_c;
+  if (tiles >= (int64_t{1} << 31)) return cudaErrorInvalidValue;   // the kernel counts tiles in 32 bits
   if (a.max_ctas > 0 && a.max_ctas < grid_cap) grid_cap = a.max_ctas;
   const int grid = static_cast<int>(tiles < grid_cap ? tiles : grid_cap);
   cudaLaunchConfig_t cfg = {};
