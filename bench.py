@@ -118,6 +118,7 @@ class Program:
         self.outputs = []      # device tensors read back by the end-to-end run
         self.grads = []        # weight gradients all-reduced across ranks
         self.named = {}        # "<linear>.<buffer>" -> device tensor (the parity tests read them)
+        self.splits = {}       # GEMM label -> split-K count the library chose (1 = none)
         self.gemm_flops = 0
         E4 = torch.float8_e4m3fn
         if recipe == "delayed":
@@ -162,8 +163,7 @@ class Program:
             if "fwd" in passes:
                 y = torch.empty(T, N, dtype=torch.bfloat16, device=device)
                 self.named[f"{g}.Y"] = y
-                self._op(f"{g}.gemm_fwd", "gemm", 2 * T * N * K,
-                         lambda a=qx, sa=sx, b=qw, sb=sw, d=y: fb.fp8blk_gemm(fb.FWD, a, sa, b, sb, d))
+                self._gemm_op(f"{g}.gemm_fwd", fb.FWD, qx, sx, qw, sw, y)
                 self.outputs.append(y)
             if "dgrad" in passes or "wgrad" in passes:
                 dy = self._dev(sp["dY"], device)
@@ -183,16 +183,14 @@ class Program:
                 if need_row_d:
                     dx = torch.empty(T, K, dtype=torch.bfloat16, device=device)
                     self.named[f"{g}.dX"] = dx
-                    self._op(f"{g}.gemm_dgrad", "gemm", 2 * T * N * K,
-                             lambda a=qd, sa=sd, b=qwT, sb=swT, d=dx: fb.fp8blk_gemm(fb.DGRAD, a, sa, b, sb, d))
+                    self._gemm_op(f"{g}.gemm_dgrad", fb.DGRAD, qd, sd, qwT, swT, dx)
                     self.outputs.append(dx)
                 if need_colt_d:
                     dw = torch.empty(N, K, dtype=torch.bfloat16, device=device)
                     self.named[f"{g}.dW"] = dw
                     # Data parallel: this rank's partial dW in fp32, summed across ranks, rounded once.
                     part = torch.empty(N, K, dtype=torch.float32, device=device) if world > 1 else dw
-                    self._op(f"{g}.gemm_wgrad", "gemm", 2 * T * N * K,
-                             lambda a=qdT, sa=sdT, b=qxT, sb=sxT, d=part: fb.fp8blk_gemm(fb.WGRAD, a, sa, b, sb, d))
+                    self._gemm_op(f"{g}.gemm_wgrad", fb.WGRAD, qdT, sdT, qxT, sxT, part)
                     self.outputs.append(dw)
                     if world > 1:
                         self.grads.append((part, dw))
@@ -232,6 +230,17 @@ class Program:
 
     def _op(self, label, kind, units, fn):
         self.ops.append((label, kind, units, fn))
+
+    def _gemm_op(self, label, layout, a, sa, b, sb, d):
+        """One blockwise GEMM op, split-K where the library's count for the shape says so (its
+        fp32 partial-tile workspace allocated here, once)."""
+        fb, torch = self.fb, self.torch
+        m, n, k = d.shape[0], d.shape[1], a.shape[1]
+        splits = fb.fp8blk_gemm_splitk_count(layout, m, n, k)
+        ws = torch.empty(splits * m * n, dtype=torch.float32, device=d.device) if splits > 1 else None
+        self.splits[label] = splits
+        self._op(label, "gemm", 2 * m * n * k,
+                 lambda: fb.fp8blk_gemm(layout, a, sa, b, sb, d, splits=splits, workspace=ws))
 
     def run(self, events=None, reduce=True):
         """One step.  events: list of (start, end) CUDA event pairs, one per op, or None.
@@ -683,6 +692,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         rate = units / (ms * 1e-3) / (1e12 if kind == "gemm" else 1e9)
         per_op[label] = {"us": round(ms * 1e3, 1), ("tflops" if kind == "gemm" else "gbs"): round(rate, 1),
                          "frac": round(rate / (fp8_peak if kind == "gemm" else peaks["hbm_gbs"]), 3)}
+        if prog.splits.get(label, 1) > 1:
+            per_op[label]["split_k"] = prog.splits[label]
     traffic_ok = args.workload == "layer" and tokens == 16384 and gemm_source_sha() == GEMM_STEP_DRAM["gemm_cu_sha256"]
     extra = {}
     if rank == 0 and world == 1 and args.workload == "layer" and not args.no_extra:
@@ -726,10 +737,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                          "(kernels back to back on the device, no host launch gaps); L2 flushed once per step",
         "e2e": {"value": flops_all * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        # one kernel per op, two for an amax EMA (partial maxima, then the EMA), and with
-        # data parallelism one rounding kernel per weight gradient after its all-reduce
-        "gpu_launches": (sum(2 if ".amax_" in label else 1 for label, _, _, _ in prog.ops)
-                         + len(prog.grads)) * args.steps,
+        # one kernel per op, two for an amax EMA (partial maxima, then the EMA) and for a
+        # split-K GEMM (the units, then the sum of their partials), and with data parallelism
+        # one rounding kernel per weight gradient after its all-reduce
+        "gpu_launches": (sum(2 if ".amax_" in label or prog.splits.get(label, 1) > 1 else 1
+                             for label, _, _, _ in prog.ops) + len(prog.grads)) * args.steps,
         "clocks": clocks,
         "device_error": prog.fb.status_string(err),
         **extra,

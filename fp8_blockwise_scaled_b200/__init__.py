@@ -34,7 +34,7 @@ __all__ = [
     "fp8blk_quantize_weight_128x128_both", "fp8blk_amax_ema", "fp8blk_amax_ema_workspace_bytes",
     "fp8blk_amax_ema_static", "AMAX_EMA_STATIC_MAX_ROWS",
     "fp8blk_quantize_tensor", "fp8blk_gemm_tensor_scaled", "fp8_linear_delayed_forward",
-    "fp8blk_gemm", "fp8blk_round_f32_to_bf16", "fp8blk_get_device_error", "fp8blk_version", "linear_forward",
+    "fp8blk_gemm", "fp8blk_gemm_splitk", "fp8blk_gemm_splitk_count", "fp8blk_gemm_splitk_workspace_bytes", "fp8blk_round_f32_to_bf16", "fp8blk_get_device_error", "fp8blk_version", "linear_forward",
     "linear_backward", "ROWWISE", "COLWISE_T", "BOTH", "E5M2", "FWD", "DGRAD", "WGRAD", "A_E5M2", "B_E5M2",
     "OUT_F32", "Fp8BlkError",
     "LIB_PATH", "status_string",
@@ -152,9 +152,21 @@ def fp8blk_quantize_weight_128x128_both(w, q=None, s=None, qT=None, sT=None, str
     return q, s, qT, sT
 
 
-def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None, out_dtype=torch.bfloat16):
+def fp8blk_gemm_splitk_count(layout, m: int, n: int, k: int) -> int:
+    """The split-K count the library picks for this GEMM shape on the current device (1 = none)."""
+    return int(lib.fp8blk_gemm_splitk_count(int(layout), int(m), int(n), int(k)))
+
+
+def fp8blk_gemm_splitk_workspace_bytes(m: int, n: int, splits: int) -> int:
+    return int(lib.fp8blk_gemm_splitk_workspace_bytes(int(m), int(n), int(splits)))
+
+
+def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None, out_dtype=torch.bfloat16, splits=1, workspace=None):
     """Blockwise-scaled E4M3 GEMM, D[M,N] = dequant(A) . dequant(B)^T in bf16 (or, with
-    out_dtype=torch.float32 or an fp32 d, the unrounded fp32 sums)."""
+    out_dtype=torch.float32 or an fp32 d, the unrounded fp32 sums).  splits > 1 (or "auto":
+    fp8blk_gemm_splitk_count) divides each output tile's K range among that many units whose
+    fp32 partials are summed in split order; workspace: a float32 CUDA tensor of at least
+    splits * M * N elements (allocated here when None)."""
     dev = _need_cuda(a, sa, b, sb, d)
     m, k = a.shape
     n = b.shape[0]
@@ -175,9 +187,28 @@ def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None, out_dtype=torch.bfloa
         raise ValueError("d must be a bfloat16 or float32 [M,N] tensor with unit column stride")
     flags = (A_E5M2 if a.dtype == E5M2_DTYPE else 0) | (B_E5M2 if b.dtype == E5M2_DTYPE else 0)
     flags |= OUT_F32 if d.dtype == torch.float32 else 0
-    _run(dev, lib.fp8blk_gemm, int(layout) | flags, m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d), d.stride(0),
-                          _stream_handle(stream, dev))
+    if splits == "auto":
+        with torch.cuda.device(dev):
+            splits = fp8blk_gemm_splitk_count(layout, m, n, k)
+    splits = int(splits)
+    if splits == 1:
+        _run(dev, lib.fp8blk_gemm, int(layout) | flags, m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d),
+             d.stride(0), _stream_handle(stream, dev))
+        return d
+    need = splits * m * n
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.float32, device=a.device)
+    elif workspace.dtype != torch.float32 or not workspace.is_contiguous() or workspace.device != a.device:
+        raise ValueError("workspace must be a contiguous float32 tensor on the operands' device")
+    _run(dev, lib.fp8blk_gemm_splitk, int(layout) | flags, m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d),
+         d.stride(0), splits, _ptr(workspace), workspace.numel() * 4, _stream_handle(stream, dev))
     return d
+
+
+def fp8blk_gemm_splitk(layout, a, sa, b, sb, splits, d=None, workspace=None, stream=None, out_dtype=torch.bfloat16):
+    """fp8blk_gemm with split-K over `splits` units per output tile (an int, or "auto")."""
+    return fp8blk_gemm(layout, a, sa, b, sb, d=d, stream=stream, out_dtype=out_dtype, splits=splits,
+                       workspace=workspace)
 
 
 def fp8blk_round_f32_to_bf16(x, y=None, stream=None):

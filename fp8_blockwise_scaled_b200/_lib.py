@@ -47,6 +47,9 @@ def _load() -> ctypes.CDLL:
         "fp8blk_quantize_tensor": [P, I64, I64, I64, P, P, P],
         "fp8blk_gemm_tensor_scaled": [I64, I64, I64, P, P, P, P, P, I64, P],
         "fp8blk_gemm": [I, I64, I64, I64, P, P, P, P, P, I64, P],
+        "fp8blk_gemm_splitk": [I, I64, I64, I64, P, P, P, P, P, I64, I, P, I64, P],
+        "fp8blk_gemm_splitk_workspace_bytes": [I64, I64, I],
+        "fp8blk_gemm_splitk_count": [I, I64, I64, I64],
         "fp8blk_round_f32_to_bf16": [P, I64, P, P],
         "fp8blk_get_device_error": [P],
         "fp8blk_status_string": [I],
@@ -56,7 +59,8 @@ def _load() -> ctypes.CDLL:
         fn = getattr(so, name)
         fn.argtypes = args
         fn.restype = {"fp8blk_status_string": ctypes.c_char_p,
-                      "fp8blk_amax_ema_workspace_bytes": ctypes.c_int64}.get(name, ctypes.c_int)
+                      "fp8blk_amax_ema_workspace_bytes": ctypes.c_int64,
+                      "fp8blk_gemm_splitk_workspace_bytes": ctypes.c_int64}.get(name, ctypes.c_int)
     return so
 
 

@@ -169,8 +169,13 @@ fp8blk_status fp8blk_quantize_weight_128x128_both(const void* w, int64_t n, int6
   return quantize_weight(w, n, k, ldw, q, s, qT, sT, stream);
 }
 
-fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uint8_t* a, const float* sa,
-                          const uint8_t* b, const float* sb, void* d, int64_t ldd, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The checks and arguments shared by the GEMM entry points (no split-K).
+fp8blk_status gemm_args(int layout, int64_t M, int64_t N, int64_t K, const uint8_t* a, const float* sa,
+                        const uint8_t* b, const float* sb, void* d, int64_t ldd, fp8blk::GemmArgs& g) {
   const int formats = layout & (FP8BLK_A_E5M2 | FP8BLK_B_E5M2);
   const bool out_f32 = (layout & FP8BLK_OUT_F32) != 0;
   layout &= ~(FP8BLK_A_E5M2 | FP8BLK_B_E5M2 | FP8BLK_OUT_F32);
@@ -186,7 +191,7 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   if (!aligned16(sa) || !aligned16(sb)) return FP8BLK_ERR_ALIGN;
   fp8blk_status st = check_device();
   if (st != FP8BLK_OK) return st;
-  fp8blk::GemmArgs g{};
+  g = fp8blk::GemmArgs{};
   g.layout = layout;
   g.out_f32 = out_f32;
   g.M = M;
@@ -213,6 +218,60 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uin
   if (const char* e = std::getenv("FP8BLK_GEMM_GROUP_M")) g.group_m = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);
   if (const char* e = std::getenv("FP8BLK_TEST_INJECT_STALL")) g.inject_stall = std::atoi(e) != 0;
+  g.splits = 1;
+  g.workspace = nullptr;
+  return FP8BLK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K, const uint8_t* a, const float* sa,
+                          const uint8_t* b, const float* sb, void* d, int64_t ldd, void* stream) {
+  fp8blk::GemmArgs g;
+  const fp8blk_status st = gemm_args(layout, M, N, K, a, sa, b, sb, d, ldd, g);
+  if (st != FP8BLK_OK) return st;
+  return launch_status(fp8blk::launch_gemm(g, static_cast<cudaStream_t>(stream)));
+}
+
+int fp8blk_gemm_splitk_count(int layout, int64_t M, int64_t N, int64_t K) {
+  const int base = layout & ~(FP8BLK_A_E5M2 | FP8BLK_B_E5M2 | FP8BLK_OUT_F32);
+  if (base != FP8BLK_FWD && base != FP8BLK_DGRAD && base != FP8BLK_WGRAD) return 0;
+  if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K)) return 0;
+  if (check_device() != FP8BLK_OK) return 0;
+  fp8blk::GemmArgs g{};
+  g.layout = base;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);
+  return fp8blk::choose_splits(g);
+}
+
+int64_t fp8blk_gemm_splitk_workspace_bytes(int64_t M, int64_t N, int splits) {
+  if (M <= 0 || N <= 0 || splits <= 1) return 0;
+  return static_cast<int64_t>(splits) * M * N * 4;
+}
+
+fp8blk_status fp8blk_gemm_splitk(int layout, int64_t M, int64_t N, int64_t K, const uint8_t* a, const float* sa,
+                                 const uint8_t* b, const float* sb, void* d, int64_t ldd, int splits,
+                                 float* workspace, int64_t workspace_bytes, void* stream) {
+  // The split arguments are checked first (host-only checks), then those of fp8blk_gemm.
+  if (splits < 1 || (K >= 128 && splits > K / 128)) return FP8BLK_ERR_INVALID_ARG;
+  if (splits > 1) {
+    if (!workspace || workspace_bytes < fp8blk_gemm_splitk_workspace_bytes(M, N, splits))
+      return FP8BLK_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return FP8BLK_ERR_ALIGN;
+    if (M * splits >= (int64_t(1) << 31)) return FP8BLK_ERR_SHAPE;   // partial-tile rows are 32-bit
+  }
+  fp8blk::GemmArgs g;
+  const fp8blk_status st = gemm_args(layout, M, N, K, a, sa, b, sb, d, ldd, g);
+  if (st != FP8BLK_OK) return st;
+  if (splits > 1) {
+    g.splits = splits;
+    g.workspace = workspace;
+  }
   return launch_status(fp8blk::launch_gemm(g, static_cast<cudaStream_t>(stream)));
 }
 

@@ -134,6 +134,19 @@ struct GemmParams {
   uint32_t fmt_bits;      // operand formats for the instruction descriptor (A: bits 7-9, B: bits 10-12; 1 = E5M2)
   const float* tsa;       // per-tensor scales (kTensor variant), device scalars
   const float* tsb;
+  int splits;             // K-splits per output tile (1-CTA kernel; 1 = none)
+  int split_rows;         // split s writes its partial tile at row offset s * split_rows of d (< 2^31 rows)
+};
+
+// Split-K: each unit keeps at least this many K-blocks (the pipeline fill and
+// the fp32 partial tile are paid once per unit).
+constexpr int64_t kMinSplitKBlocks = 16;
+
+// Work unit u of a split-K launch: split u / tiles of output tile u % tiles
+// (split-major, so the units in flight together read the same K range), over
+// K-blocks [kb0, kb1).
+struct Unit {
+  int mb, nb, split, kb0, kb1;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -331,17 +344,18 @@ __device__ __forceinline__ void scale_feed(Ctrl* ctrl, const GemmParams& p, int 
   Ring<kSRing> ring;
   int64_t issued = 0;
   bool ok = true;
-  [[maybe_unused]] float sb0 = 0.0f, sb1 = 0.0f;   // FWD/DGRAD: B scales of K-blocks (kb & ~31) + lane
+  [[maybe_unused]] float sb0 = 0.0f, sb1 = 0.0f;   // FWD/DGRAD: B scales of K-blocks kb0 + 32 i + lane
   for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
     int64_t m0, n0;
-    coords(tile, m0, n0);
-    for (int kb = 0; kb < kblocks; ++kb) {
+    int kb0, kb1;
+    coords(tile, m0, n0, kb0, kb1);
+    for (int kb = kb0; kb < kb1; ++kb) {
       if constexpr (!kWgrad) {
-        if ((kb & 31) == 0) {
+        if (((kb - kb0) & 31) == 0) {
           const int k = kb + lane;
           const float* row = p.sb + (n0 / 128) * kblocks;
-          sb0 = k < kblocks ? __ldg(row + k) : 0.0f;
-          if constexpr (BN == 256) sb1 = k < kblocks ? __ldg(row + kblocks + k) : 0.0f;
+          sb0 = k < kb1 ? __ldg(row + k) : 0.0f;
+          if constexpr (BN == 256) sb1 = k < kb1 ? __ldg(row + kblocks + k) : 0.0f;
         }
       }
       if (!__all_sync(0xFFFFFFFFu,
@@ -351,8 +365,8 @@ __device__ __forceinline__ void scale_feed(Ctrl* ctrl, const GemmParams& p, int 
       }
       ScaleSlot& ss = ctrl->slots[ring.idx];
       if constexpr (!kWgrad) {
-        const float v0 = __shfl_sync(0xFFFFFFFFu, sb0, kb & 31);
-        const float v1 = __shfl_sync(0xFFFFFFFFu, sb1, kb & 31);
+        const float v0 = __shfl_sync(0xFFFFFFFFu, sb0, (kb - kb0) & 31);
+        const float v1 = __shfl_sync(0xFFFFFFFFu, sb1, (kb - kb0) & 31);
         if (lane == 0) {
           ss.sb[0] = v0;
           if constexpr (BN == 256) ss.sb[1] = v1;
@@ -393,6 +407,15 @@ __device__ __forceinline__ void tile_coords(int tile, int num_mb, int num_nb, in
   nb = r / gm;
 }
 
+__device__ __forceinline__ Unit unit_coords(int u, int tiles, int num_mb, int num_nb, int kblocks, const GemmParams& p) {
+  Unit w;
+  w.split = u / tiles;
+  tile_coords(u - w.split * tiles, num_mb, num_nb, p.group_m, w.mb, w.nb);
+  w.kb0 = static_cast<int>(static_cast<int64_t>(w.split) * kblocks / p.splits);
+  w.kb1 = static_cast<int>(static_cast<int64_t>(w.split + 1) * kblocks / p.splits);
+  return w;
+}
+
 // kTensor: one scale per operand (per-tensor scaling).  No per-K-block
 // promotion: the MMAs accumulate the whole K loop of a tile in TMEM and the
 // promotion warps only apply sa * sb, round to bf16 and store, once per tile.
@@ -412,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_nb = static_cast<int>(p.N / BN);
   const int kblocks = static_cast<int>(p.K / BK);
   const int tiles = num_mb * num_nb;
+  const int units = tiles * p.splits;   // split-K: every tile's K-blocks divided among p.splits units
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -458,10 +482,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         Ring<C::kStages> st;
         int64_t issued = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-          int mb, nb;
-          tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
-          for (int kb = 0; kb < kblocks; ++kb) {
+        for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
+          const Unit w = unit_coords(u, tiles, num_mb, num_nb, kblocks, p);
+          const int mb = w.mb, nb = w.nb;
+          for (int kb = w.kb0; kb < w.kb1; ++kb) {
             if (!mbar_wait_bounded(&ctrl->empty[st.idx], st.phase ^ 1u, abort, p.timeout_ns, p.err)) {
               ok = false;
               break;
@@ -487,12 +511,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kScaleWarp) {
       // ---------------------------------------------------------- scale producer (whole warp)
       if constexpr (!kTensor)
-        scale_feed<BN, kWgrad>(ctrl, p, blockIdx.x, gridDim.x, tiles, kblocks,
-                               [&](int tile, int64_t& m0, int64_t& n0) {
-                                 int mb, nb;
-                                 tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
-                                 m0 = static_cast<int64_t>(mb) * BM;
-                                 n0 = static_cast<int64_t>(nb) * BN;
+        scale_feed<BN, kWgrad>(ctrl, p, blockIdx.x, gridDim.x, units, kblocks,
+                               [&](int u, int64_t& m0, int64_t& n0, int& kb0, int& kb1) {
+                                 const Unit w = unit_coords(u, tiles, num_mb, num_nb, kblocks, p);
+                                 m0 = static_cast<int64_t>(w.mb) * BM;
+                                 n0 = static_cast<int64_t>(w.nb) * BN;
+                                 kb0 = w.kb0;
+                                 kb1 = w.kb1;
                                },
                                abort, lane);
     } else {
@@ -508,7 +533,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       if (p.inject_stall) ok = mbar_wait_bounded(&ctrl->never, 0, abort, p.timeout_ns, p.err);
       ok = __all_sync(0xFFFFFFFFu, ok);
-      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+      for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
+        const Unit w = unit_coords(u, tiles, num_mb, num_nb, kblocks, p);
         if constexpr (kTensor) {   // one accumulator buffer per tile
           if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded<false>(&ctrl->tempty[acc.idx], acc.phase ^ 1u, abort,
                                                                 p.timeout_ns, p.err))) {
@@ -516,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
         }
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           const bool got =
               mbar_wait_bounded<false>(&ctrl->full[st.idx], st.phase, abort, p.timeout_ns, p.err) &&
               (kTensor || mbar_wait_bounded<false>(&ctrl->tempty[acc.idx], acc.phase ^ 1u, abort, p.timeout_ns, p.err));
@@ -530,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bdesc = smem_desc_kmajor_sw128(a_addr + C::kABytes);
           const uint32_t d_tmem = tmem_base + acc.idx * BN;
           if (leader) {
-            umma_e4m3(d_tmem, adesc, bdesc, idesc, (kTensor && kb > 0) ? 1u : 0u);
+            umma_e4m3(d_tmem, adesc, bdesc, idesc, (kTensor && kb > w.kb0) ? 1u : 0u);
 #pragma unroll
             for (int k = 1; k < BK / 32; ++k)  // 32 E4M3 values = 32 bytes = 2 x 16 B per step
               umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, 1u);
@@ -566,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (kTensor) {
       // ---------------------------------------------------------- per-tensor epilogue
       const float f = *p.tsa * *p.tsb;
-      for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+      for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {   // the host launches it with splits = 1
         int mb, nb;
         tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
         if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded<false>(&ctrl->tfull[tbuf.idx], tbuf.phase, abort,
@@ -600,13 +626,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->tempty[b]);
       };
-      for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-        int mb, nb;
-        tile_coords(tile, num_mb, num_nb, p.group_m, mb, nb);
-        if (!promote_tile<BN, kWgrad>(ctrl, p, acc, kblocks, tmem_lanes, row, col0, tbuf, sring, abort, lane,
+      for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        // The unit's coordinates are derived again for the store, so that only
+        // u stays live across the K loop.
+        const Unit k = unit_coords(u, tiles, num_mb, num_nb, kblocks, p);
+        if (!promote_tile<BN, kWgrad>(ctrl, p, acc, k.kb1 - k.kb0, tmem_lanes, row, col0, tbuf, sring, abort, lane,
                                       release))
           break;
-        store_row<kCols>(p, static_cast<int64_t>(mb) * BM + row, static_cast<int64_t>(nb) * BN + col0, acc);
+        const Unit w = unit_coords(u, tiles, num_mb, num_nb, kblocks, p);
+        store_row<kCols>(p, static_cast<int64_t>(w.split * p.split_rows + w.mb * BM + row),
+                         static_cast<int64_t>(w.nb) * BN + col0, acc);
       }
     }
   }
@@ -735,10 +764,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kScaleWarp) {
       // ---------------------------------------------------------- scale producer (whole warp)
       scale_feed<BN, kWgrad>(ctrl, p, pair, npairs, tiles, kblocks,
-                             [&](int tile, int64_t& m0, int64_t& n0) {
+                             [&](int tile, int64_t& m0, int64_t& n0, int& kb0, int& kb1) {
                                const int mp = tile % num_mp, nb = tile / num_mp;
                                m0 = static_cast<int64_t>(mp) * 2 * BM + rank * BM;
                                n0 = static_cast<int64_t>(nb) * BN;
+                               kb0 = 0;                  // the pair kernel does not split K
+                               kb1 = kblocks;
                              },
                              abort, lane);
     } else if (leader) {
@@ -897,9 +928,13 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   const int num_mb = static_cast<int>(g.M / BM);
   int group_m = g.group_m > 0 ? g.group_m : (num_mb <= 16 ? num_mb : 8);
   if (group_m > num_mb) group_m = num_mb;
-  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.out_f32, g.timeout_ns, g.err, g.inject_stall, group_m,
-               fmt_bits(g), g.tensor_sa, g.tensor_sb};
-  const int64_t tiles = (g.M / BM) * (g.N / BN);
+  // Split-K: the units write fp32 partial tiles, split s at rows s * M of the
+  // workspace, which the reduction below sums in split order.
+  const int splits = g.splits > 1 ? g.splits : 1;
+  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, splits > 1 ? static_cast<void*>(g.workspace) : g.d,
+               splits > 1 ? g.N : g.ldd, splits > 1 ? 1 : g.out_f32, g.timeout_ns, g.err, g.inject_stall, group_m,
+               fmt_bits(g), g.tensor_sa, g.tensor_sb, splits, static_cast<int>(g.M)};
+  const int64_t tiles = (g.M / BM) * (g.N / BN) * splits;
   int64_t ctas = num_sms();
   if (g.max_ctas > 0 && g.max_ctas < ctas) ctas = g.max_ctas;
   const int grid = static_cast<int>(tiles < ctas ? tiles : ctas);
@@ -912,8 +947,9 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   cfg.numAttrs = set_pdl_attr(attr, g.pdl);
   cfg.attrs = attr;
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<BN, kWgrad, kTensor>, ta, tb, p);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess || splits == 1) return e;
+  return launch_splitk_reduce(g.workspace, splits, g.M, g.N, g.d, g.ldd, g.out_f32, g.pdl, stream);
 }
 
 template <bool kWgrad>
@@ -924,7 +960,7 @@ cudaError_t launch_pair(const GemmArgs& g, cudaStream_t stream) {
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BM)) return cudaErrorInvalidValue;
   GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.out_f32, g.timeout_ns, g.err, g.inject_stall, 0, fmt_bits(g),
-               nullptr, nullptr};
+               nullptr, nullptr, 1, 0};
   const int64_t tiles = (g.M / (2 * BM)) * (g.N / kPairBN);
   int64_t max_pairs = num_sms() / 2;
   if (g.max_ctas > 1 && g.max_ctas / 2 < max_pairs) max_pairs = g.max_ctas / 2;
@@ -953,22 +989,43 @@ double wave_eff(int64_t tiles) {
   return static_cast<double>(tiles) / static_cast<double>(waves * s);
 }
 
+// Tile width of the 1-CTA kernel: 256 unless 128 fills the GPU's waves
+// clearly better (or N is not a multiple of 256).
+int choose_block_n(const GemmArgs& g) {
+  if (g.block_n != 0) return g.block_n;
+  if (g.N % 256 != 0) return 128;
+  const double e256 = wave_eff((g.M / BM) * (g.N / 256));
+  const double e128 = wave_eff((g.M / BM) * (g.N / 128));
+  return (e128 > e256 + 0.10) ? 128 : 256;
+}
+
 }  // namespace
+
+int choose_splits(const GemmArgs& g) {
+  const int64_t tiles = (g.M / BM) * (g.N / choose_block_n(g));
+  const int64_t kblocks = g.K / BK;
+  const int64_t sms = num_sms();
+  // Only a GEMM whose tiles leave SMs idle is split: with a wave or more of
+  // tiles the persistent CTAs already keep every SM busy, and the partial
+  // tiles' fp32 traffic costs more than the shorter tail gains (measured on
+  // B200: 16384 x 1536 outputs with K = 8960 or 17920 run 15-33% slower in 3
+  // splits).  Cost of a split count: waves of units, in whole-tile times.
+  if (tiles >= sms) return 1;
+  auto cost = [&](int64_t s) { return static_cast<double>((tiles * s + sms - 1) / sms) / static_cast<double>(s); };
+  int best = 1;
+  for (int64_t s = 2; s <= 4 && kblocks / s >= kMinSplitKBlocks; ++s)
+    if (cost(s) < 0.8 * cost(best)) best = static_cast<int>(s);
+  return best;
+}
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   const bool wgrad = g.layout == 2;
-  // Pair tiles (256 x 256 over two SMs) only on request, when the shape allows them.
-  if (g.pair > 0 && g.block_n == 0 && !g.tensor_sa && g.M % 256 == 0 && g.N % 256 == 0)
+  if (g.splits > 1 && (g.tensor_sa || !g.workspace || g.K / BK < g.splits || g.M * g.splits >= (int64_t{1} << 31)))
+    return cudaErrorInvalidValue;
+  // Pair tiles (256 x 256 over two SMs) only on request, when the shape allows them (never split).
+  if (g.pair > 0 && g.splits <= 1 && g.block_n == 0 && !g.tensor_sa && g.M % 256 == 0 && g.N % 256 == 0)
     return wgrad ? launch_pair<true>(g, stream) : launch_pair<false>(g, stream);
-  int bn = g.block_n;
-  if (bn == 0) {
-    bn = 128;
-    if (g.N % 256 == 0) {
-      const double e256 = wave_eff((g.M / BM) * (g.N / 256));
-      const double e128 = wave_eff((g.M / BM) * (g.N / 128));
-      bn = (e128 > e256 + 0.10) ? 128 : 256;
-    }
-  }
+  const int bn = choose_block_n(g);
   if (bn == 256 && g.N % 256 != 0) return cudaErrorInvalidValue;
   if (g.tensor_sa) {   // per-tensor scales: no per-K-block promotion, bf16 output
     if (g.layout != 0 || g.out_f32) return cudaErrorInvalidValue;

@@ -180,6 +180,43 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K,
                           void* d, int64_t ldd, void* stream);
 
 /*
+ * The same GEMM with split-K, for shapes whose output tiles do not fill the
+ * GPU (the weight gradient of a narrow layer: few output tiles, long K).  The
+ * K-blocks of every output tile are divided among `splits` work units; unit s
+ * sums its contiguous range of K-blocks (the same per-K-block promotion as
+ * fp8blk_gemm) into an fp32 partial tile in `workspace`, and a second kernel
+ * adds the partials in the order s = 0, 1, ... in fp32 and rounds the total
+ * once to bf16 (or stores it as fp32 with FP8BLK_OUT_F32).  The result is
+ * deterministic; it differs from fp8blk_gemm's only by the order of the fp32
+ * additions.
+ *   splits      1 .. K/128; 1 runs fp8blk_gemm (workspace unused).
+ *   workspace   device memory of at least
+ *               fp8blk_gemm_splitk_workspace_bytes(M, N, splits) bytes, 16-byte
+ *               aligned, owned by the caller; overwritten; it must not overlap
+ *               any operand or d, and must stay untouched until the call's
+ *               kernels have run (stream order).
+ * Errors as fp8blk_gemm; FP8BLK_ERR_INVALID_ARG for a split count out of
+ * range or a missing or short workspace, FP8BLK_ERR_ALIGN for an unaligned
+ * workspace, FP8BLK_ERR_SHAPE when M * splits >= 2^31.
+ */
+fp8blk_status fp8blk_gemm_splitk(int layout, int64_t M, int64_t N, int64_t K,
+                                 const uint8_t* a, const float* sa, const uint8_t* b, const float* sb,
+                                 void* d, int64_t ldd, int splits, float* workspace,
+                                 int64_t workspace_bytes, void* stream);
+
+/* Bytes of split-K workspace for an M x N output: splits * M * N * 4 (0 when splits <= 1). */
+int64_t fp8blk_gemm_splitk_workspace_bytes(int64_t M, int64_t N, int splits);
+
+/*
+ * The split count the library uses well for this GEMM shape on the current
+ * device: 1 when the output tiles fill at least one wave of the SMs;
+ * otherwise the count (2 to 4, each unit keeping at least 16 K-blocks) whose
+ * units shorten the run by at least 20% in whole-tile waves, else 1.  0 for
+ * an invalid layout or shape or an unsupported device.
+ */
+int fp8blk_gemm_splitk_count(int layout, int64_t M, int64_t N, int64_t K);
+
+/*
  * Per-tensor delayed scaling ([EXPL] "核心挑战：Scale Factor 管理", FP8Linear):
  * one amax buffer per tensor (the caller initialises it to 1), updated from
  * the tensor's current max |x| by an exponential moving average before the

@@ -35,10 +35,11 @@ def _operands(layout):
 
 
 @pytest.mark.parametrize("layout", [0, 2])   # per-block and per-column B scales
-@pytest.mark.parametrize("pair", ["0", "1"])  # the 1-CTA kernel and the CTA-pair kernel
+@pytest.mark.parametrize("pair", ["0", "1", "splitk"])  # the 1-CTA kernel, the CTA-pair kernel, split-K units
 def test_stalled_gemm_reports_timeout_and_recovers(layout, pair, monkeypatch):
     require_cuda()
-    monkeypatch.setenv("FP8BLK_GEMM_PAIR", pair)
+    splits = 2 if pair == "splitk" else 1
+    monkeypatch.setenv("FP8BLK_GEMM_PAIR", "0" if pair == "splitk" else pair)
     qa, sa, qb, sb = _operands(layout)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
     A, B = dev(qa).view(torch.float8_e4m3fn), dev(qb).view(torch.float8_e4m3fn)
@@ -46,11 +47,11 @@ def test_stalled_gemm_reports_timeout_and_recovers(layout, pair, monkeypatch):
     assert fb.fp8blk_get_device_error() == 0
     monkeypatch.setenv("FP8BLK_TEST_INJECT_STALL", "1")
     monkeypatch.setenv("FP8BLK_WAIT_TIMEOUT_MS", "200")
-    fb.fp8blk_gemm(layout, A, SA, B, SB)
+    fb.fp8blk_gemm(layout, A, SA, B, SB, splits=splits)
     assert fb.fp8blk_get_device_error() == TIMEOUT_STATUS
     assert fb.fp8blk_get_device_error() == 0            # the word was cleared
     monkeypatch.delenv("FP8BLK_TEST_INJECT_STALL")
-    d = fb.fp8blk_gemm(layout, A, SA, B, SB)
+    d = fb.fp8blk_gemm(layout, A, SA, B, SB, splits=splits)
     assert fb.fp8blk_get_device_error() == 0
     ref = oracle.gemm(layout, qa, sa, qb, sb)
     assert_gemm_close(d.float().cpu().numpy(), ref, "after timeout")
