@@ -26,17 +26,17 @@ import ctypes
 
 import torch
 
-from ._lib import (A_E5M2, B_E5M2, BOTH, COLWISE_T, DGRAD, E5M2, FWD, OUT_F32, ROWWISE, WGRAD, Fp8BlkError,
-                   LIB_PATH, check, lib, status_string)
+from ._lib import (A_E5M2, B_E5M2, BOTH, COLWISE_T, DGRAD, E5M2, FWD, MAX_WEIGHTS, OUT_F32, ROWWISE, WGRAD,
+                   Fp8BlkError, LIB_PATH, WeightDesc, check, lib, status_string)
 
 __all__ = [
     "fp8blk_quantize_act_1x128", "fp8blk_quantize_weight_128x128", "fp8blk_quantize_weight_128x128_t",
-    "fp8blk_quantize_weight_128x128_both", "fp8blk_amax_ema", "fp8blk_amax_ema_workspace_bytes",
+    "fp8blk_quantize_weight_128x128_both", "fp8blk_quantize_weights_128x128_both", "fp8blk_amax_ema", "fp8blk_amax_ema_workspace_bytes",
     "fp8blk_amax_ema_static", "AMAX_EMA_STATIC_MAX_ROWS",
     "fp8blk_quantize_tensor", "fp8blk_gemm_tensor_scaled", "fp8_linear_delayed_forward",
     "fp8blk_gemm", "fp8blk_gemm_splitk", "fp8blk_gemm_splitk_count", "fp8blk_gemm_splitk_workspace_bytes", "fp8blk_round_f32_to_bf16", "fp8blk_get_device_error", "fp8blk_version", "linear_forward",
     "linear_backward", "ROWWISE", "COLWISE_T", "BOTH", "E5M2", "FWD", "DGRAD", "WGRAD", "A_E5M2", "B_E5M2",
-    "OUT_F32", "Fp8BlkError",
+    "OUT_F32", "MAX_WEIGHTS", "Fp8BlkError",
     "LIB_PATH", "status_string",
 ]
 
@@ -219,6 +219,35 @@ def fp8blk_round_f32_to_bf16(x, y=None, stream=None):
     y = _out(y, tuple(x.shape), torch.bfloat16, x.device)
     _run(dev, lib.fp8blk_round_f32_to_bf16, _ptr(x), x.numel(), _ptr(y), _stream_handle(stream, dev))
     return y
+
+
+def fp8blk_quantize_weights_128x128_both(weights, outs=None, stream=None):
+    """Both 128x128 block layouts of several weights in one launch.  weights: a list of
+    [N,K] bf16 CUDA tensors (row stride may exceed K); outs: None or a list of (q, s, qT, sT)
+    per weight.  Returns the list of (q, s, qT, sT), bitwise those of
+    fp8blk_quantize_weight_128x128_both on each weight."""
+    weights = list(weights)
+    if not 1 <= len(weights) <= MAX_WEIGHTS:
+        raise ValueError(f"between 1 and {MAX_WEIGHTS} weights per launch")
+    outs = list(outs) if outs is not None else [None] * len(weights)
+    if len(outs) != len(weights):
+        raise ValueError("one output tuple per weight")
+    weights = [_bf16_2d(w) for w in weights]
+    flat = [t for w, o in zip(weights, outs) for t in (w, *(o or ()))]
+    dev = _need_cuda(*flat)
+    descs = (WeightDesc * len(weights))()
+    result = []
+    for i, (w, o) in enumerate(zip(weights, outs)):
+        n, k = w.shape
+        q, s, qT, sT = o if o is not None else (None, None, None, None)
+        q = _out(q, (n, k), E4M3, w.device)
+        s = _out(s, (n // 128, k // 128), torch.float32, w.device)
+        qT = _out(qT, (k, n), E4M3, w.device)
+        sT = _out(sT, (k // 128, n // 128), torch.float32, w.device)
+        descs[i] = WeightDesc(_ptr(w), n, k, w.stride(0), _ptr(q), _ptr(s), _ptr(qT), _ptr(sT))
+        result.append((q, s, qT, sT))
+    _run(dev, lib.fp8blk_quantize_weights_128x128_both, descs, len(weights), _stream_handle(stream, dev))
+    return result
 
 
 def fp8blk_amax_ema_workspace_bytes(rows: int) -> int:

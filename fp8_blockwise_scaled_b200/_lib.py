@@ -28,6 +28,15 @@ class Fp8BlkError(RuntimeError):
         super().__init__(f"fp8blk call failed: {STATUS_NAMES.get(status, status)}")
 
 
+class WeightDesc(ctypes.Structure):
+    """fp8blk_weight_128x128: one weight of a grouped weight quantisation."""
+    _fields_ = [("w", ctypes.c_void_p), ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("ldw", ctypes.c_int64),
+                ("q", ctypes.c_void_p), ("s", ctypes.c_void_p), ("qT", ctypes.c_void_p), ("sT", ctypes.c_void_p)]
+
+
+MAX_WEIGHTS = 8   # FP8BLK_MAX_WEIGHTS
+
+
 def _load() -> ctypes.CDLL:
     if _build._stale():
         if shutil.which(os.environ.get("NVCC", "nvcc")) is None:
@@ -41,6 +50,7 @@ def _load() -> ctypes.CDLL:
         "fp8blk_quantize_weight_128x128": [P, I64, I64, I64, P, P, P],
         "fp8blk_quantize_weight_128x128_t": [P, I64, I64, I64, P, P, P],
         "fp8blk_quantize_weight_128x128_both": [P, I64, I64, I64, P, P, P, P, P],
+        "fp8blk_quantize_weights_128x128_both": [ctypes.POINTER(WeightDesc), I, P],
         "fp8blk_amax_ema": [P, I64, I64, I64, P, P, P, I64, P],
         "fp8blk_amax_ema_workspace_bytes": [I64],
         "fp8blk_amax_ema_static": [P, I64, I64, I64, P, P, P],

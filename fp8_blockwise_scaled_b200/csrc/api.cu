@@ -131,24 +131,49 @@ fp8blk_status fp8blk_quantize_act_1x128(const void* x, int64_t rows, int64_t col
   return launch_status(fp8blk::launch_quant(kmode, a, static_cast<cudaStream_t>(stream)));
 }
 
-// Weight quantisation in 128x128 blocks: (q, s) in place and/or (qT, sT)
-// transposed; a null pair is not written.
-static fp8blk_status quantize_weight(const void* w, int64_t n, int64_t k, int64_t ldw, uint8_t* q, float* s,
-                                     uint8_t* qT, float* sT, void* stream) {
+// Checks of one weight quantisation in 128x128 blocks: (q, s) in place and/or
+// (qT, sT) transposed, a null pair not written.  Fills the kernel mode.
+static fp8blk_status check_weight(const void* w, int64_t n, int64_t k, int64_t ldw, uint8_t* q, float* s,
+                                  uint8_t* qT, float* sT, int* kmode) {
   fp8blk_status st = check_quant_common(w, n, k, ldw);
   if (st != FP8BLK_OK) return st;
-  int kmode = 0;
+  *kmode = 0;
   for (auto [codes, scales, bit] : {std::tuple{q, s, int(fp8blk::Q_BLK)}, std::tuple{qT, sT, int(fp8blk::Q_BLKT)}}) {
     if (!codes && !scales) continue;
     if (!codes || !scales) return FP8BLK_ERR_INVALID_ARG;
     if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return FP8BLK_ERR_ALIGN;
-    kmode |= bit;
+    *kmode |= bit;
   }
-  if (!kmode) return FP8BLK_ERR_INVALID_ARG;
+  return *kmode ? FP8BLK_OK : FP8BLK_ERR_INVALID_ARG;
+}
+
+static fp8blk_status quantize_weight(const void* w, int64_t n, int64_t k, int64_t ldw, uint8_t* q, float* s,
+                                     uint8_t* qT, float* sT, void* stream) {
+  int kmode = 0;
+  fp8blk_status st = check_weight(w, n, k, ldw, q, s, qT, sT, &kmode);
+  if (st != FP8BLK_OK) return st;
   if ((st = check_device()) != FP8BLK_OK) return st;
   QuantArgs a{static_cast<const uint16_t*>(w), n, k, ldw, q, s, qT, sT, n / 128, k / 128};
   if ((st = set_quant_waits(a)) != FP8BLK_OK) return st;
   return launch_status(fp8blk::launch_quant(kmode, a, static_cast<cudaStream_t>(stream)));
+}
+
+fp8blk_status fp8blk_quantize_weights_128x128_both(const fp8blk_weight_128x128* weights, int count, void* stream) {
+  if (!weights || count < 1 || count > FP8BLK_MAX_WEIGHTS) return FP8BLK_ERR_INVALID_ARG;
+  static_assert(FP8BLK_MAX_WEIGHTS <= fp8blk::kQuantMaxGroup, "the kernel's tensor table holds every weight");
+  QuantArgs a[FP8BLK_MAX_WEIGHTS];
+  for (int i = 0; i < count; ++i) {
+    const fp8blk_weight_128x128& d = weights[i];
+    if (!d.q || !d.s || !d.qT || !d.sT) return FP8BLK_ERR_INVALID_ARG;
+    int kmode = 0;
+    const fp8blk_status st = check_weight(d.w, d.n, d.k, d.ldw, d.q, d.s, d.qT, d.sT, &kmode);
+    if (st != FP8BLK_OK) return st;
+    a[i] = QuantArgs{static_cast<const uint16_t*>(d.w), d.n, d.k, d.ldw, d.q, d.s, d.qT, d.sT, d.n / 128, d.k / 128};
+  }
+  fp8blk_status st = check_device();
+  if (st != FP8BLK_OK) return st;
+  if ((st = set_quant_waits(a[0])) != FP8BLK_OK) return st;
+  return launch_status(fp8blk::launch_quant_weights(a, count, static_cast<cudaStream_t>(stream)));
 }
 
 fp8blk_status fp8blk_quantize_weight_128x128(const void* w, int64_t n, int64_t k, int64_t ldw, uint8_t* q,

@@ -28,6 +28,21 @@ struct QuantArgs {
 
 cudaError_t launch_quant(int mode, const QuantArgs& a, cudaStream_t stream);
 
+// The weight quantiser (both 128x128 block layouts) over up to kQuantMaxGroup
+// tensors in one launch; w[0] also carries the launch-wide fields (waits,
+// error word, test hook, PDL, CTA cap).
+constexpr int kQuantMaxGroup = 8;
+cudaError_t launch_quant_weights(const QuantArgs* w, int count, cudaStream_t stream);
+
+// Kernel argument of the quantiser: N tensors, their input maps, and the
+// running tile counts (tile_end[g] = tiles of tensors 0 .. g).
+template <int N>
+struct QuantLaunch {
+  CUtensorMap map[N];
+  QuantArgs t[N];
+  uint32_t tile_end[N];
+};
+
 // Per-tensor delayed scaling (tensor.cu).
 constexpr int kTensorRowsPerPartial = 8;    // rows reduced by one CTA of the amax reduction
 struct TensorArgs {

@@ -41,6 +41,8 @@
 // 448 rounds or saturates to 448.
 #include <cuda_fp8.h>
 
+#include <cstring>
+
 #include "context.h"
 #include "device.cuh"
 #include "kernels.h"
@@ -66,6 +68,7 @@ struct QCtrl {
   uint64_t full[3], empty[3];
   uint64_t never;            // completed by nothing: the stall test waits on it
   int abort;
+  uint32_t coord[3][3];      // tensor table launches: (tensor, row tile, column tile) of each stage
   float warpmax[2][8];                   // per-warp block maxima, double-buffered by tile parity
   alignas(16) float2 qs[kTile];          // per-column {s, -1/s}
   alignas(16) float4 rq[8][2][4];        // per half-warp, row pair p: {s_2p, s_2p+1, -1/s_2p, -1/s_2p+1}
@@ -109,8 +112,13 @@ __device__ __forceinline__ bool consumers_all(bool v) {
 // timeout the threads agree (one barrier reduction) to leave together, thread
 // 0 first waits for its copies in flight, and the error word records the
 // timeout.
-template <int MODE>
-__global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_constant__ CUtensorMap tm_x, QuantArgs a) {
+// L holds N tensors (N = 1: one tensor; N > 1: the weights of a layer in one
+// launch): their tiles are numbered one tensor after the other, L.tile_end[g]
+// being the tiles of tensors 0 .. g together.  With N > 1 thread 0 publishes
+// each stage's (tensor, row tile, column tile) with the stage, since the
+// consumers cannot step through the tensor boundaries on their own.
+template <int MODE, int N>
+__global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_constant__ QuantLaunch<N> L) {
   constexpr bool kRow = MODE & Q_ROW;
   constexpr bool kColT = MODE & Q_COLT;
   constexpr bool kBlk = MODE & Q_BLK;
@@ -127,11 +135,13 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
 
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
-  // Tile j covers rows 128 (j % tiles_r) .. and columns 128 (j / tiles_r) ..;
-  // a CTA's tiles are gridDim.x apart, so their coordinates advance by fixed
-  // steps (32-bit: the host rejects 2^31 tiles or more).
-  const uint32_t tiles_r = static_cast<uint32_t>(a.tiles_r);
-  const uint32_t tiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
+  const QuantArgs& a0 = L.t[0];                  // launch-wide: waits, error word, test hook
+  // Tile j covers rows 128 (j % tiles_r) .. and columns 128 (j / tiles_r) ..
+  // of its tensor; with one tensor a CTA's tiles are gridDim.x apart, so their
+  // coordinates advance by fixed steps (32-bit: the host rejects 2^31 tiles
+  // or more).
+  const uint32_t tiles_r = static_cast<uint32_t>(a0.tiles_r);
+  const uint32_t tiles = L.tile_end[N - 1];
   const uint32_t step_r = gridDim.x % tiles_r, step_c = gridDim.x / tiles_r;
   auto advance = [&](uint32_t& tr, uint32_t& tc) {
     tr += step_r;
@@ -141,14 +151,28 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
       ++tc;
     }
   };
-  auto load_tile = [&](int stage, uint32_t tr, uint32_t tc) {
+  // Loads tile j into `stage`; (ltr, ltc) are its coordinates when N == 1.
+  uint32_t lg = 0;                                                   // tensor of the next load (N > 1)
+  auto load_tile = [&](int stage, uint32_t j, uint32_t ltr, uint32_t ltc) {
+    uint32_t g = 0, tr = ltr, tc = ltc;
+    if constexpr (N > 1) {
+      while (j >= L.tile_end[lg]) ++lg;          // a CTA's tiles only move forward
+      g = lg;
+      const uint32_t local = j - (g ? L.tile_end[g - 1] : 0u);
+      const uint32_t tr_g = static_cast<uint32_t>(L.t[g].tiles_r);
+      tc = local / tr_g;
+      tr = local - tc * tr_g;
+      ctrl->coord[stage][0] = g;                 // released to the consumers by the arrive below
+      ctrl->coord[stage][1] = tr;
+      ctrl->coord[stage][2] = tc;
+    }
     mbar_arrive_expect_tx(&ctrl->full[stage], kTileBytes);
-    tma_load_2d(smem + stage * kTileBytes, &tm_x, &ctrl->full[stage], static_cast<int>(tc * kTile),
+    tma_load_2d(smem + stage * kTileBytes, &L.map[g], &ctrl->full[stage], static_cast<int>(tc * kTile),
                 static_cast<int>(tr * kTile));
   };
 
   uint32_t issued = 0;                                            // loads issued (thread 0 only)
-  uint32_t ltr = blockIdx.x % tiles_r, ltc = blockIdx.x / tiles_r;   // the next tile to load
+  uint32_t ltr = blockIdx.x % tiles_r, ltc = blockIdx.x / tiles_r;   // the next tile to load (N == 1)
   if (t == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&ctrl->full[s], 1);
@@ -157,10 +181,10 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
     mbar_init(&ctrl->never, 1);
     ctrl->abort = 0;
     fence_mbar_init();
-    tma_prefetch_map(&tm_x);
+    for (int g = 0; g < N; ++g) tma_prefetch_map(&L.map[g]);
     griddep_wait();                              // the input may come from the previous kernel
     for (uint32_t j = blockIdx.x; issued < static_cast<uint32_t>(S) && j < tiles; j += gridDim.x) {
-      load_tile(static_cast<int>(issued++), ltr, ltc);
+      load_tile(static_cast<int>(issued++), j, ltr, ltc);
       advance(ltr, ltc);
     }
   }
@@ -177,8 +201,6 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
   // group spans all 16 row blocks (two per warp).
   const int bj = lane & 15;
   const int bi = 2 * warp + (lane >> 4);
-  const uint32_t cols = static_cast<uint32_t>(a.cols);
-  const uint32_t rows = static_cast<uint32_t>(a.rows);
   float4* rq = ctrl->rq[warp][lane >> 4];
 
   uint32_t it = 0;
@@ -188,9 +210,20 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
     const uint32_t ph = (it / S) & 1;
     // Waits on the critical path: polled without the suspend hint (a
     // completed phase is seen sooner).
-    bool ok = a.inject_stall ? mbar_wait_bounded<false>(&ctrl->never, 0, abort, a.timeout_ns, a.err)
-                             : mbar_wait_bounded<false>(&ctrl->full[s], ph, abort, a.timeout_ns, a.err);
+    bool ok = a0.inject_stall ? mbar_wait_bounded<false>(&ctrl->never, 0, abort, a0.timeout_ns, a0.err)
+                              : mbar_wait_bounded<false>(&ctrl->full[s], ph, abort, a0.timeout_ns, a0.err);
+    uint32_t g = 0;
+    if constexpr (N > 1) {
+      if (ok) {                                  // read before the stage (and its slot) is handed back
+        g = ctrl->coord[s][0];
+        tr = ctrl->coord[s][1];
+        tc = ctrl->coord[s][2];
+      }
+    }
     if (!consumers_all(ok)) break;
+    const QuantArgs& a = L.t[g];
+    const uint32_t cols = static_cast<uint32_t>(a.cols);
+    const uint32_t rows = static_cast<uint32_t>(a.rows);
 
     const int64_t row0 = static_cast<int64_t>(tr) * kTile, col0 = static_cast<int64_t>(tc) * kTile;
     uint4 v[8];
@@ -202,12 +235,12 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
     __syncwarp();                                // everything else comes from registers: hand the stage back
     if (lane == 0) mbar_arrive(&ctrl->empty[s]);
     if (t == 0) {                                // and refill it with the tile S steps ahead
-      if (tile + static_cast<uint32_t>(S) * gridDim.x < tiles &&
-          mbar_wait_bounded<false>(&ctrl->empty[s], ph, abort, a.timeout_ns, a.err)) {
+      const uint32_t next = tile + static_cast<uint32_t>(S) * gridDim.x;
+      if (next < tiles && mbar_wait_bounded<false>(&ctrl->empty[s], ph, abort, a0.timeout_ns, a0.err)) {
         // The warps read the stage through the generic proxy; the TMA load
         // rewrites it through the async proxy: order the two.
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        load_tile(s, ltr, ltc);
+        load_tile(s, next, ltr, ltc);
         advance(ltr, ltc);
         ++issued;
       }
@@ -387,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 2) quant_tile_kernel(const __grid_co
   // memory goes away (on the normal path every load has been consumed).
   if (t == 0) {
     for (uint32_t j = it; j < issued; ++j)
-      mbar_wait_bounded(&ctrl->full[j % S], (j / S) & 1, nullptr, a.timeout_ns, a.err);
+      mbar_wait_bounded(&ctrl->full[j % S], (j / S) & 1, nullptr, a0.timeout_ns, a0.err);
   }
 }
 
@@ -407,26 +440,42 @@ bool make_input_map(CUtensorMap* map, const QuantArgs& a) {
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE>
-cudaError_t launch_mode(const QuantArgs& a, cudaStream_t stream) {
+// Launches quant_tile_kernel<MODE, N> over the tensors a[0 .. count-1]
+// (count <= N; the table's unused entries repeat the last tile count).
+template <int MODE, int N>
+cudaError_t launch_mode(const QuantArgs* a, int count, cudaStream_t stream) {
   static PerContext<int> resident;   // resident CTAs on the device, after the shared-memory opt-in
   constexpr int kSmem = smem_bytes_for<MODE>();
   int grid_cap = 0;
   cudaError_t e = resident.get(&grid_cap, [](int* cap) {
-    cudaError_t r = cudaFuncSetAttribute(quant_tile_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    cudaError_t r =
+        cudaFuncSetAttribute(quant_tile_kernel<MODE, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     int dev = 0, sms = 0, per_sm = 0;
     if (r == cudaSuccess) r = cudaGetDevice(&dev);
     if (r == cudaSuccess) r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (r == cudaSuccess) r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_tile_kernel<MODE>, kThreads, kSmem);
+    if (r == cudaSuccess)
+      r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_tile_kernel<MODE, N>, kThreads, kSmem);
     *cap = sms * (per_sm > 0 ? per_sm : 1);
     return r;
   });
   if (e != cudaSuccess) return e;
-  CUtensorMap map;
-  if (!make_input_map(&map, a)) return cudaErrorInvalidValue;
-  const int64_t tiles = a.tiles_r * a.tiles_c;
-  if (tiles >= (int64_t{1} << 31)) return cudaErrorInvalidValue;   // the kernel counts tiles in 32 bits
-  if (a.max_ctas > 0 && a.max_ctas < grid_cap) grid_cap = a.max_ctas;
+  if (count < 1 || count > N) return cudaErrorInvalidValue;
+  QuantLaunch<N> L;
+  std::memset(&L, 0, sizeof(L));
+  int64_t tiles = 0;
+  for (int g = 0; g < N; ++g) {
+    if (g < count) {
+      if (!make_input_map(&L.map[g], a[g])) return cudaErrorInvalidValue;
+      L.t[g] = a[g];
+      tiles += a[g].tiles_r * a[g].tiles_c;
+    } else {
+      L.map[g] = L.map[count - 1];
+      L.t[g] = a[count - 1];
+    }
+    if (tiles >= (int64_t{1} << 31)) return cudaErrorInvalidValue;   // the kernel counts tiles in 32 bits
+    L.tile_end[g] = static_cast<uint32_t>(tiles);
+  }
+  if (a[0].max_ctas > 0 && a[0].max_ctas < grid_cap) grid_cap = a[0].max_ctas;
   const int grid = static_cast<int>(tiles < grid_cap ? tiles : grid_cap);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
@@ -434,9 +483,9 @@ cudaError_t launch_mode(const QuantArgs& a, cudaStream_t stream) {
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  cfg.numAttrs = set_pdl_attr(attr, a.pdl);
+  cfg.numAttrs = set_pdl_attr(attr, a[0].pdl);
   cfg.attrs = attr;
-  e = cudaLaunchKernelEx(&cfg, quant_tile_kernel<MODE>, map, a);
+  e = cudaLaunchKernelEx(&cfg, quant_tile_kernel<MODE, N>, L);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -445,17 +494,21 @@ cudaError_t launch_mode(const QuantArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_quant(int mode, const QuantArgs& a, cudaStream_t stream) {
   switch (mode) {
-    case Q_ROW: return launch_mode<Q_ROW>(a, stream);
-    case Q_COLT: return launch_mode<Q_COLT>(a, stream);
-    case Q_ROW | Q_COLT: return launch_mode<Q_ROW | Q_COLT>(a, stream);
-    case Q_BLK: return launch_mode<Q_BLK>(a, stream);
-    case Q_BLKT: return launch_mode<Q_BLKT>(a, stream);
-    case Q_BLK | Q_BLKT: return launch_mode<Q_BLK | Q_BLKT>(a, stream);
-    case Q_ROW | Q_E5M2: return launch_mode<Q_ROW | Q_E5M2>(a, stream);
-    case Q_COLT | Q_E5M2: return launch_mode<Q_COLT | Q_E5M2>(a, stream);
-    case Q_ROW | Q_COLT | Q_E5M2: return launch_mode<Q_ROW | Q_COLT | Q_E5M2>(a, stream);
+    case Q_ROW: return launch_mode<Q_ROW, 1>(&a, 1, stream);
+    case Q_COLT: return launch_mode<Q_COLT, 1>(&a, 1, stream);
+    case Q_ROW | Q_COLT: return launch_mode<Q_ROW | Q_COLT, 1>(&a, 1, stream);
+    case Q_BLK: return launch_mode<Q_BLK, 1>(&a, 1, stream);
+    case Q_BLKT: return launch_mode<Q_BLKT, 1>(&a, 1, stream);
+    case Q_BLK | Q_BLKT: return launch_mode<Q_BLK | Q_BLKT, 1>(&a, 1, stream);
+    case Q_ROW | Q_E5M2: return launch_mode<Q_ROW | Q_E5M2, 1>(&a, 1, stream);
+    case Q_COLT | Q_E5M2: return launch_mode<Q_COLT | Q_E5M2, 1>(&a, 1, stream);
+    case Q_ROW | Q_COLT | Q_E5M2: return launch_mode<Q_ROW | Q_COLT | Q_E5M2, 1>(&a, 1, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_quant_weights(const QuantArgs* w, int count, cudaStream_t stream) {
+  return launch_mode<Q_BLK | Q_BLKT, kQuantMaxGroup>(w, count, stream);
 }
 
 }  // namespace fp8blk

@@ -151,6 +151,34 @@ fp8blk_status fp8blk_quantize_weight_128x128_both(const void* w, int64_t n, int6
                                                   void* stream);
 
 /*
+ * The weights of a layer (or any set of weights) quantised in one launch:
+ * for each entry, exactly the outputs of fp8blk_quantize_weight_128x128_both
+ * on that weight.  One launch streams all weights' tiles through the
+ * persistent CTAs, so the small weights do not each pay a launch, a first
+ * tile and a last round of their own.
+ *   weights  host array of `count` descriptors (read during the call only);
+ *            every field as for fp8blk_quantize_weight_128x128_both, all four
+ *            outputs required; the weights' buffers must not overlap each
+ *            other's outputs.
+ *   count    1 .. FP8BLK_MAX_WEIGHTS.
+ * Errors: those of fp8blk_quantize_weight_128x128_both for any entry (the
+ * first failing entry decides), FP8BLK_ERR_INVALID_ARG for a null array or a
+ * count out of range.  Nothing is launched when any entry is invalid.
+ */
+#define FP8BLK_MAX_WEIGHTS 8
+typedef struct {
+  const void* w;   /* [n][ldw] bf16 */
+  int64_t n, k, ldw;
+  uint8_t* q;      /* [n][k] E4M3 */
+  float* s;        /* [n/128][k/128] */
+  uint8_t* qT;     /* [k][n] E4M3 */
+  float* sT;       /* [k/128][n/128] */
+} fp8blk_weight_128x128;
+
+fp8blk_status fp8blk_quantize_weights_128x128_both(const fp8blk_weight_128x128* weights, int count,
+                                                   void* stream);
+
+/*
  * Blockwise-scaled FP8 GEMM with bf16 output ([EXPL] "核心挑战：Scale Factor
  * 管理": the output is linear(x_fp8 * x_scale, w_fp8 * w_scale); [DIGEST]
  * "方法关键点": the linear-layer GEMMs run in E4M3):

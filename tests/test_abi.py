@@ -117,6 +117,27 @@ def test_gemm_argument_errors(args, code):
     assert _lib.lib.fp8blk_gemm(*args) == code
 
 
+def test_quantize_weights_grouped_argument_errors():
+    L = _lib.lib
+    A, M = 0x10000, 0x10008
+
+    def descs(*entries):
+        arr = (_lib.WeightDesc * len(entries))()
+        for i, e in enumerate(entries):
+            arr[i] = _lib.WeightDesc(*e)
+        return arr
+
+    good = (A, 128, 256, 256, A, A, A, A)
+    assert L.fp8blk_quantize_weights_128x128_both(None, 1, S) == 1              # no array
+    assert L.fp8blk_quantize_weights_128x128_both(descs(good), 0, S) == 1       # count < 1
+    nine = descs(*([good] * 9))
+    assert L.fp8blk_quantize_weights_128x128_both(nine, 9, S) == 1              # count > FP8BLK_MAX_WEIGHTS
+    assert L.fp8blk_quantize_weights_128x128_both(descs(good, (A, 128, 200, 256, A, A, A, A)), 2, S) == 2
+    assert L.fp8blk_quantize_weights_128x128_both(descs(good, (A, 128, 256, 256, A, A, 0, A)), 2, S) == 1
+    assert L.fp8blk_quantize_weights_128x128_both(descs((A, 128, 256, 256, A, A, M, A), good), 2, S) == 3
+    assert L.fp8blk_quantize_weights_128x128_both(descs(good, (0, 128, 256, 256, A, A, A, A)), 2, S) == 1
+
+
 def test_gemm_splitk_argument_errors():
     L = _lib.lib
     A = ALIGNED

@@ -137,3 +137,52 @@ def test_adversarial_quotients():
             x[r, g * 128:(g + 1) * 128] = vals
     _check_act(x, fb.BOTH, "adversarial act")
     _check_weight(x, "adversarial weight")
+
+
+def _check_grouped(ws, what):
+    """The grouped weight quantiser against the oracle, weight by weight (codes and scales of both
+    block layouts bit-exact); ws: list of (bf16 bits, row padding of the device copy)."""
+    require_cuda()
+    devs = []
+    for bits, pad in ws:
+        n, k = bits.shape
+        if pad:
+            full = np.zeros((n, k + pad), np.uint16)
+            full[:, :k] = bits
+            devs.append(to_dev(full)[:, :k])
+        else:
+            devs.append(to_dev(bits))
+    outs = fb.fp8blk_quantize_weights_128x128_both(devs)
+    assert fb.fp8blk_get_device_error() == 0
+    for i, ((bits, _), (q, s, qT, sT)) in enumerate(zip(ws, outs)):
+        oq, os_ = oracle.quantize_weight(bits)
+        oqT, osT = oracle.quantize_weight_t(bits)
+        assert_bits_equal(u8(q), oq, f"{what} weight {i} codes")
+        assert_bits_equal(f32(s), os_, f"{what} weight {i} scales")
+        assert_bits_equal(u8(qT), oqT, f"{what} weight {i} ^T codes")
+        assert_bits_equal(f32(sT), osT, f"{what} weight {i} ^T scales")
+
+
+def test_grouped_weights_of_the_layer():
+    """The decoder layer's four weights (QKV 2048x1536, O 1536x1536, gate+up 17920x1536,
+    down 1536x8960) in one launch, as the bench step quantises them."""
+    d = workloads.layer(seed=4, tokens=1024)
+    _check_grouped([(d[k]["W"], 0) for k in ("qkv", "o", "gate_up", "down")], "layer")
+
+
+def test_grouped_weights_mixed_shapes_strides_and_specials():
+    rng = np.random.default_rng(31)
+    x = np.zeros((256, 512), np.uint16)
+    x[:, 128:256] = 0x8000                                                   # -0 blocks
+    x[5, 384] = workloads.f32_to_bf16(np.array([3.0], np.float32))[0]
+    ws = [(workloads.weight(rng, 128, 128), 0),                             # one tile
+          (x, 64),                                                          # special blocks, strided rows
+          (workloads.weight(rng, 384, 1152), 0),
+          (workloads.activation_with_outliers(rng, 640, 256, frac=0.01), 8)]
+    _check_grouped(ws, "mixed")
+
+
+def test_grouped_weights_maximum_count():
+    rng = np.random.default_rng(32)
+    ws = [(workloads.weight(rng, 128 * (1 + i % 3), 128 * (1 + (i * 5) % 4)), 0) for i in range(fb.MAX_WEIGHTS)]
+    _check_grouped(ws, "eight")

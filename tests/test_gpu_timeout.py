@@ -57,7 +57,7 @@ def test_stalled_gemm_reports_timeout_and_recovers(layout, pair, monkeypatch):
     assert_gemm_close(d.float().cpu().numpy(), ref, "after timeout")
 
 
-@pytest.mark.parametrize("kind", ["act_row", "act_both", "weight"])
+@pytest.mark.parametrize("kind", ["act_row", "act_both", "weight", "weights_grouped"])
 def test_stalled_quantiser_reports_timeout_and_recovers(kind, monkeypatch):
     require_cuda()
     rng = np.random.default_rng(12)
@@ -67,6 +67,9 @@ def test_stalled_quantiser_reports_timeout_and_recovers(kind, monkeypatch):
     def run():
         if kind == "weight":
             return fb.fp8blk_quantize_weight_128x128(X)
+        if kind == "weights_grouped":
+            q, s, _, _ = fb.fp8blk_quantize_weights_128x128_both([X, X[:256, :384]])[0]
+            return q, s
         q, s, qT, sT = fb.fp8blk_quantize_act_1x128(X, fb.ROWWISE if kind == "act_row" else fb.BOTH)
         return q, s
 
@@ -79,6 +82,6 @@ def test_stalled_quantiser_reports_timeout_and_recovers(kind, monkeypatch):
     monkeypatch.delenv("FP8BLK_TEST_INJECT_STALL")
     q, s = run()
     assert fb.fp8blk_get_device_error() == 0
-    oq, os_ = oracle.quantize_weight(x) if kind == "weight" else oracle.quantize_act_rowwise(x)
+    oq, os_ = oracle.quantize_weight(x) if kind.startswith("weight") else oracle.quantize_act_rowwise(x)
     assert np.array_equal(q.view(torch.uint8).cpu().numpy(), oq)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
