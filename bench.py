@@ -53,7 +53,7 @@ L2_FLUSH_BYTES = 256 << 20
 # one step; profiles/gemm_dram_layer_16384.md); algorithmic minimum 2.59 GB (codes
 # read once, bf16 outputs written once).  It describes the GEMM source whose
 # SHA-256 prefix is given; for any other source the bench reports no traffic.
-GEMM_STEP_DRAM = {"bytes": 2.850e9, "gemm_cu_sha256": "23d17fb3113bd951"}
+GEMM_STEP_DRAM = {"bytes": 2.882e9, "gemm_cu_sha256": "2558aa53e9cd9ae1"}
 GEMM_SOURCE = os.path.join(ROOT, "fp8_blockwise_scaled_b200", "csrc", "gemm.cu")
 
 WORKLOAD_DESC = {
@@ -731,8 +731,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "roofline": {"bound": "tensor", "kernel": "gemm_blockwise_kernel", "achieved": gemm_tflops,
                      "peak": fp8_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
                      "traffic": GEMM_STEP_DRAM["bytes"] if traffic_ok else None,
-                     "traffic_scope": "bytes per step, the GEMM launches together (12 GEMMs, the split-K sum included; achieved "
-                                      "is over the same launches)",
+                     "traffic_scope": "bytes per step, the GEMM launches together (12 GEMMs, the split-K sums included; "
+                                      "achieved is over the same launches)",
                      "traffic_note": "ncu capture of this GEMM source" if traffic_ok else
                                      "no capture of this GEMM source (or another workload): not reported",
                      "peak_source": f"{peak_src} bf16 burst x {FP8_PER_BF16:g} (nominal fp8/bf16 ratio); each GEMM "

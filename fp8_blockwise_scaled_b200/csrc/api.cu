@@ -271,6 +271,7 @@ int fp8blk_gemm_splitk_count(int layout, int64_t M, int64_t N, int64_t K) {
   g.N = N;
   g.K = K;
   if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);
+  if (env_int("FP8BLK_GEMM_SPLITK", 1) == 0) return 1;
   return fp8blk::choose_splits(g);
 }
 

@@ -1,7 +1,7 @@
 // fp32 -> bf16 rounding of a summed partial result (the data-parallel weight
 // gradient: each rank's fp32 partial dW is all-reduced in fp32 and rounded to
-// bf16 once, after the sum), and the sum of split-K partial tiles.  HBM bound:
-// 16-byte loads and 8-byte (bf16) or 16-byte (fp32) stores, grid-stride.
+// bf16 once, after the sum).  HBM bound: 4 B read + 2 B written per element,
+// 16-byte loads and 8-byte stores, grid-stride over the array.
 #include <cuda_bf16.h>
 
 #include "context.h"
@@ -34,66 +34,7 @@ __global__ void __launch_bounds__(kThreads) round_bf16_kernel(const float* __res
   }
 }
 
-// d[m][n] = ws[0][m][n] + ws[1][m][n] + ... (left to right, fp32), rounded
-// once to bf16 unless kF32.  One CTA per row at a time, 4 columns per thread.
-template <bool kF32>
-__global__ void __launch_bounds__(kThreads) splitk_reduce_kernel(const float* __restrict__ ws, int splits, int64_t M,
-                                                                 int64_t N, void* __restrict__ d, int64_t ldd) {
-  griddep_wait();
-  if (threadIdx.x == 0) griddep_launch_dependents();
-  const int64_t plane = M * N, n4 = N / 4;
-  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
-    for (int64_t c = threadIdx.x; c < n4; c += kThreads) {
-      const float* src = ws + m * N + 4 * c;
-      float4 acc = *reinterpret_cast<const float4*>(src);
-      for (int s = 1; s < splits; ++s) {
-        const float4 v = *reinterpret_cast<const float4*>(src + s * plane);
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
-      }
-      if constexpr (kF32) {
-        *reinterpret_cast<float4*>(static_cast<float*>(d) + m * ldd + 4 * c) = acc;
-      } else {
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 w;
-        w.x = *reinterpret_cast<const uint32_t*>(&lo);
-        w.y = *reinterpret_cast<const uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(d) + m * ldd + 4 * c) = w;
-      }
-    }
-  }
-}
-
 }  // namespace
-
-cudaError_t launch_splitk_reduce(const float* ws, int splits, int64_t M, int64_t N, void* d, int64_t ldd, int out_f32,
-                                 int pdl, cudaStream_t stream) {
-  static PerContext<int> resident;   // resident CTAs on the device
-  int cap = 0;
-  cudaError_t e = resident.get(&cap, [](int* v) {
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaError_t r = cudaGetDevice(&dev);
-    if (r == cudaSuccess) r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (r == cudaSuccess)
-      r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, splitk_reduce_kernel<false>, kThreads, 0);
-    *v = sms * (per_sm > 0 ? per_sm : 1);
-    return r;
-  });
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(M < cap ? M : cap), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  cfg.numAttrs = set_pdl_attr(attr, pdl);
-  cfg.attrs = attr;
-  e = out_f32 ? cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<true>, ws, splits, M, N, d, ldd)
-              : cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<false>, ws, splits, M, N, d, ldd);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
-}
 
 cudaError_t launch_round_bf16(const float* x, int64_t n, uint16_t* y, int pdl, cudaStream_t stream) {
   static PerContext<int> resident;   // resident CTAs on the device

@@ -134,19 +134,24 @@ struct GemmParams {
   uint32_t fmt_bits;      // operand formats for the instruction descriptor (A: bits 7-9, B: bits 10-12; 1 = E5M2)
   const float* tsa;       // per-tensor scales (kTensor variant), device scalars
   const float* tsb;
-  int splits;             // K-splits per output tile (1-CTA kernel; 1 = none)
-  int split_rows;         // split s writes its partial tile at row offset s * split_rows of d (< 2^31 rows)
+  int splits;             // K-splits of each split tile (1-CTA kernel; 1 = none)
+  int whole_tiles;        // tiles [0, whole_tiles) run whole, tiles [whole_tiles, tiles) in `splits` units
+  float* partials;        // split units' fp32 partial tiles [slot][BM][BN], slot = t * splits + split
 };
 
 // Split-K: each unit keeps at least this many K-blocks (the pipeline fill and
 // the fp32 partial tile are paid once per unit).
 constexpr int64_t kMinSplitKBlocks = 16;
+// The split tiles of a partial last round keep at least this many per unit
+// (measured on B200: 16384 x 1536 x 2048 split 2 in 8-K-block units ran 3%
+// slower than unsplit; 14 and 28 K-blocks per unit gain 8-11%).
+constexpr int64_t kMinTailKBlocks = 12;
 
-// Work unit u of a split-K launch: split u / tiles of output tile u % tiles
-// (split-major, so the units in flight together read the same K range), over
-// K-blocks [kb0, kb1).
+// Work unit of a launch: a whole tile over K-blocks [0, kblocks) (slot -1), or
+// one of the `splits` units of a split tile over K-blocks [kb0, kb1), whose
+// fp32 partial goes to partial-tile slot `slot`.
 struct Unit {
-  int mb, nb, split, kb0, kb1;
+  int mb, nb, kb0, kb1, slot;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -407,14 +412,37 @@ __device__ __forceinline__ void tile_coords(int tile, int num_mb, int num_nb, in
   nb = r / gm;
 }
 
+// Units [0, whole_tiles) are the whole tiles; the rest are the split tiles'
+// units in split-major order (the units in flight together read the same K
+// range), so with whole_tiles a multiple of the grid the split units fill the
+// last round, which whole tiles would leave mostly idle.
 __device__ __forceinline__ Unit unit_coords(int u, int tiles, int num_mb, int num_nb, int kblocks, const GemmParams& p) {
   Unit w;
-  w.split = u / tiles;
-  tile_coords(u - w.split * tiles, num_mb, num_nb, p.group_m, w.mb, w.nb);
-  w.kb0 = static_cast<int>(static_cast<int64_t>(w.split) * kblocks / p.splits);
-  w.kb1 = static_cast<int>(static_cast<int64_t>(w.split + 1) * kblocks / p.splits);
+  int tile = u;
+  w.kb0 = 0;
+  w.kb1 = kblocks;
+  w.slot = -1;
+  if (u >= p.whole_tiles) {
+    const int split_tiles = tiles - p.whole_tiles, v = u - p.whole_tiles;
+    const int split = v / split_tiles, t = v - split * split_tiles;
+    tile = p.whole_tiles + t;
+    w.kb0 = split * kblocks / p.splits;          // K < 2^31 / 128 * 128: no overflow
+    w.kb1 = (split + 1) * kblocks / p.splits;
+    w.slot = t * p.splits + split;
+  }
+  tile_coords(tile, num_mb, num_nb, p.group_m, w.mb, w.nb);
   return w;
 }
+
+// The number of K-blocks of unit u alone (the promotion warps need only that
+// before their K loop; the tile coordinates are derived after it).
+__device__ __forceinline__ int unit_kblocks(int u, int tiles, int kblocks, const GemmParams& p) {
+  const int v = u - p.whole_tiles;                    // < 0 for a whole tile
+  const int split = max(v, 0) / max(tiles - p.whole_tiles, 1);
+  const int n = (split + 1) * kblocks / p.splits - split * kblocks / p.splits;
+  return v < 0 ? kblocks : n;
+}
+
 
 // kTensor: one scale per operand (per-tensor scaling).  No per-K-block
 // promotion: the MMAs accumulate the whole K loop of a tile in TMEM and the
@@ -435,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_nb = static_cast<int>(p.N / BN);
   const int kblocks = static_cast<int>(p.K / BK);
   const int tiles = num_mb * num_nb;
-  const int units = tiles * p.splits;   // split-K: every tile's K-blocks divided among p.splits units
+  const int units = p.whole_tiles + (tiles - p.whole_tiles) * p.splits;   // split tiles: p.splits units each
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -627,15 +655,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&ctrl->tempty[b]);
       };
       for (int u = blockIdx.x; u < units; u += gridDim.x) {
-        // The unit's coordinates are derived again for the store, so that only
-        // u stays live across the K loop.
-        const Unit k = unit_coords(u, tiles, num_mb, num_nb, kblocks, p);
-        if (!promote_tile<BN, kWgrad>(ctrl, p, acc, k.kb1 - k.kb0, tmem_lanes, row, col0, tbuf, sring, abort, lane,
-                                      release))
+        // The unit's coordinates are derived after the K loop, so that only u
+        // stays live across it.
+        if (!promote_tile<BN, kWgrad>(ctrl, p, acc, unit_kblocks(u, tiles, kblocks, p), tmem_lanes, row, col0, tbuf,
+                                      sring, abort, lane, release))
           break;
+        // A whole tile goes to d (bf16, or fp32 with out_f32); a split unit's
+        // fp32 partial to its slot, summed later by gemm_splitk_sum_kernel.
         const Unit w = unit_coords(u, tiles, num_mb, num_nb, kblocks, p);
-        store_row<kCols>(p, static_cast<int64_t>(w.split * p.split_rows + w.mb * BM + row),
-                         static_cast<int64_t>(w.nb) * BN + col0, acc);
+        const bool part = w.slot >= 0;
+        const int64_t off = part ? static_cast<int64_t>(w.slot * BM + row) * BN + col0
+                                 : static_cast<int64_t>(w.mb * BM + row) * p.ldd + static_cast<int64_t>(w.nb) * BN + col0;
+        if (part || p.out_f32)
+          store_row_f32<kCols>((part ? p.partials : static_cast<float*>(p.d)) + off, acc);
+        else
+          store_row_bf16<kCols>(static_cast<uint16_t*>(p.d) + off, acc);
       }
     }
   }
@@ -859,6 +893,51 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+namespace {
+
+// Where the split tiles of a launch go: tiles [whole, tiles) of the M/BM x N/BN
+// grid (tile order as in the GEMM), `splits` partial tiles each.
+struct SplitSum {
+  int whole, splits, num_mb, num_nb, group_m;
+  void* d;
+  int64_t ldd;
+};
+
+// Sums the split units' fp32 partial tiles of each split tile in the order
+// split 0, 1, ... (fp32), and writes the tile to d, rounded once to bf16 or
+// (kF32) as fp32.  One CTA per 8 rows of a split tile, 4 columns per thread;
+// HBM (or L2) bound: splits x 4 B read + 2 or 4 B written per element.
+template <int BN, bool kF32>
+__global__ void __launch_bounds__(256) gemm_splitk_sum_kernel(const float* __restrict__ partials, SplitSum q) {
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  const int t = blockIdx.x / (BM / 8), r0 = (blockIdx.x % (BM / 8)) * 8;
+  int mb, nb;
+  tile_coords(q.whole + t, q.num_mb, q.num_nb, q.group_m, mb, nb);
+  const int64_t slot0 = static_cast<int64_t>(t) * q.splits;
+  for (int e = threadIdx.x; e < 8 * BN / 4; e += 256) {
+    const int r = r0 + e / (BN / 4), c = 4 * (e % (BN / 4));
+    const float* src = partials + (slot0 * BM + r) * BN + c;
+    float4 acc = *reinterpret_cast<const float4*>(src);
+    for (int sp = 1; sp < q.splits; ++sp) {
+      const float4 v = *reinterpret_cast<const float4*>(src + static_cast<int64_t>(sp) * BM * BN);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    const int64_t off = static_cast<int64_t>(mb * BM + r) * q.ldd + static_cast<int64_t>(nb) * BN + c;
+    if constexpr (kF32) {
+      *reinterpret_cast<float4*>(static_cast<float*>(q.d) + off) = acc;
+    } else {
+      *reinterpret_cast<uint2*>(static_cast<uint16_t*>(q.d) + off) =
+          make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+    }
+  }
+}
+
+}  // namespace
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -928,16 +1007,20 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   const int num_mb = static_cast<int>(g.M / BM);
   int group_m = g.group_m > 0 ? g.group_m : (num_mb <= 16 ? num_mb : 8);
   if (group_m > num_mb) group_m = num_mb;
-  // Split-K: the units write fp32 partial tiles, split s at rows s * M of the
-  // workspace, which the reduction below sums in split order.
-  const int splits = g.splits > 1 ? g.splits : 1;
-  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, splits > 1 ? static_cast<void*>(g.workspace) : g.d,
-               splits > 1 ? g.N : g.ldd, splits > 1 ? 1 : g.out_f32, g.timeout_ns, g.err, g.inject_stall, group_m,
-               fmt_bits(g), g.tensor_sa, g.tensor_sb, splits, static_cast<int>(g.M)};
-  const int64_t tiles = (g.M / BM) * (g.N / BN) * splits;
+  const int64_t tiles = (g.M / BM) * (g.N / BN);
   int64_t ctas = num_sms();
   if (g.max_ctas > 0 && g.max_ctas < ctas) ctas = g.max_ctas;
-  const int grid = static_cast<int>(tiles < ctas ? tiles : ctas);
+  // Split-K: with fewer tiles than CTAs every tile is split; otherwise the
+  // tiles of the last, partial round (tiles % CTAs of them) are, so that their
+  // units fill that round.  Split units write fp32 partial tiles to the
+  // workspace; gemm_splitk_sum_kernel adds them in split order afterwards.
+  int splits = g.splits > 1 ? g.splits : 1;
+  const int64_t whole = splits == 1 ? tiles : (tiles < ctas ? 0 : tiles - tiles % ctas);
+  if (whole == tiles) splits = 1;
+  GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.out_f32, g.timeout_ns, g.err, g.inject_stall, group_m,
+               fmt_bits(g), g.tensor_sa, g.tensor_sb, splits, static_cast<int>(whole), g.workspace};
+  const int64_t units = whole + (tiles - whole) * splits;
+  const int grid = static_cast<int>(units < ctas ? units : ctas);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -949,7 +1032,18 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<BN, kWgrad, kTensor>, ta, tb, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || splits == 1) return e;
-  return launch_splitk_reduce(g.workspace, splits, g.M, g.N, g.d, g.ldd, g.out_f32, g.pdl, stream);
+  const SplitSum q{static_cast<int>(whole), splits, num_mb, static_cast<int>(g.N / BN), group_m, g.d, g.ldd};
+  cudaLaunchConfig_t sc = {};
+  sc.gridDim = dim3(static_cast<unsigned>((tiles - whole) * (BM / 8)), 1, 1);
+  sc.blockDim = dim3(256, 1, 1);
+  sc.stream = stream;
+  cudaLaunchAttribute sattr[1];
+  sc.numAttrs = set_pdl_attr(sattr, g.pdl);
+  sc.attrs = sattr;
+  e = g.out_f32 ? cudaLaunchKernelEx(&sc, gemm_splitk_sum_kernel<BN, true>, g.workspace, q)
+                : cudaLaunchKernelEx(&sc, gemm_splitk_sum_kernel<BN, false>, g.workspace, q);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 template <bool kWgrad>
@@ -960,7 +1054,7 @@ cudaError_t launch_pair(const GemmArgs& g, cudaStream_t stream) {
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BM)) return cudaErrorInvalidValue;
   GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.out_f32, g.timeout_ns, g.err, g.inject_stall, 0, fmt_bits(g),
-               nullptr, nullptr, 1, 0};
+               nullptr, nullptr, 1, 0, nullptr};
   const int64_t tiles = (g.M / (2 * BM)) * (g.N / kPairBN);
   int64_t max_pairs = num_sms() / 2;
   if (g.max_ctas > 1 && g.max_ctas / 2 < max_pairs) max_pairs = g.max_ctas / 2;
@@ -1005,16 +1099,25 @@ int choose_splits(const GemmArgs& g) {
   const int64_t tiles = (g.M / BM) * (g.N / choose_block_n(g));
   const int64_t kblocks = g.K / BK;
   const int64_t sms = num_sms();
-  // Only a GEMM whose tiles leave SMs idle is split: with a wave or more of
-  // tiles the persistent CTAs already keep every SM busy, and the partial
-  // tiles' fp32 traffic costs more than the shorter tail gains (measured on
-  // B200: 16384 x 1536 outputs with K = 8960 or 17920 run 15-33% slower in 3
-  // splits).  Cost of a split count: waves of units, in whole-tile times.
-  if (tiles >= sms) return 1;
-  auto cost = [&](int64_t s) { return static_cast<double>((tiles * s + sms - 1) / sms) / static_cast<double>(s); };
+  if (tiles < sms) {
+    // Fewer tiles than SMs: all tiles split, into the count that cuts the run
+    // by at least 20% in whole-tile waves.
+    auto cost = [&](int64_t s) { return static_cast<double>((tiles * s + sms - 1) / sms) / static_cast<double>(s); };
+    int best = 1;
+    for (int64_t s = 2; s <= 4 && kblocks / s >= kMinSplitKBlocks; ++s)
+      if (cost(s) < 0.8 * cost(best)) best = static_cast<int>(s);
+    return best;
+  }
+  // A wave or more: only the tiles of the last, partial round are split (the
+  // persistent CTAs keep every SM busy before it), into as many units as fit
+  // beside each other on the SMs, each keeping at least kMinTailKBlocks.
+  // Splitting every tile instead was measured 15-33% slower on B200 (16384 x
+  // 1536 outputs, K = 8960 and 17920, 3 splits): the partial tiles' fp32
+  // traffic costs more than the shorter last round gains.
+  const int64_t tail = tiles % sms;
   int best = 1;
-  for (int64_t s = 2; s <= 4 && kblocks / s >= kMinSplitKBlocks; ++s)
-    if (cost(s) < 0.8 * cost(best)) best = static_cast<int>(s);
+  for (int64_t s = 2; tail > 0 && s <= 8 && tail * s <= sms && kblocks / s >= kMinTailKBlocks; ++s)
+    best = static_cast<int>(s);
   return best;
 }
 

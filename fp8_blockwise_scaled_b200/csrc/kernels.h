@@ -84,8 +84,8 @@ struct GemmArgs {
   const float* tensor_sa;     // non-null: one scale per operand (device scalars), no per-block scales
   const float* tensor_sb;
   unsigned int* err;          // device error word
-  int splits;                 // > 1: split-K over that many units per tile (1-CTA kernel)
-  float* workspace;           // split-K: splits * M * N floats of partial tiles
+  int splits;                 // > 1: split-K over that many units per split tile (1-CTA kernel)
+  float* workspace;           // split-K: at least splits * M * N floats of partial tiles
 };
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream);
@@ -94,11 +94,6 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream);
 // device (1 when the output tiles already fill the SMs' waves).
 int choose_splits(const GemmArgs& g);
 
-// d[m][n] = sum over s = 0 .. splits-1, in that order, of ws[s][m][n]
-// (ws: splits x M x N floats), rounded once to bf16, or stored as fp32 when
-// out_f32.  d has row stride ldd (elements of its type).
-cudaError_t launch_splitk_reduce(const float* ws, int splits, int64_t M, int64_t N, void* d, int64_t ldd, int out_f32,
-                                 int pdl, cudaStream_t stream);
 
 // y[i] = bf16_round_nearest_even(x[i]) for i < n (x, y 16-byte aligned).
 cudaError_t launch_round_bf16(const float* x, int64_t n, uint16_t* y, int pdl, cudaStream_t stream);

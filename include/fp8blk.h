@@ -45,6 +45,7 @@
  *      FP8BLK_GEMM_PAIR           1: 256x256 tiles on CTA pairs wherever M and
  *                                 N are multiples of 256; 0: never (default)
  *      FP8BLK_GEMM_GROUP_M        M-blocks per group of the GEMM tile order
+ *      FP8BLK_GEMM_SPLITK=0       fp8blk_gemm_splitk_count returns 1 (no split)
  *      FP8BLK_GEMM_MAX_CTAS       at most this many GEMM CTAs (one per SM), so
  *                                 that concurrent work on other streams finds
  *                                 free SMs (default: one per SM)
@@ -208,15 +209,17 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K,
                           void* d, int64_t ldd, void* stream);
 
 /*
- * The same GEMM with split-K, for shapes whose output tiles do not fill the
- * GPU (the weight gradient of a narrow layer: few output tiles, long K).  The
- * K-blocks of every output tile are divided among `splits` work units; unit s
- * sums its contiguous range of K-blocks (the same per-K-block promotion as
- * fp8blk_gemm) into an fp32 partial tile in `workspace`, and a second kernel
- * adds the partials in the order s = 0, 1, ... in fp32 and rounds the total
- * once to bf16 (or stores it as fp32 with FP8BLK_OUT_F32).  The result is
- * deterministic; it differs from fp8blk_gemm's only by the order of the fp32
- * additions.
+ * The same GEMM with split-K, for shapes whose output tiles leave SMs idle:
+ * with fewer tiles than SMs (the weight gradient of a narrow layer: few
+ * tiles, long K) every tile is split; with more, the tiles of the last,
+ * partial round of the persistent CTAs (tiles mod SMs of them) are, so that
+ * their units fill that round.  The K-blocks of a split tile are divided among
+ * `splits` work units; unit s sums its contiguous range of K-blocks (the same
+ * per-K-block promotion as fp8blk_gemm) into an fp32 partial tile in
+ * `workspace`, and a second kernel adds the partials in the order s = 0, 1,
+ * ... in fp32 and rounds the total once to bf16 (or stores it as fp32 with
+ * FP8BLK_OUT_F32).  The result is deterministic; it differs from
+ * fp8blk_gemm's only by the order of the fp32 additions in the split tiles.
  *   splits      1 .. K/128; 1 runs fp8blk_gemm (workspace unused).
  *   workspace   device memory of at least
  *               fp8blk_gemm_splitk_workspace_bytes(M, N, splits) bytes, 16-byte
@@ -237,10 +240,12 @@ int64_t fp8blk_gemm_splitk_workspace_bytes(int64_t M, int64_t N, int splits);
 
 /*
  * The split count the library uses well for this GEMM shape on the current
- * device: 1 when the output tiles fill at least one wave of the SMs;
- * otherwise the count (2 to 4, each unit keeping at least 16 K-blocks) whose
- * units shorten the run by at least 20% in whole-tile waves, else 1.  0 for
- * an invalid layout or shape or an unsupported device.
+ * device.  With fewer output tiles than SMs (all tiles are split): the count
+ * (2 to 4, each unit keeping at least 16 K-blocks) whose units shorten the
+ * run by at least 20% in whole-tile waves, else 1.  With more (only the tiles
+ * of the last, partial round of the SMs are split): the largest count up to 8
+ * whose units fit beside each other on the SMs with at least 12 K-blocks
+ * each, else 1.  0 for an invalid layout or shape or an unsupported device.
  */
 int fp8blk_gemm_splitk_count(int layout, int64_t M, int64_t N, int64_t K);
 

@@ -1,7 +1,9 @@
 """Split-K GEMM (fp8blk_gemm_splitk) against the CPU oracle.
 
-The K-blocks of every output tile are divided among `splits` work units whose
-fp32 partial tiles are summed in split order and rounded once.  Every output
+The K-blocks of a split tile are divided among `splits` work units whose fp32
+partial tiles are summed in split order and rounded once.  With fewer tiles
+than SMs every tile is split; with more, only the tiles of the last, partial
+round of the persistent CTAs.  Every output
 element is compared with the oracle at the tolerance of the unsplit GEMM
 (test_gpu_gemm.py); the result must be bitwise reproducible run to run; the
 fp32-output form must match the oracle too (it is what a data-parallel rank
@@ -106,7 +108,8 @@ def test_splitk_one_is_the_plain_gemm():
 
 
 def test_splitk_count_for_the_layer_shapes():
-    """On a 148-SM B200 the library splits only the QKV weight gradient (96 output tiles)."""
+    """On a 148-SM B200: the QKV weight gradient (96 output tiles) is split whole; the 768-tile
+    GEMMs with K >= 16 K-blocks have their last round's 28 tiles split."""
     require_cuda()
     if torch.cuda.get_device_properties(0).multi_processor_count != 148:
         pytest.skip("the pinned counts are those of a 148-SM B200")
@@ -115,9 +118,10 @@ def test_splitk_count_for_the_layer_shapes():
     assert fb.fp8blk_gemm_splitk_count(fb.WGRAD, 1536, 1536, t) == 1      # O dW: 144 tiles of 128 x 128
     assert fb.fp8blk_gemm_splitk_count(fb.WGRAD, 17920, 1536, t) == 1
     assert fb.fp8blk_gemm_splitk_count(fb.WGRAD, 1536, 8960, t) == 1
-    for n, k in ((2048, 1536), (1536, 1536), (17920, 1536), (1536, 8960)):
-        assert fb.fp8blk_gemm_splitk_count(fb.FWD, t, n, k) == 1
-        assert fb.fp8blk_gemm_splitk_count(fb.DGRAD, t, k, n) == 1
+    for (n, k), fwd, dgrad in (((2048, 1536), 1, 1), ((1536, 1536), 1, 1), ((17920, 1536), 1, 5),
+                               ((1536, 8960), 5, 1)):
+        assert fb.fp8blk_gemm_splitk_count(fb.FWD, t, n, k) == fwd
+        assert fb.fp8blk_gemm_splitk_count(fb.DGRAD, t, k, n) == dgrad
     assert fb.fp8blk_gemm_splitk_count(fb.FWD, 1024, 2048, 1536) == 1     # 12 K-blocks: too few to split
     assert fb.fp8blk_gemm_splitk_count(fb.DGRAD, 1024, 1536, 17920) == 3  # 48 tiles, 140 K-blocks
 
@@ -132,3 +136,19 @@ def test_splitk_full_size_qkv_weight_gradient():
     d = _splitk(oracle.WGRAD, ops, splits)
     assert_gemm_close(d.float().cpu().numpy().astype(np.float64), oracle.gemm(oracle.WGRAD, *ops),
                       f"qkv dW 2048x1536x16384 split-K {splits}")
+
+
+@pytest.mark.parametrize("layout,block_n", [(oracle.FWD, "auto"), (oracle.DGRAD, "128"), (oracle.WGRAD, "auto")])
+def test_splitk_of_the_last_round(layout, block_n, monkeypatch):
+    """More tiles than SMs: only the last round's tiles are split (150 tiles of 128 x 256 on 148 SMs:
+    2 split tiles; 300 of 128 x 128: 4), the rest run whole.  Every output element against the oracle."""
+    require_cuda()
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("the tile counts are chosen for a 148-SM B200")
+    if block_n != "auto":
+        monkeypatch.setenv("FP8BLK_GEMM_BLOCK_N", block_n)
+    m, n, k = 3200, 1536, 4096
+    ops = _operands(layout, m, n, k, seed=77 + layout)
+    d = _splitk(layout, ops, 4)
+    assert_gemm_close(d.float().cpu().numpy().astype(np.float64), oracle.gemm(layout, *ops),
+                      f"last-round split-K layout {layout} bn={block_n}")
