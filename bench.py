@@ -53,7 +53,7 @@ L2_FLUSH_BYTES = 256 << 20
 # one step; profiles/gemm_dram_layer_16384.md); algorithmic minimum 2.59 GB (codes
 # read once, bf16 outputs written once).  It describes the GEMM source whose
 # SHA-256 prefix is given; for any other source the bench reports no traffic.
-GEMM_STEP_DRAM = {"bytes": 2.882e9, "gemm_cu_sha256": "2558aa53e9cd9ae1"}
+GEMM_STEP_DRAM = {"bytes": 2.884e9, "gemm_cu_sha256": "3c4379681c834dd8"}
 GEMM_SOURCE = os.path.join(ROOT, "fp8_blockwise_scaled_b200", "csrc", "gemm.cu")
 
 WORKLOAD_DESC = {
@@ -249,7 +249,8 @@ class Program:
         fb, torch = self.fb, self.torch
         m, n, k = d.shape[0], d.shape[1], a.shape[1]
         splits = fb.fp8blk_gemm_splitk_count(layout, m, n, k)
-        ws = torch.empty(splits * m * n, dtype=torch.float32, device=d.device) if splits > 1 else None
+        ws = (torch.empty(fb.fp8blk_gemm_splitk_workspace_bytes(layout, m, n, k, splits) // 4, dtype=torch.float32,
+                          device=d.device) if splits > 1 else None)
         self.splits[label] = splits
         self._op(label, "gemm", 2 * m * n * k,
                  lambda: fb.fp8blk_gemm(layout, a, sa, b, sb, d, splits=splits, workspace=ws))

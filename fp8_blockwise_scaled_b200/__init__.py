@@ -157,8 +157,9 @@ def fp8blk_gemm_splitk_count(layout, m: int, n: int, k: int) -> int:
     return int(lib.fp8blk_gemm_splitk_count(int(layout), int(m), int(n), int(k)))
 
 
-def fp8blk_gemm_splitk_workspace_bytes(m: int, n: int, splits: int) -> int:
-    return int(lib.fp8blk_gemm_splitk_workspace_bytes(int(m), int(n), int(splits)))
+def fp8blk_gemm_splitk_workspace_bytes(layout, m: int, n: int, k: int, splits: int) -> int:
+    """Bytes of workspace fp8blk_gemm_splitk needs for this shape and split count on the current device."""
+    return int(lib.fp8blk_gemm_splitk_workspace_bytes(int(layout), int(m), int(n), int(k), int(splits)))
 
 
 def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None, out_dtype=torch.bfloat16, splits=1, workspace=None):
@@ -166,7 +167,7 @@ def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None, out_dtype=torch.bfloa
     out_dtype=torch.float32 or an fp32 d, the unrounded fp32 sums).  splits > 1 (or "auto":
     fp8blk_gemm_splitk_count) divides each output tile's K range among that many units whose
     fp32 partials are summed in split order; workspace: a float32 CUDA tensor of at least
-    splits * M * N elements (allocated here when None)."""
+    fp8blk_gemm_splitk_workspace_bytes(...) bytes (allocated here when None)."""
     dev = _need_cuda(a, sa, b, sb, d)
     m, k = a.shape
     n = b.shape[0]
@@ -195,9 +196,12 @@ def fp8blk_gemm(layout, a, sa, b, sb, d=None, stream=None, out_dtype=torch.bfloa
         _run(dev, lib.fp8blk_gemm, int(layout) | flags, m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d),
              d.stride(0), _stream_handle(stream, dev))
         return d
-    need = splits * m * n
     if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.float32, device=a.device)
+        with torch.cuda.device(dev):
+            need = fp8blk_gemm_splitk_workspace_bytes(layout, m, n, k, splits)
+        if need < 0:
+            raise ValueError("invalid split-K arguments for this device")
+        workspace = torch.empty(max(need // 4, 4), dtype=torch.float32, device=a.device)
     elif workspace.dtype != torch.float32 or not workspace.is_contiguous() or workspace.device != a.device:
         raise ValueError("workspace must be a contiguous float32 tensor on the operands' device")
     _run(dev, lib.fp8blk_gemm_splitk, int(layout) | flags, m, n, k, _ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(d),

@@ -58,7 +58,7 @@ def _load() -> ctypes.CDLL:
         "fp8blk_gemm_tensor_scaled": [I64, I64, I64, P, P, P, P, P, I64, P],
         "fp8blk_gemm": [I, I64, I64, I64, P, P, P, P, P, I64, P],
         "fp8blk_gemm_splitk": [I, I64, I64, I64, P, P, P, P, P, I64, I, P, I64, P],
-        "fp8blk_gemm_splitk_workspace_bytes": [I64, I64, I],
+        "fp8blk_gemm_splitk_workspace_bytes": [I, I64, I64, I64, I],
         "fp8blk_gemm_splitk_count": [I, I64, I64, I64],
         "fp8blk_round_f32_to_bf16": [P, I64, P, P],
         "fp8blk_get_device_error": [P],

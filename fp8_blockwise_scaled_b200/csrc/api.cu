@@ -275,21 +275,31 @@ int fp8blk_gemm_splitk_count(int layout, int64_t M, int64_t N, int64_t K) {
   return fp8blk::choose_splits(g);
 }
 
-int64_t fp8blk_gemm_splitk_workspace_bytes(int64_t M, int64_t N, int splits) {
-  if (M <= 0 || N <= 0 || splits <= 1) return 0;
-  return static_cast<int64_t>(splits) * M * N * 4;
+int64_t fp8blk_gemm_splitk_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int splits) {
+  const int base = layout & ~(FP8BLK_A_E5M2 | FP8BLK_B_E5M2 | FP8BLK_OUT_F32);
+  if (base != FP8BLK_FWD && base != FP8BLK_DGRAD && base != FP8BLK_WGRAD) return -1;
+  if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K) || splits < 1) return -1;
+  if (splits == 1) return 0;
+  if (check_device() != FP8BLK_OK) return -1;
+  fp8blk::GemmArgs g{};
+  g.layout = base;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.splits = splits;
+  if (const char* e = std::getenv("FP8BLK_GEMM_BLOCK_N")) g.block_n = std::atoi(e);
+  return fp8blk::splitk_workspace_bytes(g);
 }
 
 fp8blk_status fp8blk_gemm_splitk(int layout, int64_t M, int64_t N, int64_t K, const uint8_t* a, const float* sa,
                                  const uint8_t* b, const float* sb, void* d, int64_t ldd, int splits,
                                  float* workspace, int64_t workspace_bytes, void* stream) {
-  // The split arguments are checked first (host-only checks), then those of fp8blk_gemm.
+  // The split arguments the host can check alone come first, then those of
+  // fp8blk_gemm, then the workspace size (it depends on the device).
   if (splits < 1 || (K >= 128 && splits > K / 128)) return FP8BLK_ERR_INVALID_ARG;
   if (splits > 1) {
-    if (!workspace || workspace_bytes < fp8blk_gemm_splitk_workspace_bytes(M, N, splits))
-      return FP8BLK_ERR_INVALID_ARG;
+    if (!workspace) return FP8BLK_ERR_INVALID_ARG;
     if (!aligned16(workspace)) return FP8BLK_ERR_ALIGN;
-    if (M * splits >= (int64_t(1) << 31)) return FP8BLK_ERR_SHAPE;   // partial-tile rows are 32-bit
   }
   fp8blk::GemmArgs g;
   const fp8blk_status st = gemm_args(layout, M, N, K, a, sa, b, sb, d, ldd, g);
@@ -297,6 +307,8 @@ fp8blk_status fp8blk_gemm_splitk(int layout, int64_t M, int64_t N, int64_t K, co
   if (splits > 1) {
     g.splits = splits;
     g.workspace = workspace;
+    g.workspace_bytes = workspace_bytes;
+    if (workspace_bytes < fp8blk::splitk_workspace_bytes(g)) return FP8BLK_ERR_INVALID_ARG;
   }
   return launch_status(fp8blk::launch_gemm(g, static_cast<cudaStream_t>(stream)));
 }

@@ -435,12 +435,21 @@ __device__ __forceinline__ Unit unit_coords(int u, int tiles, int num_mb, int nu
 }
 
 // The number of K-blocks of unit u alone (the promotion warps need only that
-// before their K loop; the tile coordinates are derived after it).
+// before their K loop; the tile coordinates are derived after it).  Two
+// equivalent forms: with each, ptxas keeps its tile width's promotion warps
+// within their 208 registers (the other form spills a few bytes there).
+template <int BN>
 __device__ __forceinline__ int unit_kblocks(int u, int tiles, int kblocks, const GemmParams& p) {
-  const int v = u - p.whole_tiles;                    // < 0 for a whole tile
-  const int split = max(v, 0) / max(tiles - p.whole_tiles, 1);
-  const int n = (split + 1) * kblocks / p.splits - split * kblocks / p.splits;
-  return v < 0 ? kblocks : n;
+  if constexpr (BN == 128) {
+    if (u < p.whole_tiles) return kblocks;
+    const int split = (u - p.whole_tiles) / (tiles - p.whole_tiles);
+    return (split + 1) * kblocks / p.splits - split * kblocks / p.splits;
+  } else {
+    const int v = u - p.whole_tiles;                  // < 0 for a whole tile
+    const int split = max(v, 0) / max(tiles - p.whole_tiles, 1);
+    const int n = (split + 1) * kblocks / p.splits - split * kblocks / p.splits;
+    return v < 0 ? kblocks : n;
+  }
 }
 
 
@@ -657,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = blockIdx.x; u < units; u += gridDim.x) {
         // The unit's coordinates are derived after the K loop, so that only u
         // stays live across it.
-        if (!promote_tile<BN, kWgrad>(ctrl, p, acc, unit_kblocks(u, tiles, kblocks, p), tmem_lanes, row, col0, tbuf,
+        if (!promote_tile<BN, kWgrad>(ctrl, p, acc, unit_kblocks<BN>(u, tiles, kblocks, p), tmem_lanes, row, col0, tbuf,
                                       sring, abort, lane, release))
           break;
         // A whole tile goes to d (bf16, or fp32 with out_f32); a split unit's
@@ -983,6 +992,23 @@ int num_sms() {
   return (e == cudaSuccess && sms > 0) ? sms : 1;
 }
 
+// Tiles of a launch that run whole: all of them without a split; with one,
+// none when there are fewer tiles than SMs, else all but the last, partial
+// round of the SMs (tiles mod SMs).  The SM count, not a CTA cap, decides, so
+// that the split tiles (and the workspace they need) depend on the shape, the
+// split count and the device alone.
+int64_t whole_tiles(int64_t tiles, int splits) {
+  if (splits <= 1) return tiles;
+  const int64_t sms = num_sms();
+  return tiles < sms ? 0 : tiles - tiles % sms;
+}
+
+int64_t gemm_ctas(const GemmArgs& g) {
+  int64_t ctas = num_sms();
+  if (g.max_ctas > 0 && g.max_ctas < ctas) ctas = g.max_ctas;
+  return ctas;
+}
+
 // Opts a kernel into `bytes` of dynamic shared memory, once per context.
 template <typename Kernel>
 cudaError_t set_smem_once(PerContext<int>& cache, Kernel kernel, int bytes) {
@@ -1008,15 +1034,15 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   int group_m = g.group_m > 0 ? g.group_m : (num_mb <= 16 ? num_mb : 8);
   if (group_m > num_mb) group_m = num_mb;
   const int64_t tiles = (g.M / BM) * (g.N / BN);
-  int64_t ctas = num_sms();
-  if (g.max_ctas > 0 && g.max_ctas < ctas) ctas = g.max_ctas;
-  // Split-K: with fewer tiles than CTAs every tile is split; otherwise the
-  // tiles of the last, partial round (tiles % CTAs of them) are, so that their
+  const int64_t ctas = gemm_ctas(g);
+  // Split-K: with fewer tiles than SMs every tile is split; otherwise the
+  // tiles of the last, partial round (tiles % SMs of them) are, so that their
   // units fill that round.  Split units write fp32 partial tiles to the
   // workspace; gemm_splitk_sum_kernel adds them in split order afterwards.
   int splits = g.splits > 1 ? g.splits : 1;
-  const int64_t whole = splits == 1 ? tiles : (tiles < ctas ? 0 : tiles - tiles % ctas);
+  const int64_t whole = whole_tiles(tiles, splits);
   if (whole == tiles) splits = 1;
+  if (splits > 1 && g.workspace_bytes < (tiles - whole) * splits * BM * BN * 4) return cudaErrorInvalidValue;
   GemmParams p{g.M, g.N, g.K, g.sa, g.sb, g.d, g.ldd, g.out_f32, g.timeout_ns, g.err, g.inject_stall, group_m,
                fmt_bits(g), g.tensor_sa, g.tensor_sb, splits, static_cast<int>(whole), g.workspace};
   const int64_t units = whole + (tiles - whole) * splits;
@@ -1095,6 +1121,14 @@ int choose_block_n(const GemmArgs& g) {
 
 }  // namespace
 
+int64_t splitk_workspace_bytes(const GemmArgs& g) {
+  if (g.splits <= 1) return 0;
+  const int bn = choose_block_n(g);
+  const int64_t tiles = (g.M / BM) * (g.N / bn);
+  const int64_t split_tiles = tiles - whole_tiles(tiles, g.splits);
+  return split_tiles * g.splits * BM * bn * 4;
+}
+
 int choose_splits(const GemmArgs& g) {
   const int64_t tiles = (g.M / BM) * (g.N / choose_block_n(g));
   const int64_t kblocks = g.K / BK;
@@ -1123,8 +1157,7 @@ int choose_splits(const GemmArgs& g) {
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   const bool wgrad = g.layout == 2;
-  if (g.splits > 1 && (g.tensor_sa || !g.workspace || g.K / BK < g.splits || g.M * g.splits >= (int64_t{1} << 31)))
-    return cudaErrorInvalidValue;
+  if (g.splits > 1 && (g.tensor_sa || !g.workspace || g.K / BK < g.splits)) return cudaErrorInvalidValue;
   // Pair tiles (256 x 256 over two SMs) only on request, when the shape allows them (never split).
   if (g.pair > 0 && g.splits <= 1 && g.block_n == 0 && !g.tensor_sa && g.M % 256 == 0 && g.N % 256 == 0)
     return wgrad ? launch_pair<true>(g, stream) : launch_pair<false>(g, stream);

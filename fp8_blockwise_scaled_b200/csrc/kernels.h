@@ -85,7 +85,8 @@ struct GemmArgs {
   const float* tensor_sb;
   unsigned int* err;          // device error word
   int splits;                 // > 1: split-K over that many units per split tile (1-CTA kernel)
-  float* workspace;           // split-K: at least splits * M * N floats of partial tiles
+  float* workspace;           // split-K: fp32 partial tiles (splitk_workspace_bytes)
+  int64_t workspace_bytes;
 };
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream);
@@ -93,6 +94,10 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t stream);
 // The split count launch_gemm would use well for this shape on the current
 // device (1 when the output tiles already fill the SMs' waves).
 int choose_splits(const GemmArgs& g);
+
+// Bytes of fp32 partial tiles launch_gemm writes for g.splits on the current
+// device (tile width and SM count as the launch will use them).
+int64_t splitk_workspace_bytes(const GemmArgs& g);
 
 
 // y[i] = bf16_round_nearest_even(x[i]) for i < n (x, y 16-byte aligned).

@@ -212,8 +212,8 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K,
  * The same GEMM with split-K, for shapes whose output tiles leave SMs idle:
  * with fewer tiles than SMs (the weight gradient of a narrow layer: few
  * tiles, long K) every tile is split; with more, the tiles of the last,
- * partial round of the persistent CTAs (tiles mod SMs of them) are, so that
- * their units fill that round.  The K-blocks of a split tile are divided among
+ * partial round of the SMs (tiles mod SMs of them) are, so that their units
+ * fill that round.  The K-blocks of a split tile are divided among
  * `splits` work units; unit s sums its contiguous range of K-blocks (the same
  * per-K-block promotion as fp8blk_gemm) into an fp32 partial tile in
  * `workspace`, and a second kernel adds the partials in the order s = 0, 1,
@@ -222,21 +222,27 @@ fp8blk_status fp8blk_gemm(int layout, int64_t M, int64_t N, int64_t K,
  * fp8blk_gemm's only by the order of the fp32 additions in the split tiles.
  *   splits      1 .. K/128; 1 runs fp8blk_gemm (workspace unused).
  *   workspace   device memory of at least
- *               fp8blk_gemm_splitk_workspace_bytes(M, N, splits) bytes, 16-byte
+ *               fp8blk_gemm_splitk_workspace_bytes(layout, M, N, K, splits) bytes, 16-byte
  *               aligned, owned by the caller; overwritten; it must not overlap
  *               any operand or d, and must stay untouched until the call's
  *               kernels have run (stream order).
  * Errors as fp8blk_gemm; FP8BLK_ERR_INVALID_ARG for a split count out of
  * range or a missing or short workspace, FP8BLK_ERR_ALIGN for an unaligned
- * workspace, FP8BLK_ERR_SHAPE when M * splits >= 2^31.
+ * workspace (its size is checked after fp8blk_gemm's checks, on the device).
  */
 fp8blk_status fp8blk_gemm_splitk(int layout, int64_t M, int64_t N, int64_t K,
                                  const uint8_t* a, const float* sa, const uint8_t* b, const float* sb,
                                  void* d, int64_t ldd, int splits, float* workspace,
                                  int64_t workspace_bytes, void* stream);
 
-/* Bytes of split-K workspace for an M x N output: splits * M * N * 4 (0 when splits <= 1). */
-int64_t fp8blk_gemm_splitk_workspace_bytes(int64_t M, int64_t N, int splits);
+/*
+ * Bytes of split-K workspace fp8blk_gemm_splitk needs for this GEMM and split
+ * count on the current device: (split tiles) x splits x 128 x (tile width) x 4
+ * (the split tiles: all of them with fewer tiles than SMs, else the last
+ * round's tiles mod SMs; never more than splits * M * N * 4).  0 when splits == 1, -1 for an invalid
+ * layout, shape or split count or an unsupported device.
+ */
+int64_t fp8blk_gemm_splitk_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int splits);
 
 /*
  * The split count the library uses well for this GEMM shape on the current

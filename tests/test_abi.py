@@ -142,14 +142,14 @@ def test_gemm_splitk_argument_errors():
     L = _lib.lib
     A = ALIGNED
     base = (2, 256, 256, 2048, A, A, A, A, A, 256)                  # WGRAD, 16 K-blocks
-    ws = L.fp8blk_gemm_splitk_workspace_bytes(256, 256, 3)
-    assert ws == 3 * 256 * 256 * 4
-    assert L.fp8blk_gemm_splitk_workspace_bytes(256, 256, 1) == 0
-    assert L.fp8blk_gemm_splitk_workspace_bytes(0, 256, 3) == 0
+    ws = 3 * 256 * 256 * 4
+    assert L.fp8blk_gemm_splitk_workspace_bytes(2, 256, 256, 2048, 1) == 0
+    assert L.fp8blk_gemm_splitk_workspace_bytes(2, 0, 256, 2048, 3) == -1
+    assert L.fp8blk_gemm_splitk_workspace_bytes(3, 256, 256, 2048, 3) == -1
+    assert L.fp8blk_gemm_splitk_workspace_bytes(2, 256, 256, 2048, 0) == -1
     assert L.fp8blk_gemm_splitk(*base, 0, A, ws, S) == 1            # splits < 1
     assert L.fp8blk_gemm_splitk(*base, 17, A, 1 << 40, S) == 1      # more splits than K-blocks
     assert L.fp8blk_gemm_splitk(*base, 3, NULL, ws, S) == 1         # no workspace
-    assert L.fp8blk_gemm_splitk(*base, 3, A, ws - 4, S) == 1        # short workspace
     assert L.fp8blk_gemm_splitk(*base, 3, MISALIGNED, ws, S) == 3   # unaligned workspace
     bad_layout = (3,) + base[1:]
     assert L.fp8blk_gemm_splitk(*bad_layout, 3, A, ws, S) == 1      # then fp8blk_gemm's own checks
@@ -171,6 +171,7 @@ def test_valid_call_without_a_gpu_reports_a_cuda_error():
     st = _lib.lib.fp8blk_quantize_act_1x128(ALIGNED, 128, 128, 128, 1, ALIGNED, ALIGNED, NULL, NULL, S)
     assert st in (4, 7)
     assert _lib.lib.fp8blk_gemm_splitk_count(2, 2048, 1536, 16384) == 0     # no device: no answer
+    assert _lib.lib.fp8blk_gemm_splitk_workspace_bytes(2, 2048, 1536, 16384, 3) == -1
 
 
 def test_delayed_scaling_argument_errors():

@@ -152,3 +152,44 @@ def test_splitk_of_the_last_round(layout, block_n, monkeypatch):
     d = _splitk(layout, ops, 4)
     assert_gemm_close(d.float().cpu().numpy().astype(np.float64), oracle.gemm(layout, *ops),
                       f"last-round split-K layout {layout} bn={block_n}")
+
+
+def test_splitk_workspace_bytes_and_a_short_workspace():
+    """The library's workspace size is exactly the split tiles' partials; one byte less is refused."""
+    require_cuda()
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("the tile counts are chosen for a 148-SM B200")
+    assert fb.fp8blk_gemm_splitk_workspace_bytes(fb.WGRAD, 2048, 1536, 16384, 3) == 96 * 3 * 128 * 256 * 4
+    assert fb.fp8blk_gemm_splitk_workspace_bytes(fb.DGRAD, 16384, 1536, 17920, 5) == 28 * 5 * 128 * 256 * 4
+    ops = _operands(oracle.WGRAD, 256, 512, 2048, seed=9)
+    qa, sa, qb, sb = ops
+    need = fb.fp8blk_gemm_splitk_workspace_bytes(fb.WGRAD, 256, 512, 2048, 3)
+    assert need == 4 * 3 * 128 * 256 * 4                             # 2 x 2 tiles of 128 x 256, all split
+    short = torch.empty(need // 4 - 1, dtype=torch.float32, device="cuda")
+    with pytest.raises(fb.Fp8BlkError):
+        fb.fp8blk_gemm_splitk(oracle.WGRAD, _dev_codes(qa), _dev_f32(sa), _dev_codes(qb), _dev_f32(sb), 3,
+                              workspace=short)
+    exact = torch.empty(need // 4, dtype=torch.float32, device="cuda")
+    d = fb.fp8blk_gemm_splitk(oracle.WGRAD, _dev_codes(qa), _dev_f32(sa), _dev_codes(qb), _dev_f32(sb), 3,
+                              workspace=exact)
+    assert fb.fp8blk_get_device_error() == 0
+    assert_gemm_close(d.float().cpu().numpy().astype(np.float64), oracle.gemm(oracle.WGRAD, *ops), "exact workspace")
+
+
+def test_splitk_under_a_cta_cap(monkeypatch):
+    """With the GEMM grid capped below the SM count (the SM-partitioned step), the split tiles and the
+    workspace size stay those of the device's SM count; the result still matches the oracle."""
+    require_cuda()
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("the tile counts are chosen for a 148-SM B200")
+    m, n, k = 3200, 1536, 4096                       # 150 tiles of 128 x 256: 2 split tiles
+    need = fb.fp8blk_gemm_splitk_workspace_bytes(fb.FWD, m, n, k, 4)
+    assert need == 2 * 4 * 128 * 256 * 4
+    monkeypatch.setenv("FP8BLK_GEMM_MAX_CTAS", "100")
+    assert fb.fp8blk_gemm_splitk_workspace_bytes(fb.FWD, m, n, k, 4) == need
+    ops = _operands(oracle.FWD, m, n, k, seed=12)
+    qa, sa, qb, sb = ops
+    ws = torch.empty(need // 4, dtype=torch.float32, device="cuda")
+    d = fb.fp8blk_gemm_splitk(oracle.FWD, _dev_codes(qa), _dev_f32(sa), _dev_codes(qb), _dev_f32(sb), 4, workspace=ws)
+    assert fb.fp8blk_get_device_error() == 0
+    assert_gemm_close(d.float().cpu().numpy().astype(np.float64), oracle.gemm(oracle.FWD, *ops), "split-K, 100 CTAs")
