@@ -682,7 +682,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     h_out = [[(d, torch.empty(d.shape, dtype=d.dtype, pin_memory=True)) for d in p.outputs] for p in progs]
     h2d = sum(h.numel() * h.element_size() for _, h in h_in[0])
     d2h = sum(h.numel() * h.element_size() for _, h in h_out[0])
-    e2e_steps = max(3, min(args.steps, 10))
+    e2e_steps = max(3, args.steps)                   # the same steps as the device-timed value
     progs[1].run()                                   # set-up of the second buffer set, outside the timing
     copy_in, copy_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     barrier()
