@@ -36,13 +36,18 @@
 //               f32x2 FMAs:
 //                   FWD/DGRAD: acc += P * (sa[m] * sb[n-block])
 //                   WGRAD    : acc += (P * sb[n]) * sa[m]
-//               after the last K-block it rounds the tile to bf16 and stores
-//               it with 32-byte vector stores.
+//               after the last K-block it rounds its slice of the tile to
+//               bf16 into a shared-memory staging area and one lane issues
+//               TMA stores of it, which drain while the warp goes on to the
+//               next tile (BN = 128 tiles, fp32 outputs and split-K partial
+//               tiles leave by 32-byte vector stores).
 // Waits on the critical path (MMA issuer, promotion) poll without a
 // suspend-time hint; the producers, which run ahead, sleep in theirs.
 //
 // gemm_blockwise_kernel: one CTA per SM, 128 x BN tiles (BN = 256 or 128),
-// double-buffered TMEM (2 x 256 or 4 x 128 columns).
+// double-buffered TMEM (2 x 256 or 4 x 128 columns); BN = 256: 3 operand
+// stages beside the 64 KB bf16 staging area of the epilogue, BN = 128: 6
+// stages and the bf16 tile stored from registers.
 // gemm_pair_kernel: a cluster of two CTAs computes a 256 x 256 tile with
 // tcgen05.mma.cta_group::2 (M = 256): each CTA loads its own 128 A rows and
 // half of the 256 B rows, so a K-block moves 32 KB into each SM instead of
@@ -85,7 +90,13 @@ static_assert(kLowRegs % 8 == 0 && kHighRegs % 8 == 0, "setmaxnreg takes multipl
 
 template <int BN>
 struct Cfg {
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  // BN = 256 stages its bf16 tile in shared memory for TMA stores and keeps
+  // 3 operand stages beside it (measured on the layer's GEMMs, a fourth stage
+  // gains less than the staged epilogue does); BN = 128 stores from registers
+  // and keeps 6.
+  static constexpr bool kStagedOut = BN == 256;
+  static constexpr int kStages = kStagedOut ? 3 : 6;
+  static constexpr int kOutBytes = kStagedOut ? BM * BN * 2 : 0;
   static constexpr int kABytes = BM * BK;
   static constexpr int kBBytes = BN * BK;
   static constexpr int kStageBytes = kABytes + kBBytes;
@@ -117,8 +128,9 @@ static_assert(offsetof(Ctrl, slots) % 16 == 0, "scale slots are filled with 16-b
 
 template <int BN>
 constexpr int smem_bytes() {
-  return 1024 + Cfg<BN>::kStages * Cfg<BN>::kStageBytes + static_cast<int>(sizeof(Ctrl));
+  return 1024 + Cfg<BN>::kStages * Cfg<BN>::kStageBytes + Cfg<BN>::kOutBytes + static_cast<int>(sizeof(Ctrl));
 }
+static_assert(smem_bytes<256>() <= 227 * 1024 && smem_bytes<128>() <= 227 * 1024, "shared memory per CTA");
 
 struct GemmParams {
   int64_t M, N, K;
@@ -380,7 +392,7 @@ __device__ __forceinline__ void scale_feed(Ctrl* ctrl, const GemmParams& p, int 
       if (lane == 0) {
         // The promotion warps read this slot through the generic proxy; the
         // bulk copies below write it through the async proxy: order them.
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        fence_proxy_async_shared();
         constexpr uint32_t kBytes = BM * 4 + (kWgrad ? BN * 4 : 0);
         mbar_arrive_expect_tx(&ctrl->sfull[ring.idx], kBytes);   // releases the sb stores above
         bulk_load(ss.sa, p.sa + static_cast<int64_t>(kb) * p.M + m0, BM * 4, &ctrl->sfull[ring.idx]);
@@ -459,12 +471,13 @@ __device__ __forceinline__ int unit_kblocks(int u, int tiles, int kblocks, const
 template <int BN, bool kWgrad, bool kTensor = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_blockwise_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                          const GemmParams p) {
+                          const __grid_constant__ CUtensorMap tm_d, const GemmParams p) {
   using C = Cfg<BN>;
   constexpr int kCols = BN / 2;   // columns per promotion warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + C::kStages * C::kStageBytes);
+  uint8_t* smem_out = smem + C::kStages * C::kStageBytes;   // epilogue staging, 1024-byte aligned
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem_out + C::kOutBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -658,6 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       Ring<kSRing> sring;
       float2 acc[BN / 4];
+      bool staged = false;   // this warp's staging area holds a tile whose stores may still be reading it
       auto release = [&](int b) {
         tc_fence_before_sync();
         __syncwarp();
@@ -675,10 +689,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool part = w.slot >= 0;
         const int64_t off = part ? static_cast<int64_t>(w.slot * BM + row) * BN + col0
                                  : static_cast<int64_t>(w.mb * BM + row) * p.ldd + static_cast<int64_t>(w.nb) * BN + col0;
-        if (part || p.out_f32)
+        if (part || p.out_f32) {
           store_row_f32<kCols>((part ? p.partials : static_cast<float*>(p.d)) + off, acc);
-        else
+        } else if constexpr (!C::kStagedOut) {
           store_row_bf16<kCols>(static_cast<uint16_t*>(p.d) + off, acc);
+        } else {
+          // bf16: the warp's 32 rows x kCols columns go to its slice of the
+          // staging area as kCols / 64 boxes of 32 x 64 in the 128-byte
+          // swizzle that the output map names (16-byte chunk j of row r at
+          // chunk j ^ (r % 8): the eight rows of a 128-byte bank line spread
+          // over all banks), then one lane stores the boxes with TMA.
+          uint8_t* stg = smem_out + ew * (32 * kCols * 2);
+          if (staged) {
+            if (lane == 0) bulk_wait_group_read0();   // the previous tile's stores have read it
+            __syncwarp();
+          }
+#pragma unroll
+          for (int b = 0; b < kCols / 64; ++b) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float2* a = acc + b * 32 + j * 4;   // columns 64 b + 8 j .. + 7
+              *reinterpret_cast<uint4*>(stg + b * 4096 + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                  make_uint4(pack_bf16x2(a[0].x, a[0].y), pack_bf16x2(a[1].x, a[1].y), pack_bf16x2(a[2].x, a[2].y),
+                             pack_bf16x2(a[3].x, a[3].y));
+            }
+          }
+          fence_proxy_async_shared();                   // the writes above, then the TMA's reads
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int b = 0; b < kCols / 64; ++b)
+              tma_store_2d(&tm_d, stg + b * 4096, w.nb * BN + col0 + b * 64, w.mb * BM + quarter * 32);
+            bulk_commit_group();
+          }
+          staged = true;
+        }
+      }
+      // The stores in flight complete before the CTA (and its shared memory) goes.
+      if constexpr (C::kStagedOut) {
+        if (lane == 0) bulk_wait_group0();
       }
     }
   }
@@ -974,6 +1023,22 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, in
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Map of the output for the TMA-store epilogue: bf16 [rows][ld], boxes of 32
+// rows x 64 columns (128 bytes) in the 128-byte swizzle.  An fp32 output
+// leaves by plain stores; its map (the same extent read as bf16, the fp32 row
+// pitch) is never used.
+bool make_out_map(CUtensorMap* map, void* base, int64_t rows, int64_t cols, int64_t ld, bool f32) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * (f32 ? 4 : 2))};
+  const cuuint32_t box[2] = {64, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Instruction-descriptor bits of the operand formats (kind::f8f6f4: E4M3 = 0, E5M2 = 1).
 uint32_t fmt_bits(const GemmArgs& g) {
   return (static_cast<uint32_t>(g.a_e5m2 != 0) << 7) | (static_cast<uint32_t>(g.b_e5m2 != 0) << 10);
@@ -1025,8 +1090,10 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   constexpr int kSmem = smem_bytes<BN>();
   if (cudaError_t e = set_smem_once(smem_set, gemm_blockwise_kernel<BN, kWgrad, kTensor>, kSmem); e != cudaSuccess)
     return e;
-  CUtensorMap ta, tb;
-  if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BN)) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb, td;
+  if (!make_map(&ta, g.a, g.M, g.K, BM) || !make_map(&tb, g.b, g.N, g.K, BN) ||
+      !make_out_map(&td, g.d, g.M, g.N, g.ldd, g.out_f32 != 0))
+    return cudaErrorInvalidValue;
   // Tile order: groups of 8 M-blocks; with at most 16 M-blocks (the weight
   // gradients of the narrow layers, M = out features) one group holds them
   // all, so every B column block is streamed once while all M-blocks use it.
@@ -1055,7 +1122,7 @@ cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   cudaLaunchAttribute attr[1];
   cfg.numAttrs = set_pdl_attr(attr, g.pdl);
   cfg.attrs = attr;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<BN, kWgrad, kTensor>, ta, tb, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<BN, kWgrad, kTensor>, ta, tb, td, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || splits == 1) return e;
   const SplitSum q{static_cast<int>(whole), splits, num_mb, static_cast<int>(g.N / BN), group_m, g.d, g.ldd};
