@@ -46,8 +46,8 @@
 //
 // gemm_blockwise_kernel: one CTA per SM, 128 x BN tiles (BN = 256 or 128),
 // double-buffered TMEM (2 x 256 or 4 x 128 columns); BN = 256: 3 operand
-// stages beside the 64 KB bf16 staging area of the epilogue, BN = 128: 6
-// stages and the bf16 tile stored from registers.
+// stages beside the 64 KB bf16 staging area of the epilogue, BN = 128 and the
+// one-scale variant: 6 / 4 stages and the bf16 tile stored from registers.
 // gemm_pair_kernel: a cluster of two CTAs computes a 256 x 256 tile with
 // tcgen05.mma.cta_group::2 (M = 256): each CTA loads its own 128 A rows and
 // half of the 256 B rows, so a K-block moves 32 KB into each SM instead of
@@ -88,14 +88,17 @@ constexpr int kHighRegs = 208;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * 168, "register split exceeds the launch allocation");
 static_assert(kLowRegs % 8 == 0 && kHighRegs % 8 == 0, "setmaxnreg takes multiples of 8");
 
-template <int BN>
+// kTensor: the one-scale-per-operand variant (no per-K-block promotion).
+template <int BN, bool kTensor = false>
 struct Cfg {
-  // BN = 256 stages its bf16 tile in shared memory for TMA stores and keeps
-  // 3 operand stages beside it (measured on the layer's GEMMs, a fourth stage
-  // gains less than the staged epilogue does); BN = 128 stores from registers
-  // and keeps 6.
-  static constexpr bool kStagedOut = BN == 256;
-  static constexpr int kStages = kStagedOut ? 3 : 6;
+  // The blockwise kernel with BN = 256 stages its bf16 tile in shared memory
+  // for TMA stores and keeps 3 operand stages beside it (measured on the
+  // layer's GEMMs, a fourth stage gains less than the staged epilogue does).
+  // BN = 128 stores from registers and keeps 6 stages; so does the
+  // one-scale variant with 4 (its K loop, with no promotion, runs ahead of 3
+  // stages: measured 10% slower with the staged epilogue).
+  static constexpr bool kStagedOut = BN == 256 && !kTensor;
+  static constexpr int kStages = kStagedOut ? 3 : (BN == 256 ? 4 : 6);
   static constexpr int kOutBytes = kStagedOut ? BM * BN * 2 : 0;
   static constexpr int kABytes = BM * BK;
   static constexpr int kBBytes = BN * BK;
@@ -126,11 +129,14 @@ struct Ctrl {
 };
 static_assert(offsetof(Ctrl, slots) % 16 == 0, "scale slots are filled with 16-byte copies");
 
-template <int BN>
+template <int BN, bool kTensor>
 constexpr int smem_bytes() {
-  return 1024 + Cfg<BN>::kStages * Cfg<BN>::kStageBytes + Cfg<BN>::kOutBytes + static_cast<int>(sizeof(Ctrl));
+  using C = Cfg<BN, kTensor>;
+  return 1024 + C::kStages * C::kStageBytes + C::kOutBytes + static_cast<int>(sizeof(Ctrl));
 }
-static_assert(smem_bytes<256>() <= 227 * 1024 && smem_bytes<128>() <= 227 * 1024, "shared memory per CTA");
+static_assert(smem_bytes<256, false>() <= 227 * 1024 && smem_bytes<128, false>() <= 227 * 1024 &&
+                  smem_bytes<256, true>() <= 227 * 1024 && smem_bytes<128, true>() <= 227 * 1024,
+              "shared memory per CTA");
 
 struct GemmParams {
   int64_t M, N, K;
@@ -472,7 +478,7 @@ template <int BN, bool kWgrad, bool kTensor = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_blockwise_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const __grid_constant__ CUtensorMap tm_d, const GemmParams p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, kTensor>;
   constexpr int kCols = BN / 2;   // columns per promotion warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1087,7 +1093,7 @@ cudaError_t set_smem_once(PerContext<int>& cache, Kernel kernel, int bytes) {
 template <int BN, bool kWgrad, bool kTensor = false>
 cudaError_t launch_variant(const GemmArgs& g, cudaStream_t stream) {
   static PerContext<int> smem_set;
-  constexpr int kSmem = smem_bytes<BN>();
+  constexpr int kSmem = smem_bytes<BN, kTensor>();
   if (cudaError_t e = set_smem_once(smem_set, gemm_blockwise_kernel<BN, kWgrad, kTensor>, kSmem); e != cudaSuccess)
     return e;
   CUtensorMap ta, tb, td;

@@ -86,6 +86,27 @@ def test_gemm_tensor_scaled_small(m, n, k):
     assert_gemm_close(got, ref, f"tensor-scaled {m}x{n}x{k}")
 
 
+def test_gemm_tensor_scaled_wide_tiles_with_row_pitch():
+    """A shape on which the library picks 256-column tiles (1024 x 4096: 128 tiles of 128 x 256
+    fill the SMs as well as 256 of 128 x 128), whose bf16 epilogue stores through a tensor map:
+    every element against the oracle, written into a wider buffer whose padding stays untouched."""
+    require_cuda()
+    m, n, k = 1024, 4096, 512
+    xa, wb = _x(m, k, 11, 1.0), _x(n, k, 12, 0.02)
+    sa = oracle.tensor_scale(np.abs(workloads.bf16_to_f32(xa)).max())
+    sb = oracle.tensor_scale(np.abs(workloads.bf16_to_f32(wb)).max())
+    qa, qb = oracle.quantize_tensor(xa, sa), oracle.quantize_tensor(wb, sb)
+    dev = lambda a: torch.from_numpy(a).cuda().view(torch.float8_e4m3fn)  # noqa: E731
+    sc = lambda v: torch.tensor([v], dtype=torch.float32, device="cuda")  # noqa: E731
+    wide = torch.full((m, n + 256), -3.0, dtype=torch.bfloat16, device="cuda")
+    fb.fp8blk_gemm_tensor_scaled(dev(qa), sc(sa), dev(qb), sc(sb), d=wide[:, :n])
+    torch.cuda.synchronize()
+    assert fb.fp8blk_get_device_error() == 0
+    assert bool((wide[:, n:] == -3.0).all()), "padding columns written"
+    ref = oracle.gemm_tensor(qa, sa, qb, sb)
+    assert_gemm_close(wide[:, :n].float().cpu().numpy().astype(np.float64), ref, "tensor-scaled 1024x4096x512 pitched")
+
+
 def test_gemm_tensor_scaled_full_size():
     require_cuda()
     rows = np.sort(np.random.default_rng(5).choice(8192, 16, replace=False))

@@ -144,3 +144,29 @@ def test_both_kernels(m, n, k, layout, pair, monkeypatch):
         b_src = workloads.weight(rng, n, k)
     got, ref = _run(layout, *_operands(layout, a_src, b_src))
     assert_gemm_close(got, ref, f"layout {layout} {m}x{n}x{k} pair={pair}")
+
+
+@pytest.mark.parametrize("layout", [oracle.FWD, oracle.WGRAD])
+@pytest.mark.parametrize("block_n", ["128", "256"])
+def test_output_with_row_pitch(layout, block_n, monkeypatch):
+    """D written into the first N columns of a wider buffer (row pitch ldd = N + 128): every
+    element against the oracle, and the 128 padding columns of every row untouched (the bf16
+    epilogue of BN = 256 tiles stores through a tensor map whose pitch is ldd)."""
+    require_cuda()
+    monkeypatch.setenv("FP8BLK_GEMM_BLOCK_N", block_n)
+    m, n, k = 768, 512, 640
+    rng = np.random.default_rng(91 + int(block_n) + layout)
+    if layout == oracle.FWD:
+        x, w = workloads.activation_with_outliers(rng, m, k, frac=0.01), workloads.weight(rng, n, k)
+    else:                                  # WGRAD: dY [T=k, out=m], X [T=k, in=n]
+        x, w = workloads.grad_output(rng, k, m), workloads.swiglu_like(rng, k, n)
+    qa, sa, qb, sb = _operands(layout, x, w)
+    wide = torch.full((m, n + 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    d = fb.fp8blk_gemm(layout, _dev_u8(qa), _dev_f32(sa), _dev_u8(qb), _dev_f32(sb), d=wide[:, :n])
+    torch.cuda.synchronize()
+    assert fb.fp8blk_get_device_error() == 0
+    assert d.data_ptr() == wide.data_ptr() and d.stride(0) == n + 128
+    assert bool((wide[:, n:] == 7.0).all()), "padding columns written"
+    ref = oracle.gemm(layout, qa, sa, qb, sb)
+    assert_gemm_close(wide[:, :n].float().cpu().numpy().astype(np.float64), ref,
+                      f"layout {layout} bn={block_n} with row pitch")
